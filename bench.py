@@ -1,0 +1,326 @@
+"""Throughput of the matched Siddon projector pair on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload I] [--impl ours|reference]
+
+A step is one forward projection and one back projection of the workload
+(default: parallel beam, 512^3 volume, 900 views, 512x736 detector), inputs
+resident in HBM.  value = (forward updates + back updates) / step time, in
+Gupdates/s (ray-voxel updates), summed over ranks; with N > 1 every rank runs
+its own copy of the workload (independent problems, weak scaling, no
+collective on the data path).  Rank 0 prints one JSON line.
+
+--impl reference times the FP64 CPU oracle on a bounded sample of the same
+workload (the reference arm; slow by design).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "fwd & adjoint Gupdates/s (ray-voxel) and achieved HBM GB/s vs roofline, 1 B200"
+UNIT = "Gupdates/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload_config(wl):
+    g = wl.geom
+    beam = "parallel" if g.beam == 0 else ("helical cone" if np.ptp(g.src[:, 2]) > 0 else "circular cone")
+    det = "flat" if g.detector == 0 else "cylindrical"
+    return {"workload": wl.name, "index": wl.index, "beam": beam, "detector": det,
+            "volume_zyx": [g.nz, g.ny, g.nx], "n_views": g.n_views, "detector_rows_cols": [g.n_rows, g.n_cols],
+            "seed": wl.seed, "l2": "inputs larger than L2 (volume and sinogram each > 126 MB)"}
+
+
+def algorithmic_bytes(U, n_vox, n_rays):
+    """4 B per ray-voxel update (one FP32 voxel read or accumulation) plus the
+    compulsory read/write of every voxel and every sinogram element once."""
+    return 4.0 * U + 4.0 * n_vox + 4.0 * n_rays
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"ctp_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_oracle_sample(wl, n_views_sample=1):
+    """FP64 oracle forward + back over an evenly spaced subset of views, on one
+    host core.  Returns (updates/s, seconds, updates, description)."""
+    import oracle
+    g = wl.geom
+    views = np.linspace(0, g.n_views - 1, n_views_sample).round().astype(np.int64)
+    gs = g.subset_views(views)
+    vol = np.random.default_rng(wl.seed).random(g.vol_shape, dtype=np.float32)
+    sino = np.random.default_rng(wl.seed + 1).random(gs.sino_shape, dtype=np.float32)
+    U = oracle.count_updates(gs)
+    t0 = time.perf_counter()
+    oracle.forward(gs, vol)
+    oracle.back(gs, sino)
+    dt = time.perf_counter() - t0
+    desc = (f"FP64 oracle forward + back of {n_views_sample} of {g.n_views} views (evenly spaced) of workload "
+            f"{wl.index}, {2 * U} updates, one host thread")
+    return 2 * U / dt, dt, 2 * U, desc
+
+
+def run_reference(args, rank, world):
+    from ray_forward_back_b200 import workloads as W
+    if rank != 0:
+        return 0
+    wl = W.workload(args.workload)
+    vals = []
+    for _ in range(args.warmup):
+        cpu_oracle_sample(wl, 1)
+    desc = ""
+    for _ in range(args.steps):
+        v, dt, U, desc = cpu_oracle_sample(wl, 1)
+        vals.append(v / 1e9)
+    value = float(np.median(vals))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(wl),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from ray_forward_back_b200 import ctp
+    from ray_forward_back_b200 import workloads as W
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = W.workload(args.workload)
+    g = wl.geom
+    P = ctp.Projector(g, device=local_rank)
+    info = P.info()
+    stream = torch.cuda.Stream(device=dev)
+    vol_host = wl.phantom()
+    with torch.cuda.stream(stream):
+        vol = torch.from_numpy(vol_host).to(dev)
+        sino_in = torch.from_numpy(wl.sinogram()).to(dev)
+        sino_out = torch.empty(g.sino_shape, dtype=torch.float32, device=dev)
+        vol_out = torch.empty(g.vol_shape, dtype=torch.float32, device=dev)
+    stream.synchronize()
+    U = P.count_updates(stream=stream)
+
+    def step():
+        P.forward(vol, out=sino_out, stream=stream)
+        P.back(sino_in, out=vol_out, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    stream.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = ClockSampler(local_rank)
+    if rank == 0:
+        clocks.start()
+        time.sleep(0.3)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for k in range(args.steps):
+        e0, e1, e2 = ev[k]
+        e0.record(stream)
+        P.forward(vol, out=sino_out, stream=stream)
+        e1.record(stream)
+        P.back(sino_in, out=vol_out, stream=stream)
+        e2.record(stream)
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop() if rank == 0 else None
+    total_ms = start.elapsed_time(end)
+    fwd_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(args.steps)]
+    back_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(args.steps)]
+    t = torch.tensor([total_ms, float(np.mean(fwd_ms)), float(np.mean(back_ms))], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, fwd_avg, back_avg = t.tolist()
+    ms_per_step = total_ms / args.steps
+    value = world * 2 * U / (ms_per_step * 1e-3) / 1e9
+
+    # end to end through the public API with host buffers (pinned), every step
+    e2e = None
+    if not args.no_e2e:
+        vol_pin = torch.from_numpy(vol_host).pin_memory()
+        sino_pin = torch.from_numpy(wl.sinogram()).pin_memory()
+        sino_res = torch.empty(g.sino_shape, dtype=torch.float32).pin_memory()
+        vol_res = torch.empty(g.vol_shape, dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            with torch.cuda.stream(stream):
+                vol_d = vol_pin.to(dev, non_blocking=True)
+                y = P.forward(vol_d, stream=stream)
+                sino_res.copy_(y, non_blocking=True)
+                sino_d = sino_pin.to(dev, non_blocking=True)
+                x = P.back(sino_d, stream=stream)
+                vol_res.copy_(x, non_blocking=True)
+
+        for _ in range(max(1, min(args.warmup, 2))):
+            e2e_step()
+        stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        et = torch.tensor([s0.elapsed_time(s1) / args.steps], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(et, op=dist.ReduceOp.MAX)
+        e2e_ms = et.item()
+        e2e = {"value": world * 2 * U / (e2e_ms * 1e-3) / 1e9, "unit": UNIT, "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": int(vol_pin.numel() * 4 + sino_pin.numel() * 4),
+               "d2h_bytes_per_step": int(sino_res.numel() * 4 + vol_res.numel() * 4)}
+
+    if rank != 0:
+        return 0
+    peak, peak_kind = measured_hbm_peak()
+    B = algorithmic_bytes(U, g.n_vox, g.n_rays)
+    dominant = "back" if back_avg >= fwd_avg else "forward"
+    dom_ms = max(back_avg, fwd_avg)
+    achieved = B / (dom_ms * 1e-3) / 1e9
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        v, dt, Ucpu, desc = cpu_oracle_sample(wl, 1)
+        cpu = {"value": v / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
+               "seconds": round(dt, 2)}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32 (fp64 ray setup)", "data": "synthetic",
+        "config": workload_config(wl),
+        "updates_per_direction": U,
+        "forward": {"ms": fwd_avg, "gupdates_s": U / (fwd_avg * 1e-3) / 1e9,
+                    "views_s": g.n_views / (fwd_avg * 1e-3),
+                    "effective_gbs": B / (fwd_avg * 1e-3) / 1e9,
+                    "frac_of_hbm": B / (fwd_avg * 1e-3) / 1e9 / peak},
+        "back": {"ms": back_avg, "gupdates_s": U / (back_avg * 1e-3) / 1e9,
+                 "views_s": g.n_views / (back_avg * 1e-3),
+                 "effective_gbs": B / (back_avg * 1e-3) / 1e9,
+                 "frac_of_hbm": B / (back_avg * 1e-3) / 1e9 / peak,
+                 "variant": info["adjoint_variant"], "brick": info["brick"], "view_groups": info["view_groups"]},
+        "roofline": {"kernel": "back_brick_kernel" if dominant == "back" else "forward_kernel",
+                     "bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs",
+                     "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                     "algorithmic_bytes_per_launch": B},
+        "clocks": clk,
+        "e2e": e2e,
+        "gpu_launches": args.steps * (2 + (1 if info["n_transposed_views"] > 0 else 0)),
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", type=int, default=4)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,177 @@
+/*
+ * ctp — matched cell-constant Siddon projector pair for one NVIDIA B200 (sm_100a).
+ *
+ * Forward projection y = A x turns a voxel volume into a sinogram of ray line
+ * integrals; back projection x = A^T y is its exact adjoint.  The coefficient
+ * a_ij is the physical length of ray i inside voxel j: the cell-constant
+ * Siddon ray-voxel intersection model in physical coordinates (diffct,
+ * "Execution", section "Precision, training and reconstruction", first
+ * paragraph; section "Batch dimensions and axis spacing": traversal scales
+ * each world coordinate by its axis pitch and integrates in physical length
+ * units).  Forward and back use the same coefficients ("matched
+ * interpolation/traversal coefficients", same section), up to FP32 rounding
+ * and summation order; the floating-point scatter order is not deterministic.
+ *
+ * Precision: per-ray clipping and entry setup in FP64, traversal and data in
+ * FP32 (same page, table row backend="numba"; and the paragraph "Segment
+ * setup starts from the endpoint nearer the volume center ...").
+ *
+ * Layouts (same page, "Batch dimensions and axis spacing"):
+ *   volume    float32 [nz][ny][nx], x fastest, contiguous
+ *   sinogram  float32 [n_views][n_rows][n_cols], column fastest, contiguous
+ *   geometry  world coordinates (x, y, z), per-axis spacing (dx, dy, dz)
+ *
+ * Geometry model (the pages fix no vector convention; this is the reading):
+ *   cone beam:     src[v] is the source position; each ray is the finite
+ *                  segment from the source to a pixel centre.
+ *   parallel beam: src[v] is the ray direction (any non-zero length); each
+ *                  ray is the whole line through a pixel centre.
+ *   flat detector: pixel centre p(r, c) = det_c + (c - (n_cols-1)/2) det_u
+ *                                             + (r - (n_rows-1)/2) det_v
+ *   cylindrical detector (cone only): the cylinder axis passes through the
+ *                  source along det_v; its radius R is the distance of det_c
+ *                  from that axis; |det_u| is the arc pitch; column c sits at
+ *                  angle (c - (n_cols-1)/2) |det_u| / R from det_c, rows step
+ *                  by det_v.  det_u must be orthogonal to det_v and to
+ *                  det_c - src.
+ *   volume:        voxel (i, j, k) covers [origin + (i,j,k) * spacing,
+ *                  origin + (i+1,j+1,k+1) * spacing), half-open per axis.
+ *
+ * Calls are asynchronous: ctp_forward and ctp_back only enqueue kernels on
+ * the caller's stream, never synchronise and never read device memory back
+ * to the host.  Outputs are overwritten.  Input and output must not overlap.
+ * A geometry handle may be used from one stream at a time (its scratch
+ * buffers are shared by all calls on it); make one handle per stream for
+ * concurrent use.  Errors from a kernel that already ran surface as
+ * CTP_ERR_CUDA on a later call or on the caller's next synchronisation.
+ */
+#ifndef CTP_H
+#define CTP_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct ctp_geom ctp_geom; /* opaque, library-owned, immutable after create */
+
+typedef enum {
+  CTP_OK = 0,
+  CTP_ERR_INVALID_ARGUMENT = 1, /* bad pointer, size, enum, non-finite vector, wrong device */
+  CTP_ERR_DEGENERATE_RAY = 2,   /* a source coincides with a pixel centre, or a zero direction */
+  CTP_ERR_OUT_OF_RANGE = 3,     /* distance or pitch guard violated */
+  CTP_ERR_UNSUPPORTED = 4,      /* e.g. cylindrical detector with parallel beam */
+  CTP_ERR_OUT_OF_MEMORY = 5,    /* device scratch could not be allocated */
+  CTP_ERR_CUDA = 6              /* a CUDA runtime call failed; see ctp_last_error_detail() */
+} ctp_status;
+
+enum { CTP_BEAM_PARALLEL = 0, CTP_BEAM_CONE = 1 };
+enum { CTP_DET_FLAT = 0, CTP_DET_CYLINDRICAL = 1 };
+
+/* Adjoint variants.  AUTO picks by the collision ratio measured at create. */
+enum { CTP_ADJOINT_AUTO = 0, CTP_ADJOINT_BRICK = 1, CTP_ADJOINT_SORT = 2 };
+
+/* Optional plan overrides (all zero = library defaults). */
+typedef struct {
+  int32_t adjoint_variant;   /* CTP_ADJOINT_* */
+  int32_t brick[3];          /* adjoint brick (bx, by, bz) in voxels; 0 = automatic */
+  int32_t view_groups;       /* adjoint: split the views over this many CTA groups; 0 = automatic */
+  int32_t forward_layout;    /* 0 = automatic per view, 1 = always x-fastest volume, 2 = always y-fastest */
+  int32_t reserved[10];
+} ctp_plan;
+
+/* Acquisition and volume description.  All pointers are HOST pointers; the
+ * vectors are copied during ctp_geom_create and not referenced afterwards. */
+typedef struct {
+  int32_t beam;                 /* CTP_BEAM_PARALLEL | CTP_BEAM_CONE */
+  int32_t detector;             /* CTP_DET_FLAT | CTP_DET_CYLINDRICAL (cone only) */
+  int64_t n_views, n_rows, n_cols;
+  const double *src;            /* [n_views][3] source (cone) or direction (parallel) */
+  const double *det_c;          /* [n_views][3] detector centre */
+  const double *det_u;          /* [n_views][3] column step (length = pitch) */
+  const double *det_v;          /* [n_views][3] row step (length = pitch) */
+  int64_t nx, ny, nz;           /* volume voxels */
+  double origin[3];             /* world position of the min corner of voxel (0,0,0) */
+  double spacing[3];            /* (dx, dy, dz), each in [1e-6, 1e6], max/min <= 1e4 */
+  int32_t device;               /* CUDA device ordinal that will run the calls */
+  int32_t reserved0;
+  const ctp_plan *plan;         /* optional (NULL = defaults) */
+} ctp_geom_desc;
+
+/* Read-only facts about a created geometry. */
+typedef struct {
+  int64_t n_rays, n_vox;
+  int64_t scratch_bytes;        /* device memory the handle owns */
+  int32_t adjoint_variant;      /* variant ctp_back will run (BRICK or SORT) */
+  int32_t brick[3];
+  int32_t view_groups;
+  int32_t n_transposed_views;   /* views whose forward gathers from the y-fastest copy */
+  double collision_ratio;       /* updates / distinct voxels per sort batch, measured at create */
+} ctp_geom_info;
+
+/*
+ * ctp_geom_create — validate the description, copy the per-view vectors to
+ * the device and allocate the handle's scratch.
+ *
+ * Guards (each returns an error and leaves nothing allocated), following
+ * diffct "Execution": finite vectors; positive sizes; per-axis pitch in
+ * [1e-6, 1e6] with largest/smallest <= 1e4 (section "Batch dimensions and axis
+ * spacing"); cone beam: every view needs one ray endpoint within 1e6 voxels of
+ * the volume centre and both within 1e15, distance measured as
+ * |((x-cx)/dx, (y-cy)/dy, (z-cz)/dz)| (section "Precision, training and
+ * reconstruction"); no source may coincide with a pixel centre (section
+ * "Batch dimensions and axis spacing": finite rays are degenerate when their
+ * endpoints coincide); flat detectors are checked at their corners (section
+ * "Call-time trajectory validation").  Validation runs on the host before any
+ * CUDA call.  *out receives the handle on success and is untouched on error.
+ */
+ctp_status ctp_geom_create(const ctp_geom_desc *desc, ctp_geom **out);
+
+/* Free a handle and its device memory (synchronises the device first).  NULL is a no-op. */
+void ctp_geom_destroy(ctp_geom *geom);
+
+/* Fill *info.  Host-only, no CUDA call. */
+ctp_status ctp_geom_query(const ctp_geom *geom, ctp_geom_info *info);
+
+/*
+ * ctp_forward — sino = A vol (diffct "Execution": Projector.project).
+ * vol:  device pointer, float32 [nz][ny][nx], read only.
+ * sino: device pointer, float32 [n_views][n_rows][n_cols], overwritten
+ *       (rays that miss the volume get 0).
+ * stream: a cudaStream_t (NULL = legacy default stream) on the handle's device.
+ * Both pointers must be device (or managed) memory of the handle's device,
+ * else CTP_ERR_INVALID_ARGUMENT.  No synchronisation.
+ */
+ctp_status ctp_forward(const ctp_geom *geom, const float *vol, float *sino, void *stream);
+
+/*
+ * ctp_back — vol = A^T sino, the exact transpose of ctp_forward's
+ * coefficients (diffct "Execution": backward applies the matched adjoint).
+ * sino: device pointer, float32 [n_views][n_rows][n_cols], read only.
+ * vol:  device pointer, float32 [nz][ny][nx], overwritten.
+ * Same pointer, stream and synchronisation rules as ctp_forward.
+ */
+ctp_status ctp_back(const ctp_geom *geom, const float *sino, float *vol, void *stream);
+
+/*
+ * ctp_count_updates — the number of positive-length ray-voxel segments of the
+ * whole acquisition (the work measure of both projectors), computed on the
+ * device.  Synchronous: waits for the count and writes it to *host_out.
+ */
+ctp_status ctp_count_updates(const ctp_geom *geom, int64_t *host_out, void *stream);
+
+/* Static description of a status code. */
+const char *ctp_status_string(ctp_status status);
+
+/* Detail message of the last failing call on this host thread ("" if none). */
+const char *ctp_last_error_detail(void);
+
+/* Library version, "major.minor.patch". */
+const char *ctp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CTP_H */

@@ -1,0 +1,555 @@
+// C-ABI entry points of libctp: geometry validation and planning on the host,
+// device upload of the per-view FP64 records, and the asynchronous forward /
+// adjoint calls.  See include/ctp.h for the contract of every function.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "ctp_internal.h"
+
+using ctp::BackLaunch;
+using ctp::FwdLaunch;
+using ctp::ViewRec;
+using ctp::VolDesc;
+
+struct ctp_geom {
+  int device = 0;
+  int beam = 0, det = 0;
+  int64_t n_views = 0, n_rows = 0, n_cols = 0;
+  int64_t nx = 0, ny = 0, nz = 0;
+  int64_t n_rays = 0, n_vox = 0;
+  bool wide_index = false;
+  VolDesc vol{};
+  ctp::Dims dims{};
+  FwdLaunch fwd{};
+  BackLaunch back{};
+  int adjoint_variant = CTP_ADJOINT_BRICK;
+  int n_transposed = 0;
+  double collision_ratio = 0.0;
+  ViewRec *d_views = nullptr;
+  double *d_trig = nullptr;
+  float *d_volT = nullptr;
+  unsigned long long *d_counter = nullptr;
+  int64_t scratch_bytes = 0;
+};
+
+namespace {
+
+thread_local char g_detail[512] = "";
+
+ctp_status fail(ctp_status s, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_detail, sizeof(g_detail), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+ctp_status cuda_fail(cudaError_t e, const char *where) {
+  return fail(CTP_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+double dot(const double *a, const double *b) { return a[0] * b[0] + a[1] * b[1] + a[2] * b[2]; }
+double norm(const double *a) { return std::sqrt(dot(a, a)); }
+void cross(const double *a, const double *b, double *c) {
+  c[0] = a[1] * b[2] - a[2] * b[1];
+  c[1] = a[2] * b[0] - a[0] * b[2];
+  c[2] = a[0] * b[1] - a[1] * b[0];
+}
+bool finite3(const double *p) { return std::isfinite(p[0]) && std::isfinite(p[1]) && std::isfinite(p[2]); }
+
+// Inverse of the 3x3 matrix with the given columns; false if (near) singular.
+bool invert_columns(const double *c0, const double *c1, const double *c2, double *inv) {
+  double m[9] = {c0[0], c1[0], c2[0], c0[1], c1[1], c2[1], c0[2], c1[2], c2[2]};
+  double det = m[0] * (m[4] * m[8] - m[5] * m[7]) - m[1] * (m[3] * m[8] - m[5] * m[6]) +
+               m[2] * (m[3] * m[7] - m[4] * m[6]);
+  double scale = norm(c0) * norm(c1) * norm(c2);
+  if (!(std::fabs(det) > 1e-12 * scale) || !std::isfinite(det)) return false;
+  double id = 1.0 / det;
+  inv[0] = (m[4] * m[8] - m[5] * m[7]) * id;
+  inv[1] = (m[2] * m[7] - m[1] * m[8]) * id;
+  inv[2] = (m[1] * m[5] - m[2] * m[4]) * id;
+  inv[3] = (m[5] * m[6] - m[3] * m[8]) * id;
+  inv[4] = (m[0] * m[8] - m[2] * m[6]) * id;
+  inv[5] = (m[2] * m[3] - m[0] * m[5]) * id;
+  inv[6] = (m[3] * m[7] - m[4] * m[6]) * id;
+  inv[7] = (m[1] * m[6] - m[0] * m[7]) * id;
+  inv[8] = (m[0] * m[4] - m[1] * m[3]) * id;
+  return true;
+}
+
+constexpr double kNearLimit = 1e6;  // one endpoint within this many voxels of the centre
+constexpr double kFarLimit = 1e15;  // both endpoints within this many voxels
+
+// Voxel-scaled distance |((p - centre) / spacing)|.
+double vox_dist(const double *p, const double *centre_w, const double *sp) {
+  double s = 0.0;
+  for (int k = 0; k < 3; ++k) {
+    double d = (p[k] - centre_w[k]) / sp[k];
+    s += d * d;
+  }
+  return std::sqrt(s);
+}
+
+// World pixel centre, same formulas the kernels use (see ViewRec).
+void host_pixel(const ViewRec &V, int det, int64_t r, int64_t c, double *p) {
+  if (det == CTP_DET_FLAT) {
+    for (int k = 0; k < 3; ++k) p[k] = V.p00[k] + (double)c * V.du[k] + (double)r * V.dv[k];
+  } else {
+    double g = V.gam0 + (double)c * V.dgam;
+    for (int k = 0; k < 3; ++k)
+      p[k] = V.p00[k] + (double)r * V.dv[k] + V.R * (std::cos(g) * V.w[k] + std::sin(g) * V.du[k]);
+  }
+}
+
+ctp_status validate_desc(const ctp_geom_desc *d) {
+  if (!d) return fail(CTP_ERR_INVALID_ARGUMENT, "desc is NULL");
+  if (d->beam != CTP_BEAM_PARALLEL && d->beam != CTP_BEAM_CONE)
+    return fail(CTP_ERR_INVALID_ARGUMENT, "beam %d is not CTP_BEAM_PARALLEL or CTP_BEAM_CONE", d->beam);
+  if (d->detector != CTP_DET_FLAT && d->detector != CTP_DET_CYLINDRICAL)
+    return fail(CTP_ERR_INVALID_ARGUMENT, "detector %d is not CTP_DET_FLAT or CTP_DET_CYLINDRICAL", d->detector);
+  if (d->detector == CTP_DET_CYLINDRICAL && d->beam != CTP_BEAM_CONE)
+    return fail(CTP_ERR_UNSUPPORTED, "a cylindrical detector needs a cone beam");
+  const int64_t lim = 0x7fffffff;
+  if (d->n_views <= 0 || d->n_rows <= 0 || d->n_cols <= 0)
+    return fail(CTP_ERR_INVALID_ARGUMENT, "detector sizes must be positive (views %lld rows %lld cols %lld)",
+                (long long)d->n_views, (long long)d->n_rows, (long long)d->n_cols);
+  if (d->nx <= 0 || d->ny <= 0 || d->nz <= 0)
+    return fail(CTP_ERR_INVALID_ARGUMENT, "volume sizes must be positive (%lld, %lld, %lld)", (long long)d->nx,
+                (long long)d->ny, (long long)d->nz);
+  if (d->n_views > lim || d->n_rows > lim || d->n_cols > lim || d->nx > lim || d->ny > lim || d->nz > lim)
+    return fail(CTP_ERR_OUT_OF_RANGE, "a size exceeds 2^31-1");
+  // element counts below 2^62 (offsets are 64-bit where needed)
+  const double rays = (double)d->n_views * (double)d->n_rows * (double)d->n_cols;
+  const double vox = (double)d->nx * (double)d->ny * (double)d->nz;
+  if (rays >= 4.6e18 || vox >= 4.6e18) return fail(CTP_ERR_OUT_OF_RANGE, "element count too large");
+  const double row_blocks = (double)((d->n_rows + 7) / 8) * (double)d->n_views * (double)((d->n_cols + 31) / 32);
+  if (row_blocks > 2147483647.0) return fail(CTP_ERR_OUT_OF_RANGE, "too many detector tiles for one launch");
+  for (int k = 0; k < 3; ++k) {
+    if (!std::isfinite(d->origin[k])) return fail(CTP_ERR_INVALID_ARGUMENT, "origin[%d] is not finite", k);
+    double s = d->spacing[k];
+    if (!std::isfinite(s) || s < 1e-6 || s > 1e6)
+      return fail(CTP_ERR_OUT_OF_RANGE, "spacing[%d] = %g outside [1e-6, 1e6]", k, s);
+  }
+  double smax = std::fmax(d->spacing[0], std::fmax(d->spacing[1], d->spacing[2]));
+  double smin = std::fmin(d->spacing[0], std::fmin(d->spacing[1], d->spacing[2]));
+  if (smax / smin > 1e4) return fail(CTP_ERR_OUT_OF_RANGE, "largest/smallest spacing %g exceeds 1e4", smax / smin);
+  if (!d->src || !d->det_c || !d->det_u || !d->det_v)
+    return fail(CTP_ERR_INVALID_ARGUMENT, "a per-view vector array is NULL");
+  if (d->plan) {
+    const ctp_plan *p = d->plan;
+    if (p->adjoint_variant < CTP_ADJOINT_AUTO || p->adjoint_variant > CTP_ADJOINT_SORT)
+      return fail(CTP_ERR_INVALID_ARGUMENT, "plan.adjoint_variant %d", p->adjoint_variant);
+    if (p->adjoint_variant == CTP_ADJOINT_SORT)
+      return fail(CTP_ERR_UNSUPPORTED, "the sort/segment-reduce adjoint is not available in this build");
+    for (int k = 0; k < 3; ++k)
+      if (p->brick[k] < 0 || p->brick[k] > 1024) return fail(CTP_ERR_INVALID_ARGUMENT, "plan.brick[%d]", k);
+    if (p->view_groups < 0) return fail(CTP_ERR_INVALID_ARGUMENT, "plan.view_groups");
+    if (p->forward_layout < 0 || p->forward_layout > 2) return fail(CTP_ERR_INVALID_ARGUMENT, "plan.forward_layout");
+  }
+  return CTP_OK;
+}
+
+// Per-view records and per-view guards.  Host FP64 throughout.
+ctp_status build_views(const ctp_geom_desc *d, std::vector<ViewRec> &views, std::vector<double> &trig) {
+  const int64_t nv = d->n_views, nr = d->n_rows, nc = d->n_cols;
+  const double cc = 0.5 * (double)(nc - 1), rc = 0.5 * (double)(nr - 1);
+  const double n3[3] = {(double)d->nx, (double)d->ny, (double)d->nz};
+  double centre_w[3];
+  for (int k = 0; k < 3; ++k) centre_w[k] = d->origin[k] + 0.5 * n3[k] * d->spacing[k];
+  const double smin = std::fmin(d->spacing[0], std::fmin(d->spacing[1], d->spacing[2]));
+  views.assign((size_t)nv, ViewRec{});
+  if (d->detector == CTP_DET_CYLINDRICAL) trig.assign((size_t)(2 * nv * nc), 0.0);
+  for (int64_t v = 0; v < nv; ++v) {
+    const double *s = d->src + 3 * v, *dc = d->det_c + 3 * v, *du = d->det_u + 3 * v, *dv = d->det_v + 3 * v;
+    if (!finite3(s) || !finite3(dc) || !finite3(du) || !finite3(dv))
+      return fail(CTP_ERR_INVALID_ARGUMENT, "view %lld: a vector is not finite", (long long)v);
+    const double nu = norm(du), nvl = norm(dv);
+    if (!(nu > 0.0) || !(nvl > 0.0))
+      return fail(CTP_ERR_INVALID_ARGUMENT, "view %lld: det_u and det_v must be non-zero", (long long)v);
+    ViewRec &V = views[(size_t)v];
+    V.vlen = nvl;
+    for (int k = 0; k < 3; ++k) V.vhat[k] = dv[k] / nvl;
+    for (int k = 0; k < 3; ++k) V.dv[k] = dv[k];
+    if (d->beam == CTP_BEAM_PARALLEL) {
+      const double ns = norm(s);
+      if (!(ns > 0.0)) return fail(CTP_ERR_DEGENERATE_RAY, "view %lld: zero ray direction", (long long)v);
+      for (int k = 0; k < 3; ++k) {
+        V.s[k] = s[k] / ns;
+        V.p00[k] = dc[k] - cc * du[k] - rc * dv[k];
+        V.du[k] = du[k];
+        const double dvox = V.s[k] / d->spacing[k];
+        V.rcp_dir[k] = dvox != 0.0 ? 1.0 / dvox : HUGE_VAL;
+      }
+      if (!invert_columns(du, dv, V.s, V.minv))
+        return fail(CTP_ERR_DEGENERATE_RAY, "view %lld: ray direction lies in the detector plane", (long long)v);
+    } else if (d->detector == CTP_DET_FLAT) {
+      double n[3];
+      cross(du, dv, n);
+      const double nn = norm(n);
+      if (!(nn > 1e-12 * nu * nvl))
+        return fail(CTP_ERR_INVALID_ARGUMENT, "view %lld: det_u and det_v are parallel", (long long)v);
+      for (int k = 0; k < 3; ++k) {
+        V.s[k] = s[k];
+        V.p00[k] = dc[k] - cc * du[k] - rc * dv[k];
+        V.du[k] = du[k];
+      }
+      // Source / pixel coincidence: only possible if the source lies in the detector plane.
+      double rel[3] = {s[0] - dc[0], s[1] - dc[1], s[2] - dc[2]};
+      const double h = std::fabs(dot(rel, n)) / nn;
+      const double scale = std::fmax(norm(rel), std::fmax(nu, nvl));
+      double sp00[3] = {V.p00[0] - s[0], V.p00[1] - s[1], V.p00[2] - s[2]};
+      if (!(h > 1e-12 * scale)) {
+        // coordinates of the source in the pixel lattice
+        double inv[9];
+        double a[3] = {s[0] - V.p00[0], s[1] - V.p00[1], s[2] - V.p00[2]};
+        if (invert_columns(du, dv, n, inv)) {
+          const double cs = inv[0] * a[0] + inv[1] * a[1] + inv[2] * a[2];
+          const double rs = inv[3] * a[0] + inv[4] * a[1] + inv[5] * a[2];
+          const double ci = std::round(cs), ri = std::round(rs);
+          if (std::fabs(cs - ci) < 1e-9 && std::fabs(rs - ri) < 1e-9 && ci >= 0 && ci < (double)nc && ri >= 0 &&
+              ri < (double)nr)
+            return fail(CTP_ERR_DEGENERATE_RAY, "view %lld: the source coincides with pixel (%g, %g)", (long long)v,
+                        ri, ci);
+        }
+        V.full_footprint = 1;
+      } else if (!invert_columns(sp00, du, dv, V.minv)) {
+        V.full_footprint = 1;
+      }
+      // distance guards at the detector corners (pixel distance is convex over the plane)
+      const double ds = vox_dist(s, centre_w, d->spacing);
+      double dp_max = 0.0;
+      for (int corner = 0; corner < 4; ++corner) {
+        double p[3];
+        host_pixel(V, CTP_DET_FLAT, (corner & 1) ? nr - 1 : 0, (corner & 2) ? nc - 1 : 0, p);
+        dp_max = std::fmax(dp_max, vox_dist(p, centre_w, d->spacing));
+      }
+      if (!(ds <= kFarLimit && dp_max <= kFarLimit))
+        return fail(CTP_ERR_OUT_OF_RANGE, "view %lld: an endpoint is beyond 1e15 voxels", (long long)v);
+      if (!(ds <= kNearLimit || dp_max <= kNearLimit))
+        return fail(CTP_ERR_OUT_OF_RANGE, "view %lld: no endpoint within 1e6 voxels of the volume centre",
+                    (long long)v);
+    } else {
+      // cylindrical detector centred on the source's axis
+      const double uhat[3] = {du[0] / nu, du[1] / nu, du[2] / nu};
+      double w0[3] = {dc[0] - s[0], dc[1] - s[1], dc[2] - s[2]};
+      const double axial = dot(w0, V.vhat);
+      double wp[3];
+      for (int k = 0; k < 3; ++k) wp[k] = w0[k] - axial * V.vhat[k];
+      const double R = norm(wp);
+      if (!(R > 1e-9 * std::fmax(norm(w0), 1.0)))
+        return fail(CTP_ERR_DEGENERATE_RAY, "view %lld: the detector centre lies on the source's axis", (long long)v);
+      if (std::fabs(dot(uhat, V.vhat)) > 1e-9)
+        return fail(CTP_ERR_INVALID_ARGUMENT, "view %lld: det_u must be orthogonal to det_v", (long long)v);
+      if (std::fabs(dot(uhat, wp)) > 1e-9 * R)
+        return fail(CTP_ERR_INVALID_ARGUMENT, "view %lld: det_u must be orthogonal to det_c - src", (long long)v);
+      V.R = R;
+      for (int k = 0; k < 3; ++k) {
+        V.s[k] = s[k];
+        V.w[k] = wp[k] / R;
+        V.du[k] = uhat[k];
+      }
+      V.dgam = nu / R;
+      V.gam0 = -cc * V.dgam;
+      V.axial0 = axial - rc * nvl;
+      for (int k = 0; k < 3; ++k) V.p00[k] = s[k] + V.axial0 * V.vhat[k];
+      for (int64_t c = 0; c < nc; ++c) {
+        const double g = V.gam0 + (double)c * V.dgam;
+        trig[(size_t)(2 * (v * nc + c))] = std::cos(g);
+        trig[(size_t)(2 * (v * nc + c) + 1)] = std::sin(g);
+      }
+      // distance guards: a bound first, the exact per-pixel check only if it fails
+      const double ds = vox_dist(s, centre_w, d->spacing);
+      const double row_ext = std::fmax(std::fabs(V.axial0), std::fabs(V.axial0 + (double)(nr - 1) * nvl));
+      const double bound = ds + (R + row_ext) / smin;
+      double dp_max = bound;
+      if (!(ds <= kNearLimit || bound <= kNearLimit) || !(bound <= kFarLimit)) {
+        dp_max = 0.0;
+        for (int64_t r = 0; r < nr; ++r)
+          for (int64_t c = 0; c < nc; ++c) {
+            double p[3];
+            const double g = V.gam0 + (double)c * V.dgam;
+            for (int k = 0; k < 3; ++k)
+              p[k] = V.p00[k] + (double)r * V.dv[k] + R * (std::cos(g) * V.w[k] + std::sin(g) * V.du[k]);
+            dp_max = std::fmax(dp_max, vox_dist(p, centre_w, d->spacing));
+          }
+      }
+      if (!(ds <= kFarLimit && dp_max <= kFarLimit))
+        return fail(CTP_ERR_OUT_OF_RANGE, "view %lld: an endpoint is beyond 1e15 voxels", (long long)v);
+      if (!(ds <= kNearLimit || dp_max <= kNearLimit))
+        return fail(CTP_ERR_OUT_OF_RANGE, "view %lld: no endpoint within 1e6 voxels of the volume centre",
+                    (long long)v);
+    }
+    // forward gather layout: y-fastest copy when the column step runs mostly along y
+    const double ux = std::fabs(du[0] / d->spacing[0]), uy = std::fabs(du[1] / d->spacing[1]),
+                 uz = std::fabs(du[2] / d->spacing[2]);
+    V.layout = (uy > ux && uy >= uz) ? 1 : 0;
+    if (d->plan && d->plan->forward_layout == 1) V.layout = 0;
+    if (d->plan && d->plan->forward_layout == 2) V.layout = 1;
+  }
+  return CTP_OK;
+}
+
+void plan_back(ctp_geom *g, const ctp_plan *plan) {
+  int b[3];
+  if (g->beam == CTP_BEAM_PARALLEL) {
+    b[0] = 64, b[1] = 64, b[2] = 4;
+  } else {
+    b[0] = 32, b[1] = 32, b[2] = 16;
+  }
+  if (plan)
+    for (int k = 0; k < 3; ++k)
+      if (plan->brick[k] > 0) b[k] = plan->brick[k];
+  const int64_t n[3] = {g->nx, g->ny, g->nz};
+  for (int k = 0; k < 3; ++k) b[k] = (int)std::min<int64_t>(b[k], n[k]);
+  BackLaunch &p = g->back;
+  p.dims = g->dims;
+  p.vol = g->vol;
+  int64_t nb = 1;
+  for (int k = 0; k < 3; ++k) {
+    p.brick[k] = b[k];
+    p.nbrick[k] = (int)((n[k] + b[k] - 1) / b[k]);
+    nb *= p.nbrick[k];
+  }
+  p.pitch_x = b[0] + 1;
+  const int64_t target = 148 * 3 * 2;  // two waves of three resident CTAs per SM
+  int groups = 1;
+  if (nb < target) groups = (int)std::min<int64_t>((target + nb - 1) / nb, std::max<int64_t>(1, g->n_views / 4));
+  if (plan && plan->view_groups > 0) groups = (int)std::min<int64_t>(plan->view_groups, g->n_views);
+  int vpg = (int)((g->n_views + groups - 1) / groups);
+  groups = (int)((g->n_views + vpg - 1) / vpg);
+  p.view_groups = groups;
+  p.views_per_group = vpg;
+}
+
+bool is_device_pointer(const void *ptr, int device) {
+  if (!ptr) return false;
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, ptr) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) && a.device == device;
+}
+
+struct DeviceGuard {
+  int prev = -1;
+  bool switched = false;
+  cudaError_t err = cudaSuccess;
+  explicit DeviceGuard(int dev) {
+    err = cudaGetDevice(&prev);
+    if (err == cudaSuccess && prev != dev) {
+      err = cudaSetDevice(dev);
+      switched = err == cudaSuccess;
+    }
+  }
+  ~DeviceGuard() {
+    if (switched) cudaSetDevice(prev);
+  }
+};
+
+void free_geom(ctp_geom *g) {
+  if (!g) return;
+  cudaFree(g->d_views);
+  cudaFree(g->d_trig);
+  cudaFree(g->d_volT);
+  cudaFree(g->d_counter);
+  delete g;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *ctp_version(void) { return "0.1.0"; }
+
+const char *ctp_status_string(ctp_status s) {
+  switch (s) {
+    case CTP_OK: return "ok";
+    case CTP_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case CTP_ERR_DEGENERATE_RAY: return "degenerate ray";
+    case CTP_ERR_OUT_OF_RANGE: return "out of range";
+    case CTP_ERR_UNSUPPORTED: return "unsupported";
+    case CTP_ERR_OUT_OF_MEMORY: return "out of device memory";
+    case CTP_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+const char *ctp_last_error_detail(void) { return g_detail; }
+
+ctp_status ctp_geom_create(const ctp_geom_desc *desc, ctp_geom **out) {
+  g_detail[0] = '\0';
+  if (!out) return fail(CTP_ERR_INVALID_ARGUMENT, "out is NULL");
+  ctp_status st = validate_desc(desc);
+  if (st != CTP_OK) return st;
+  std::vector<ViewRec> views;
+  std::vector<double> trig;
+  st = build_views(desc, views, trig);
+  if (st != CTP_OK) return st;
+
+  ctp_geom *g = new (std::nothrow) ctp_geom();
+  if (!g) return fail(CTP_ERR_OUT_OF_MEMORY, "host allocation failed");
+  g->device = desc->device;
+  g->beam = desc->beam;
+  g->det = desc->detector;
+  g->n_views = desc->n_views;
+  g->n_rows = desc->n_rows;
+  g->n_cols = desc->n_cols;
+  g->nx = desc->nx;
+  g->ny = desc->ny;
+  g->nz = desc->nz;
+  g->n_rays = g->n_views * g->n_rows * g->n_cols;
+  g->n_vox = g->nx * g->ny * g->nz;
+  g->wide_index = g->n_vox >= (int64_t)0x7fffffff;
+  VolDesc &vd = g->vol;
+  vd.n[0] = (int32_t)g->nx;
+  vd.n[1] = (int32_t)g->ny;
+  vd.n[2] = (int32_t)g->nz;
+  for (int k = 0; k < 3; ++k) {
+    vd.origin[k] = desc->origin[k];
+    vd.spacing[k] = desc->spacing[k];
+    vd.inv_spacing[k] = 1.0 / desc->spacing[k];
+    vd.centre[k] = 0.5 * (double)vd.n[k];
+  }
+  ctp::Dims &dm = g->dims;
+  dm.beam = g->beam;
+  dm.det = g->det;
+  dm.n_views = (int32_t)g->n_views;
+  dm.n_rows = (int32_t)g->n_rows;
+  dm.n_cols = (int32_t)g->n_cols;
+  for (const ViewRec &V : views) g->n_transposed += V.layout != 0;
+  FwdLaunch &f = g->fwd;
+  f.dims = dm;
+  f.vol = vd;
+  f.n_col_tiles = (int32_t)((g->n_cols + 31) / 32);
+  f.n_row_bands = (int32_t)((g->n_rows + 7) / 8);
+  f.any_transposed = g->n_transposed > 0;
+  const ctp_plan *plan = desc->plan;
+  g->adjoint_variant = CTP_ADJOINT_BRICK;
+  plan_back(g, plan);
+  if (ctp::back_brick_smem_bytes(g->back.brick) > 227 * 1024) {
+    delete g;
+    return fail(CTP_ERR_INVALID_ARGUMENT, "adjoint brick needs more than 227 KB of shared memory");
+  }
+
+  DeviceGuard dg(g->device);
+  if (dg.err != cudaSuccess) {
+    ctp_status s = cuda_fail(dg.err, "cudaSetDevice");
+    delete g;
+    return s;
+  }
+  auto alloc = [&](void **p, size_t bytes, const char *what) -> ctp_status {
+    cudaError_t e = cudaMalloc(p, bytes);
+    if (e == cudaErrorMemoryAllocation) {
+      cudaGetLastError();
+      return fail(CTP_ERR_OUT_OF_MEMORY, "cudaMalloc(%zu) for %s failed", bytes, what);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc");
+    g->scratch_bytes += (int64_t)bytes;
+    return CTP_OK;
+  };
+  size_t vbytes = sizeof(ViewRec) * views.size();
+  st = alloc((void **)&g->d_views, vbytes, "view records");
+  if (st == CTP_OK && !trig.empty()) st = alloc((void **)&g->d_trig, sizeof(double) * trig.size(), "column angles");
+  if (st == CTP_OK && f.any_transposed)
+    st = alloc((void **)&g->d_volT, sizeof(float) * (size_t)g->n_vox, "y-fastest volume copy");
+  if (st == CTP_OK) st = alloc((void **)&g->d_counter, sizeof(unsigned long long), "counter");
+  cudaError_t e = cudaSuccess;
+  if (st == CTP_OK) {
+    e = cudaMemcpy(g->d_views, views.data(), vbytes, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && !trig.empty())
+      e = cudaMemcpy(g->d_trig, trig.data(), sizeof(double) * trig.size(), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = ctp::prepare_back_brick(ctp::back_brick_smem_bytes(g->back.brick));
+    if (e != cudaSuccess) st = cuda_fail(e, "geometry upload");
+  }
+  if (st != CTP_OK) {
+    free_geom(g);
+    return st;
+  }
+  *out = g;
+  return CTP_OK;
+}
+
+void ctp_geom_destroy(ctp_geom *g) {
+  if (!g) return;
+  DeviceGuard dg(g->device);
+  cudaDeviceSynchronize();
+  free_geom(g);
+}
+
+ctp_status ctp_geom_query(const ctp_geom *g, ctp_geom_info *info) {
+  if (!g || !info) return fail(CTP_ERR_INVALID_ARGUMENT, "NULL argument");
+  info->n_rays = g->n_rays;
+  info->n_vox = g->n_vox;
+  info->scratch_bytes = g->scratch_bytes;
+  info->adjoint_variant = g->adjoint_variant;
+  for (int k = 0; k < 3; ++k) info->brick[k] = g->back.brick[k];
+  info->view_groups = g->back.view_groups;
+  info->n_transposed_views = g->n_transposed;
+  info->collision_ratio = g->collision_ratio;
+  return CTP_OK;
+}
+
+ctp_status ctp_forward(const ctp_geom *g, const float *vol, float *sino, void *stream) {
+  g_detail[0] = '\0';
+  if (!g) return fail(CTP_ERR_INVALID_ARGUMENT, "geometry is NULL");
+  DeviceGuard dg(g->device);
+  if (dg.err != cudaSuccess) return cuda_fail(dg.err, "cudaSetDevice");
+  if (!is_device_pointer(vol, g->device))
+    return fail(CTP_ERR_INVALID_ARGUMENT, "vol is not device memory of device %d", g->device);
+  if (!is_device_pointer(sino, g->device))
+    return fail(CTP_ERR_INVALID_ARGUMENT, "sino is not device memory of device %d", g->device);
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "pending error before ctp_forward");
+  if (g->fwd.any_transposed) {
+    e = ctp::launch_transpose_xy(vol, g->d_volT, g->vol, s);
+    if (e != cudaSuccess) return cuda_fail(e, "transpose launch");
+  }
+  e = ctp::launch_forward(g->fwd, g->d_views, g->d_trig, vol, g->d_volT, sino, g->wide_index, s);
+  if (e != cudaSuccess) return cuda_fail(e, "forward launch");
+  return CTP_OK;
+}
+
+ctp_status ctp_back(const ctp_geom *g, const float *sino, float *vol, void *stream) {
+  g_detail[0] = '\0';
+  if (!g) return fail(CTP_ERR_INVALID_ARGUMENT, "geometry is NULL");
+  DeviceGuard dg(g->device);
+  if (dg.err != cudaSuccess) return cuda_fail(dg.err, "cudaSetDevice");
+  if (!is_device_pointer(sino, g->device))
+    return fail(CTP_ERR_INVALID_ARGUMENT, "sino is not device memory of device %d", g->device);
+  if (!is_device_pointer(vol, g->device))
+    return fail(CTP_ERR_INVALID_ARGUMENT, "vol is not device memory of device %d", g->device);
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "pending error before ctp_back");
+  if (g->back.view_groups > 1) {
+    e = cudaMemsetAsync(vol, 0, sizeof(float) * (size_t)g->n_vox, s);
+    if (e != cudaSuccess) return cuda_fail(e, "volume zero-fill");
+  }
+  e = ctp::launch_back_brick(g->back, g->d_views, g->d_trig, sino, vol, g->wide_index, s);
+  if (e != cudaSuccess) return cuda_fail(e, "adjoint launch");
+  return CTP_OK;
+}
+
+ctp_status ctp_count_updates(const ctp_geom *g, int64_t *host_out, void *stream) {
+  g_detail[0] = '\0';
+  if (!g || !host_out) return fail(CTP_ERR_INVALID_ARGUMENT, "NULL argument");
+  DeviceGuard dg(g->device);
+  if (dg.err != cudaSuccess) return cuda_fail(dg.err, "cudaSetDevice");
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(g->d_counter, 0, sizeof(unsigned long long), s);
+  if (e == cudaSuccess) e = ctp::launch_count(g->fwd, g->d_views, g->d_trig, g->d_counter, s);
+  unsigned long long n = 0;
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&n, g->d_counter, sizeof(n), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "count");
+  *host_out = (int64_t)n;
+  return CTP_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,79 @@
+// Internal types shared by the host entry points (ctp_api.cu) and the kernels
+// (ctp_kernels.cu).  Not part of the public C ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "ctp.h"
+
+namespace ctp {
+
+// Per-view geometry in FP64, prepared on the host at create time.
+//
+// Pixel centre of (row r, column c), world coordinates:
+//   flat:        p = p00 + c * du + r * dv
+//   cylindrical: p = p00 + r * dv + R * (cos g * w + sin g * du),  g = gam0 + c * dgam
+// (for the cylindrical detector du holds the unit tangent u^ and p00 the
+// point on the source's axis at the height of row 0).
+struct ViewRec {
+  double s[3];        // cone: source position; parallel: unit ray direction
+  double p00[3];
+  double du[3];
+  double dv[3];
+  double w[3];        // cylindrical: unit radial direction of the middle column
+  double vhat[3];     // unit row direction
+  double rcp_dir[3];  // parallel: 1 / (direction in voxel units), +-inf where 0
+  double minv[9];     // footprint matrix: parallel flat [du dv s]^-1, cone flat [p00-s du dv]^-1
+  double R, gam0, dgam, axial0, vlen;
+  int32_t layout;     // forward gather: 0 = x-fastest volume, 1 = y-fastest copy
+  int32_t full_footprint;  // 1: the footprint test cannot bound this view; scan all pixels
+};
+
+struct VolDesc {
+  int32_t n[3];       // nx, ny, nz
+  int32_t pad;
+  double origin[3];
+  double spacing[3];
+  double inv_spacing[3];
+  double centre[3];   // volume centre in voxel units (n / 2)
+};
+
+struct Dims {
+  int32_t beam, det;
+  int32_t n_views, n_rows, n_cols;
+  int32_t pad;
+};
+
+struct FwdLaunch {
+  Dims dims;
+  VolDesc vol;
+  int32_t n_col_tiles, n_row_bands;
+  int32_t any_transposed;
+};
+
+struct BackLaunch {
+  Dims dims;
+  VolDesc vol;
+  int32_t brick[3];      // brick size
+  int32_t nbrick[3];     // bricks per axis
+  int32_t pitch_x;       // shared-memory row pitch (brick[0] + 1)
+  int32_t view_groups;   // CTA groups over the views; >1 means atomic flush into a zeroed volume
+  int32_t views_per_group;
+  int32_t pad;
+};
+
+// Launchers (ctp_kernels.cu).  All enqueue on `stream` and return the launch error.
+cudaError_t launch_transpose_xy(const float* vol, float* volT, const VolDesc& vd, cudaStream_t stream);
+cudaError_t launch_forward(const FwdLaunch& p, const ViewRec* views, const double* trig, const float* vol,
+                           const float* volT, float* sino, bool wide_index, cudaStream_t stream);
+cudaError_t launch_back_brick(const BackLaunch& p, const ViewRec* views, const double* trig, const float* sino,
+                              float* vol, bool wide_index, cudaStream_t stream);
+cudaError_t launch_count(const FwdLaunch& p, const ViewRec* views, const double* trig,
+                         unsigned long long* counter, cudaStream_t stream);
+size_t back_brick_smem_bytes(const int32_t brick[3]);
+cudaError_t prepare_back_brick(size_t smem_bytes);
+
+}  // namespace ctp

@@ -1,0 +1,264 @@
+"""Python binding of libctp (ctypes): argument marshalling only.
+
+The names mirror the C ABI in include/ctp.h: ``ctp_geom_create``,
+``ctp_forward``, ``ctp_back``, ``ctp_count_updates`` ...  Every step of the
+projectors runs in the library's CUDA kernels; there is no fallback.  If the
+library is missing or CUDA is unavailable the calls raise.
+
+``Projector`` is the convenience wrapper over a geometry handle that takes
+torch CUDA tensors and the current torch stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libctp.so")
+
+CTP_OK = 0
+CTP_ERR_INVALID_ARGUMENT = 1
+CTP_ERR_DEGENERATE_RAY = 2
+CTP_ERR_OUT_OF_RANGE = 3
+CTP_ERR_UNSUPPORTED = 4
+CTP_ERR_OUT_OF_MEMORY = 5
+CTP_ERR_CUDA = 6
+
+CTP_BEAM_PARALLEL = 0
+CTP_BEAM_CONE = 1
+CTP_DET_FLAT = 0
+CTP_DET_CYLINDRICAL = 1
+CTP_ADJOINT_AUTO = 0
+CTP_ADJOINT_BRICK = 1
+CTP_ADJOINT_SORT = 2
+
+EXPORTED = ["ctp_geom_create", "ctp_geom_destroy", "ctp_geom_query", "ctp_forward", "ctp_back",
+            "ctp_count_updates", "ctp_status_string", "ctp_last_error_detail", "ctp_version"]
+
+
+class ctp_plan(ctypes.Structure):
+    _fields_ = [("adjoint_variant", ctypes.c_int32), ("brick", ctypes.c_int32 * 3),
+                ("view_groups", ctypes.c_int32), ("forward_layout", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 10)]
+
+
+class ctp_geom_desc(ctypes.Structure):
+    _fields_ = [("beam", ctypes.c_int32), ("detector", ctypes.c_int32),
+                ("n_views", ctypes.c_int64), ("n_rows", ctypes.c_int64), ("n_cols", ctypes.c_int64),
+                ("src", ctypes.c_void_p), ("det_c", ctypes.c_void_p),
+                ("det_u", ctypes.c_void_p), ("det_v", ctypes.c_void_p),
+                ("nx", ctypes.c_int64), ("ny", ctypes.c_int64), ("nz", ctypes.c_int64),
+                ("origin", ctypes.c_double * 3), ("spacing", ctypes.c_double * 3),
+                ("device", ctypes.c_int32), ("reserved0", ctypes.c_int32),
+                ("plan", ctypes.POINTER(ctp_plan))]
+
+
+class ctp_geom_info(ctypes.Structure):
+    _fields_ = [("n_rays", ctypes.c_int64), ("n_vox", ctypes.c_int64), ("scratch_bytes", ctypes.c_int64),
+                ("adjoint_variant", ctypes.c_int32), ("brick", ctypes.c_int32 * 3),
+                ("view_groups", ctypes.c_int32), ("n_transposed_views", ctypes.c_int32),
+                ("collision_ratio", ctypes.c_double)]
+
+
+class CtpError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"{status_string(status)}: {detail}")
+        self.status = status
+        self.detail = detail
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load libctp.so (built by ``ray_forward_back_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise RuntimeError(f"libctp.so is not built ({path}); run python -m ray_forward_back_b200.build")
+        lib = ctypes.CDLL(path)
+        vp, i64 = ctypes.c_void_p, ctypes.c_int64
+        lib.ctp_geom_create.argtypes = [ctypes.POINTER(ctp_geom_desc), ctypes.POINTER(vp)]
+        lib.ctp_geom_create.restype = ctypes.c_int
+        lib.ctp_geom_destroy.argtypes = [vp]
+        lib.ctp_geom_destroy.restype = None
+        lib.ctp_geom_query.argtypes = [vp, ctypes.POINTER(ctp_geom_info)]
+        lib.ctp_geom_query.restype = ctypes.c_int
+        lib.ctp_forward.argtypes = [vp, vp, vp, vp]
+        lib.ctp_forward.restype = ctypes.c_int
+        lib.ctp_back.argtypes = [vp, vp, vp, vp]
+        lib.ctp_back.restype = ctypes.c_int
+        lib.ctp_count_updates.argtypes = [vp, ctypes.POINTER(i64), vp]
+        lib.ctp_count_updates.restype = ctypes.c_int
+        lib.ctp_status_string.argtypes = [ctypes.c_int]
+        lib.ctp_status_string.restype = ctypes.c_char_p
+        lib.ctp_last_error_detail.argtypes = []
+        lib.ctp_last_error_detail.restype = ctypes.c_char_p
+        lib.ctp_version.argtypes = []
+        lib.ctp_version.restype = ctypes.c_char_p
+        _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return load().ctp_status_string(status).decode()
+
+
+def last_error_detail() -> str:
+    return load().ctp_last_error_detail().decode()
+
+
+def _check(status: int):
+    if status != CTP_OK:
+        raise CtpError(status, last_error_detail())
+
+
+def _ptr(t) -> int:
+    if t is None:
+        return 0
+    if isinstance(t, int):
+        return t
+    return int(t.data_ptr())
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        import torch
+        return int(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return stream
+    return int(stream.cuda_stream)
+
+
+class _Desc:
+    """A ctp_geom_desc with the host arrays it points at kept alive."""
+
+    def __init__(self, geom, device: int = 0, plan: Optional[dict] = None):
+        self.arrays = [np.ascontiguousarray(a, dtype=np.float64) for a in
+                       (geom.src, geom.det_c, geom.det_u, geom.det_v)]
+        for a in self.arrays:
+            if a.shape != (geom.n_views, 3):
+                raise ValueError("per-view vectors must have shape (n_views, 3)")
+        d = ctp_geom_desc()
+        d.beam, d.detector = int(geom.beam), int(geom.detector)
+        d.n_views, d.n_rows, d.n_cols = int(geom.n_views), int(geom.n_rows), int(geom.n_cols)
+        d.src, d.det_c, d.det_u, d.det_v = [a.ctypes.data for a in self.arrays]
+        d.nx, d.ny, d.nz = int(geom.nx), int(geom.ny), int(geom.nz)
+        d.origin[:] = [float(x) for x in geom.origin]
+        d.spacing[:] = [float(x) for x in geom.spacing]
+        d.device = int(device)
+        self.plan = None
+        if plan:
+            p = ctp_plan()
+            p.adjoint_variant = int(plan.get("adjoint_variant", 0))
+            p.brick[:] = [int(x) for x in plan.get("brick", (0, 0, 0))]
+            p.view_groups = int(plan.get("view_groups", 0))
+            p.forward_layout = int(plan.get("forward_layout", 0))
+            self.plan = p
+            d.plan = ctypes.pointer(p)
+        self.desc = d
+
+
+def ctp_geom_create(geom, device: int = 0, plan: Optional[dict] = None) -> int:
+    """Validate and upload a geometry; returns the opaque handle."""
+    lib = load()
+    desc = _Desc(geom, device, plan)
+    h = ctypes.c_void_p()
+    _check(lib.ctp_geom_create(ctypes.byref(desc.desc), ctypes.byref(h)))
+    return int(h.value)
+
+
+def ctp_geom_destroy(handle: int) -> None:
+    if handle:
+        load().ctp_geom_destroy(handle)
+
+
+def ctp_geom_query(handle: int) -> dict:
+    info = ctp_geom_info()
+    _check(load().ctp_geom_query(handle, ctypes.byref(info)))
+    return {"n_rays": info.n_rays, "n_vox": info.n_vox, "scratch_bytes": info.scratch_bytes,
+            "adjoint_variant": info.adjoint_variant, "brick": tuple(info.brick), "view_groups": info.view_groups,
+            "n_transposed_views": info.n_transposed_views, "collision_ratio": info.collision_ratio}
+
+
+def ctp_forward(handle: int, vol, sino, stream=None) -> None:
+    _check(load().ctp_forward(handle, _ptr(vol), _ptr(sino), _stream_handle(stream)))
+
+
+def ctp_back(handle: int, sino, vol, stream=None) -> None:
+    _check(load().ctp_back(handle, _ptr(sino), _ptr(vol), _stream_handle(stream)))
+
+
+def ctp_count_updates(handle: int, stream=None) -> int:
+    n = ctypes.c_int64()
+    _check(load().ctp_count_updates(handle, ctypes.byref(n), _stream_handle(stream)))
+    return int(n.value)
+
+
+def ctp_version() -> str:
+    return load().ctp_version().decode()
+
+
+class Projector:
+    """Matched forward / back projector on one CUDA device.
+
+    ``forward(vol)`` takes a float32 CUDA tensor (nz, ny, nx) and returns the
+    sinogram (n_views, n_rows, n_cols); ``back(sino)`` the reverse.  Both run
+    on the current torch stream unless a stream is given, and never
+    synchronise.
+    """
+
+    def __init__(self, geom, device: int = 0, plan: Optional[dict] = None):
+        self.geom = geom
+        self.device = device
+        self.handle = ctp_geom_create(geom, device, plan)
+
+    def close(self):
+        if getattr(self, "handle", 0):
+            ctp_geom_destroy(self.handle)
+            self.handle = 0
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def info(self) -> dict:
+        return ctp_geom_query(self.handle)
+
+    def _check_tensor(self, t, shape, name):
+        import torch
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.float32 or not t.is_cuda:
+            raise TypeError(f"{name} must be a float32 CUDA tensor")
+        if tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous with shape {tuple(shape)}")
+
+    def forward(self, vol, out=None, stream=None):
+        import torch
+        self._check_tensor(vol, self.geom.vol_shape, "vol")
+        if out is None:
+            out = torch.empty(self.geom.sino_shape, dtype=torch.float32, device=vol.device)
+        self._check_tensor(out, self.geom.sino_shape, "out")
+        ctp_forward(self.handle, vol, out, stream)
+        return out
+
+    def back(self, sino, out=None, stream=None):
+        import torch
+        self._check_tensor(sino, self.geom.sino_shape, "sino")
+        if out is None:
+            out = torch.empty(self.geom.vol_shape, dtype=torch.float32, device=sino.device)
+        self._check_tensor(out, self.geom.vol_shape, "out")
+        ctp_back(self.handle, sino, out, stream)
+        return out
+
+    def count_updates(self, stream=None) -> int:
+        return ctp_count_updates(self.handle, stream)

@@ -1,0 +1,273 @@
+"""GPU parity: the CUDA projector pair against the FP64 oracle.
+
+Every case calls the library through its C ABI (ctypes binding) on seeded
+inputs.  Small and ragged geometries of every kind, and workloads 0 and 1,
+are compared element by element; the full-size workloads 2-4 are compared on
+sampled rays, on sparse sinograms whose back projection the oracle builds
+segment by segment, and through the adjoint identity.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from ray_forward_back_b200 import workloads as W
+from tests.gpu_helpers import (EPS32, adjoint_mismatch, check_back, check_forward, gpu_back, gpu_forward,
+                               oracle_chords, projector, rel_l2)
+from tests.helpers import small_geometries
+
+pytestmark = pytest.mark.gpu
+
+
+def ragged_geometries():
+    """Sizes that leave partial tiles everywhere: detector tiles are 32 columns
+    x 8 rows, adjoint bricks 64x64x4 (parallel) and 32x32x16 (cone)."""
+    gs = dict(small_geometries())
+    gs["parallel_ragged"] = W.make_parallel(70, 45, 33, 9, 37, 77, pitch_u=1.1, pitch_v=0.9,
+                                            spacing=(1.0, 1.1, 0.95), start=0.05)
+    g = W.make_cone(48, 40, 36, 7, 29, 51, sid=120.0, sdd=210.0, pitch_u=1.9, pitch_v=2.1,
+                    spacing=(1.0, 0.9, 1.1), start=0.17)
+    g.det_c = g.det_c + np.array([0.0123, -0.0211, 0.0377])
+    gs["cone_ragged"] = g
+    pu = W.helical_fan_pitch(61, 30.0, 70.0, 120.0)
+    g = W.make_cone(56, 50, 24, 21, 13, 61, sid=70.0, sdd=120.0, pitch_u=pu, pitch_v=1.3,
+                    spacing=(1.0, 1.05, 0.95), detector=W.DET_CYLINDRICAL, z_start=-9.3, z_end=8.9, start=0.11)
+    gs["helical_ragged"] = g
+    # parallel beam whose rays tilt out of the slice planes (3-D traversal)
+    src, dc, du, dv = W.parallel_trajectory(6, start=0.2)
+    src[:, 2] = 0.31
+    gs["parallel_tilted"] = W.Geometry(W.BEAM_PARALLEL, W.DET_FLAT, 21, 35, src, dc, du, dv, 30, 28, 26,
+                                       W.centred_origin(30, 28, 26), (1.0, 1.0, 1.0))
+    return gs
+
+
+def _local_len(P, geom):
+    b = np.array(P.info()["brick"], dtype=np.float64) * np.array(geom.spacing)
+    return float(np.linalg.norm(b))
+
+
+def _seeded_volume(geom, seed):
+    rng = np.random.default_rng(seed)
+    return rng.random(geom.vol_shape).astype(np.float32)
+
+
+@pytest.mark.parametrize("name", sorted(ragged_geometries()))
+def test_forward_matches_oracle_small(name):
+    g = ragged_geometries()[name]
+    vol = _seeded_volume(g, 1)
+    P = projector(g)
+    y = gpu_forward(P, vol)
+    check_forward(y, oracle.forward(g, vol), oracle_chords(g), min(g.spacing), name)
+
+
+@pytest.mark.parametrize("name", sorted(ragged_geometries()))
+def test_back_matches_oracle_small(name):
+    g = ragged_geometries()[name]
+    rng = np.random.default_rng(2)
+    sino = rng.random(g.sino_shape).astype(np.float32)
+    P = projector(g)
+    x = gpu_back(P, sino)
+    check_back(x, oracle.back(g, sino), oracle.back(g, np.abs(sino), power=0), _local_len(P, g), name)
+
+
+@pytest.mark.parametrize("name", sorted(ragged_geometries()))
+def test_adjoint_identity_small(name):
+    g = ragged_geometries()[name]
+    P = projector(g)
+    assert adjoint_mismatch(P, g) <= 1e-5
+
+
+@pytest.mark.parametrize("index", [0, 1])
+def test_workload_full_parity(index):
+    """Workloads 0 and 1 element by element, forward and back."""
+    wl = W.workload(index)
+    g = wl.geom
+    vol = wl.phantom()
+    sino = wl.sinogram()
+    P = projector(g)
+    y = gpu_forward(P, vol)
+    check_forward(y, oracle.forward(g, vol), oracle_chords(g), min(g.spacing), wl.name)
+    x = gpu_back(P, sino)
+    check_back(x, oracle.back(g, sino), oracle.back(g, sino, power=0), _local_len(P, g), wl.name)
+    assert adjoint_mismatch(P, g) <= 1e-5
+
+
+def test_workload0_axis_views_are_plain_sums():
+    """Views at 0 and 90 degrees of workload 0 pass through voxel centres: the
+    GPU result equals the numpy sum along the axis to FP32 rounding."""
+    wl = W.workload(0)
+    vol = wl.phantom()
+    P = projector(wl.geom)
+    y = gpu_forward(P, vol)
+    np.testing.assert_allclose(y[0], vol.astype(np.float64).sum(axis=2), rtol=2e-6)
+    np.testing.assert_allclose(y[32], vol.astype(np.float64).sum(axis=1)[:, ::-1], rtol=2e-6)
+
+
+@pytest.mark.parametrize("name", ["parallel_ragged", "cone_ragged", "helical_ragged"])
+def test_update_count(name):
+    g = ragged_geometries()[name]
+    P = projector(g)
+    n_gpu = P.count_updates()
+    n_ref = oracle.count_updates(g)
+    assert abs(n_gpu - n_ref) <= 1e-3 * n_ref, (n_gpu, n_ref)
+
+
+def _sample_rays(geom, n, rng):
+    return (rng.integers(0, geom.n_views, n), rng.integers(0, geom.n_rows, n), rng.integers(0, geom.n_cols, n))
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("index", [2, 3, 4])
+def test_workload_full_size_sampled(index):
+    """Full-size workloads: the whole GPU sinogram, checked on 1500 sampled
+    rays against the oracle, with the per-ray criterion."""
+    import torch
+    wl = W.workload(index)
+    g = wl.geom
+    vol = wl.phantom()
+    P = projector(g)
+    y = P.forward(torch.from_numpy(vol).cuda())
+    rng = np.random.default_rng(100 + index)
+    vs, rs, cs = _sample_rays(g, 1500, rng)
+    got = y[torch.from_numpy(vs).cuda(), torch.from_numpy(rs).cuda(), torch.from_numpy(cs).cuda()].cpu().numpy()
+    ref = oracle.forward_rays(g, vol, vs, rs, cs)
+    chord = oracle.forward_rays(g, np.ones(g.vol_shape, np.float32), vs, rs, cs)
+    ymax = float(y.abs().max().item())
+    err = np.abs(got - ref)
+    crossing = (chord >= min(g.spacing)) & (np.abs(ref) >= 1e-3 * ymax)
+    assert crossing.sum() > 100
+    assert float((err[crossing] / np.abs(ref[crossing])).max()) <= 1e-4
+    assert np.all(err <= 1e-4 * np.abs(ref) + 1e-6 * ymax)
+    assert rel_l2(got, ref) <= 1e-5
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("index", [2, 3, 4])
+def test_workload_full_size_sparse_back(index):
+    """Full-size adjoint on a sinogram with 24 non-zero rays: the result is the
+    weighted sum of those rays' oracle coefficient lists, voxel by voxel, and
+    zero elsewhere."""
+    import torch
+    wl = W.workload(index)
+    g = wl.geom
+    P = projector(g)
+    rng = np.random.default_rng(200 + index)
+    sino = torch.zeros(g.sino_shape, dtype=torch.float32, device="cuda")
+    expect = {}
+    count = {}
+    k = 0
+    while k < 24:
+        v, r, c = int(rng.integers(g.n_views)), int(rng.integers(g.n_rows)), int(rng.integers(g.n_cols))
+        idx, w = oracle.ray_segments(g, v, r, c)
+        if idx.size < 10 or sino[v, r, c].item() != 0:
+            continue
+        val = float(np.float32(rng.uniform(0.5, 2.0)))
+        sino[v, r, c] = val
+        for i, wi in zip(idx.tolist(), w.tolist()):
+            expect[i] = expect.get(i, 0.0) + wi * val
+            count[i] = count.get(i, 0.0) + val
+        k += 1
+    x = P.back(sino).reshape(-1)
+    keys = np.array(sorted(expect))
+    ref = np.array([expect[i] for i in keys])
+    cnt = np.array([count[i] for i in keys])
+    got = x[torch.from_numpy(keys).cuda()].double().cpu().numpy()
+    tau = 8 * EPS32 * float(np.linalg.norm(np.array(P.info()["brick"]) * np.array(g.spacing)))
+    assert np.all(np.abs(got - ref) <= 1e-4 * np.abs(ref) + tau * cnt)
+    # nothing outside the rays' support beyond FP32 crumbs
+    mask = torch.ones(g.n_vox, dtype=torch.bool, device="cuda")
+    mask[torch.from_numpy(keys).cuda()] = False
+    outside = x[mask].abs().max().item()
+    assert outside <= tau * 2.0
+    assert rel_l2(got, ref) <= 1e-5
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("index", [2, 3, 4])
+def test_workload_full_size_adjoint_identity(index):
+    wl = W.workload(index)
+    P = projector(wl.geom)
+    assert adjoint_mismatch(P, wl.geom) <= 1e-5
+
+
+def _ladder():
+    rows = []
+    path = __file__.replace("test_parity_gpu.py", "golden/fp32_clipping_error_ladder.txt")
+    for line in open(path):
+        if line.strip() and not line.startswith("#"):
+            sid, err = line.split()
+            rows.append((float(sid), float(err)))
+    return rows
+
+
+@pytest.mark.parametrize("sid,fp32_err", _ladder())
+def test_fp64_setup_beats_fp32_clipping_ladder(sid, fp32_err):
+    """64^3 cone scan, 16 views, at growing source distance.  With FP32
+    clipping the pages measure max relative errors 3e-5 / 9e-3 / 4e-2; the
+    FP64 setup here must stay within 1e-4 at every distance."""
+    sdd = 2 * sid if sid <= 1e3 else sid + 1000.0
+    wl = W.workload(1)
+    g = W.make_cone(64, 64, 64, 16, 128, 128, sid=sid, sdd=sdd, pitch_u=sdd / sid * 0.5, pitch_v=sdd / sid * 0.5)
+    vol = wl.phantom()
+    P = projector(g)
+    y = gpu_forward(P, vol).astype(np.float64)
+    ref = oracle.forward(g, vol)
+    m = np.abs(ref) >= 1e-3 * np.abs(ref).max()
+    worst = float((np.abs(y - ref)[m] / np.abs(ref[m])).max())
+    assert worst <= 1e-4
+    if sid >= 1e5:
+        assert worst < fp32_err / 10
+
+
+def test_rays_missing_the_volume_are_zero_and_back_is_zero():
+    g = W.make_parallel(16, 16, 16, 3, 4, 6)
+    g.det_c = g.det_c + np.array([0.0, 0.0, 100.0])  # detector rows far above the volume
+    P = projector(g)
+    y = gpu_forward(P, np.ones(g.vol_shape, np.float32))
+    assert np.all(y == 0)
+    x = gpu_back(P, np.ones(g.sino_shape, np.float32))
+    assert np.all(x == 0)
+
+
+def test_degenerate_sizes():
+    """Single voxel / single pixel / single view cases against the oracle."""
+    cases = [
+        W.make_parallel(1, 1, 1, 1, 1, 1, start=0.3),
+        W.make_parallel(1, 3, 1, 2, 1, 5, pitch_u=0.5, start=0.4),
+        W.make_cone(2, 1, 3, 3, 2, 1, sid=10.0, sdd=15.0, pitch_u=0.4, pitch_v=0.6, start=0.2),
+    ]
+    rng = np.random.default_rng(4)
+    for g in cases:
+        vol = rng.random(g.vol_shape).astype(np.float32) + 0.5
+        P = projector(g)
+        y = gpu_forward(P, vol)
+        ref = oracle.forward(g, vol)
+        np.testing.assert_allclose(y, ref, rtol=1e-5, atol=1e-6)
+        sino = rng.random(g.sino_shape).astype(np.float32)
+        np.testing.assert_allclose(gpu_back(P, sino), oracle.back(g, sino), rtol=1e-5, atol=1e-6)
+
+
+@pytest.mark.parametrize("plan", [{"forward_layout": 1}, {"forward_layout": 2}, {"brick": (8, 8, 8)},
+                                  {"brick": (16, 8, 4), "view_groups": 3}, {"view_groups": 1}])
+def test_plan_overrides_keep_results(plan):
+    """Layout, brick and view-group choices change scheduling, not values."""
+    g = ragged_geometries()["cone_ragged"]
+    vol = _seeded_volume(g, 5)
+    rng = np.random.default_rng(6)
+    sino = rng.random(g.sino_shape).astype(np.float32)
+    P = projector(g, plan)
+    check_forward(gpu_forward(P, vol), oracle.forward(g, vol), oracle_chords(g), min(g.spacing), str(plan))
+    check_back(gpu_back(P, sino), oracle.back(g, sino), oracle.back(g, sino, power=0), _local_len(P, g), str(plan))
+
+
+def test_host_pointer_is_rejected():
+    import torch
+    from ray_forward_back_b200 import ctp
+    g = small_geometries()["parallel"]
+    P = projector(g)
+    host = torch.zeros(g.vol_shape, dtype=torch.float32)
+    dev = torch.zeros(g.sino_shape, dtype=torch.float32, device="cuda")
+    with pytest.raises(ctp.CtpError) as ei:
+        ctp.ctp_forward(P.handle, host.data_ptr(), dev.data_ptr())
+    assert ei.value.status == ctp.CTP_ERR_INVALID_ARGUMENT
