@@ -125,11 +125,23 @@ def cpu_oracle_sample(wl, n_views_sample=1):
     return 2 * U / dt, dt, 2 * U, desc
 
 
+def select_workload(args):
+    import dataclasses
+
+    from ray_forward_back_b200 import workloads as W
+    wl = W.workload(args.workload)
+    if args.views and args.views < wl.geom.n_views:
+        views = np.linspace(0, wl.geom.n_views - 1, args.views).round().astype(np.int64)
+        wl = dataclasses.replace(wl, geom=wl.geom.subset_views(views),
+                                 name=f"{wl.name} (views subset: {args.views})")
+    return wl
+
+
 def run_reference(args, rank, world):
     from ray_forward_back_b200 import workloads as W
     if rank != 0:
         return 0
-    wl = W.workload(args.workload)
+    wl = select_workload(args)
     vals = []
     for _ in range(args.warmup):
         cpu_oracle_sample(wl, 1)
@@ -157,7 +169,7 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    wl = W.workload(args.workload)
+    wl = select_workload(args)
     g = wl.geom
     P = ctp.Projector(g, device=local_rank)
     info = P.info()
@@ -297,6 +309,8 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", type=int, default=4)
+    ap.add_argument("--views", type=int, default=0,
+                    help="use this many evenly spaced views of the workload (0 = all); for profiling")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -33,18 +33,22 @@ def _stale() -> bool:
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    if not force and not _stale():
+def build(force: bool = False, verbose_ptxas: bool = False, out: str = None, defines=()) -> str:
+    """Compile the library; ``defines`` are extra -D tuning macros and ``out``
+    another output path (the default build goes in-tree)."""
+    lib = out or LIB
+    if not force and out is None and not defines and not _stale():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [nvcc_path(), "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
            "-Xcompiler", "-fPIC", "-shared", "-I", INCLUDE, "-o", tmp]
     if verbose_ptxas:
         cmd += ["-Xptxas", "-v"]
+    cmd += [f"-D{d}" for d in defines]
     cmd += [os.path.join(CSRC, s) for s in SOURCES]
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":

@@ -283,6 +283,16 @@ ctp_status build_views(const ctp_geom_desc *d, std::vector<ViewRec> &views, std:
         return fail(CTP_ERR_OUT_OF_RANGE, "view %lld: no endpoint within 1e6 voxels of the volume centre",
                     (long long)v);
     }
+    // extent of one voxel's projection, used to bound the rays per voxel
+    if (d->beam == CTP_BEAM_PARALLEL) {
+      for (int i = 0; i < 2; ++i)
+        V.vox_ext[i] = std::fabs(V.minv[3 * i]) * d->spacing[0] + std::fabs(V.minv[3 * i + 1]) * d->spacing[1] +
+                       std::fabs(V.minv[3 * i + 2]) * d->spacing[2];
+    } else if (d->detector == CTP_DET_FLAT) {
+      for (int i = 0; i < 3; ++i)
+        V.vox_ext[i] = std::fabs(V.minv[3 * i]) * d->spacing[0] + std::fabs(V.minv[3 * i + 1]) * d->spacing[1] +
+                       std::fabs(V.minv[3 * i + 2]) * d->spacing[2];
+    }
     // forward gather layout: y-fastest copy when the column step runs mostly along y
     const double ux = std::fabs(du[0] / d->spacing[0]), uy = std::fabs(du[1] / d->spacing[1]),
                  uz = std::fabs(du[2] / d->spacing[2]);
@@ -293,12 +303,13 @@ ctp_status build_views(const ctp_geom_desc *d, std::vector<ViewRec> &views, std:
   return CTP_OK;
 }
 
-void plan_back(ctp_geom *g, const ctp_plan *plan) {
+void plan_back(ctp_geom *g, const ctp_plan *plan, int sm_count) {
   int b[3];
+  // measured on B200: flat, wide bricks amortise the per-ray FP64 entry best
   if (g->beam == CTP_BEAM_PARALLEL) {
-    b[0] = 64, b[1] = 64, b[2] = 4;
+    b[0] = 128, b[1] = 64, b[2] = 2;
   } else {
-    b[0] = 32, b[1] = 32, b[2] = 16;
+    b[0] = 64, b[1] = 64, b[2] = 4;
   }
   if (plan)
     for (int k = 0; k < 3; ++k)
@@ -315,9 +326,16 @@ void plan_back(ctp_geom *g, const ctp_plan *plan) {
     nb *= p.nbrick[k];
   }
   p.pitch_x = b[0] + 1;
-  const int64_t target = 148 * 3 * 2;  // two waves of three resident CTAs per SM
+  // Resident CTAs per SM: shared memory (brick + staged footprints + the
+  // 1 KB the runtime reserves per CTA) and registers (three 256-thread CTAs).
+  const int64_t per_cta = (int64_t)ctp::back_brick_smem_bytes(p.brick) + 6 * 1024;
+  const int64_t per_sm = std::max<int64_t>(1, std::min<int64_t>(3, (228 * 1024) / per_cta));
+  const int64_t slots = (int64_t)sm_count * per_sm;
+  // at least four waves of CTAs, so the last partial wave costs little:
+  // split the views over groups when there are too few bricks
   int groups = 1;
-  if (nb < target) groups = (int)std::min<int64_t>((target + nb - 1) / nb, std::max<int64_t>(1, g->n_views / 4));
+  if (nb < 4 * slots)
+    groups = (int)std::min<int64_t>((4 * slots + nb - 1) / nb, std::max<int64_t>(1, (g->n_views + 7) / 8));
   if (plan && plan->view_groups > 0) groups = (int)std::min<int64_t>(plan->view_groups, g->n_views);
   int vpg = (int)((g->n_views + groups - 1) / groups);
   groups = (int)((g->n_views + vpg - 1) / vpg);
@@ -430,17 +448,20 @@ ctp_status ctp_geom_create(const ctp_geom_desc *desc, ctp_geom **out) {
   f.any_transposed = g->n_transposed > 0;
   const ctp_plan *plan = desc->plan;
   g->adjoint_variant = CTP_ADJOINT_BRICK;
-  plan_back(g, plan);
-  if (ctp::back_brick_smem_bytes(g->back.brick) > 227 * 1024) {
-    delete g;
-    return fail(CTP_ERR_INVALID_ARGUMENT, "adjoint brick needs more than 227 KB of shared memory");
-  }
 
   DeviceGuard dg(g->device);
-  if (dg.err != cudaSuccess) {
-    ctp_status s = cuda_fail(dg.err, "cudaSetDevice");
+  int sm_count = 0;
+  cudaError_t de = dg.err;
+  if (de == cudaSuccess) de = cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, g->device);
+  if (de != cudaSuccess) {
+    ctp_status s = cuda_fail(de, "device query");
     delete g;
     return s;
+  }
+  plan_back(g, plan, sm_count);
+  if (ctp::back_brick_smem_bytes(g->back.brick) > 200 * 1024) {
+    delete g;
+    return fail(CTP_ERR_INVALID_ARGUMENT, "adjoint brick needs more than 200 KB of shared memory");
   }
   auto alloc = [&](void **p, size_t bytes, const char *what) -> ctp_status {
     cudaError_t e = cudaMalloc(p, bytes);

@@ -27,6 +27,8 @@ struct ViewRec {
   double vhat[3];     // unit row direction
   double rcp_dir[3];  // parallel: 1 / (direction in voxel units), +-inf where 0
   double minv[9];     // footprint matrix: parallel flat [du dv s]^-1, cone flat [p00-s du dv]^-1
+  double vox_ext[3];  // one voxel's projected extent: parallel (columns, rows, -);
+                      // cone flat: sum_k |minv row i, k| * spacing_k for rows i = 0, 1, 2
   double R, gam0, dgam, axial0, vlen;
   int32_t layout;     // forward gather: 0 = x-fastest volume, 1 = y-fastest copy
   int32_t full_footprint;  // 1: the footprint test cannot bound this view; scan all pixels

@@ -38,10 +38,39 @@
 namespace ctp {
 namespace {
 
+// Tuning knobs (compile-time; the defaults are the measured choices).
+#ifndef CTP_FWD_MIN_BLOCKS
+#define CTP_FWD_MIN_BLOCKS 5
+#endif
+#ifndef CTP_BACK_MIN_BLOCKS
+#define CTP_BACK_MIN_BLOCKS 3
+#endif
+#ifndef CTP_WALK2_UNROLL
+#define CTP_WALK2_UNROLL 4
+#endif
+#ifndef CTP_WALK3_UNROLL
+#define CTP_WALK3_UNROLL 2
+#endif
+#ifndef CTP_LANE_WALK2_UNROLL
+#define CTP_LANE_WALK2_UNROLL 8
+#endif
+constexpr int kWalk2Unroll = CTP_WALK2_UNROLL;
+constexpr int kLaneWalk2Unroll = CTP_LANE_WALK2_UNROLL;
+constexpr int kWalk3Unroll = CTP_WALK3_UNROLL;
+
 constexpr int kFwdCols = 32;  // threads along detector columns per block
 constexpr int kFwdRows = 8;   // detector rows per block (row band height)
 constexpr int kBackThreads = 256;
-constexpr int kBackChunk = 8;  // views whose footprints are staged together
+#ifndef CTP_BACK_WARP_WALK
+#define CTP_BACK_WARP_WALK 0
+#endif
+#ifndef CTP_BACK_ALIGN
+#define CTP_BACK_ALIGN 0
+#endif
+#ifndef CTP_BACK_STAGE
+#define CTP_BACK_STAGE 64
+#endif
+constexpr int kBackStage = CTP_BACK_STAGE;  // views per fixed-point accumulation stage of the adjoint
 
 struct Ray {
   double A[3];    // parameter origin, voxel units relative to the volume min corner
@@ -169,48 +198,215 @@ __device__ __forceinline__ void entry(const Ray& R, double t_in, double t_out, c
       W.N[k] = 0;
       W.step[k] = 1;
       W.l0[k] = CUDART_INF_F;
-      W.inc[k] = 0.f;
+      W.inc[k] = CUDART_INF_F;
     }
   }
   W.L = (float)((t_out - t_in) * R.len);
 }
 
-// FP32 Siddon walk: visits (offset, physical segment length) for every voxel
-// of the clipped segment in order; offsets advance by the signed strides.
+template <typename T>
+__device__ __forceinline__ T pick3(int k, T a0, T a1, T a2) {
+  return k == 0 ? a0 : (k == 1 ? a1 : a2);
+}
+
+// Axis roles of a walk: a = major (crossed most often, smallest spacing
+// between crossings), c = the minor axis crossed least often, b = the other.
+__device__ __forceinline__ void walk_axes(const Walk& W, int& a, int& b, int& c) {
+  const float i0 = W.inc[0], i1 = W.inc[1], i2 = W.inc[2];
+  a = (i0 <= i1 && i0 <= i2) ? 0 : (i1 <= i2 ? 1 : 2);
+  if (a == 0) {
+    b = i1 <= i2 ? 1 : 2;
+    c = 3 - b;
+  } else if (a == 1) {
+    b = i0 <= i2 ? 0 : 2;
+    c = 2 - b;
+  } else {
+    b = i0 <= i1 ? 0 : 1;
+    c = 1 - b;
+  }
+}
+
+// FP32 Siddon walk in major-axis slabs, one lane per ray (lanes run
+// independently).  Each slab between two successive planes of the major axis
+// a holds at most one crossing of each minor axis, so it is one, two or three
+// segments.  The walk is branch-free: every slab makes the same visit calls,
+// a segment that does not exist in that slab being visited with length 0 at
+// a valid offset.  visit(offset, physical length) is called for every segment
+// (zero-length ones included);
+// offsets move by the signed strides s0, s1, s2 of axes x, y, z.  Crossings
+// are l0 + j * inc from exact integers j and the FP64 counts N cap every
+// axis, so offsets never leave the clipped box; a minor crossing that rounds
+// past the exit is dropped (its error is below one ulp of the walk length).
 template <typename Off, typename Visit>
-__device__ __forceinline__ void walk(const Walk& W, Off off, Off sx, Off sy, Off sz, Visit&& visit) {
-  float nx = W.N[0] > 0 ? W.l0[0] : CUDART_INF_F;
-  float ny = W.N[1] > 0 ? W.l0[1] : CUDART_INF_F;
-  float nz = W.N[2] > 0 ? W.l0[2] : CUDART_INF_F;
-  int jx = 0, jy = 0, jz = 0;
-  const int total = W.N[0] + W.N[1] + W.N[2];
+__device__ __forceinline__ void walk_lane(const Walk& W, Off off, Off s0, Off s1, Off s2, Visit&& visit) {
+  int a, b, c;
+  walk_axes(W, a, b, c);
+  const int Na = pick3(a, W.N[0], W.N[1], W.N[2]);
+  const int Nb = pick3(b, W.N[0], W.N[1], W.N[2]);
+  const int Nc = pick3(c, W.N[0], W.N[1], W.N[2]);
+  const float l0a = pick3(a, W.l0[0], W.l0[1], W.l0[2]), inca = pick3(a, W.inc[0], W.inc[1], W.inc[2]);
+  const float l0b = pick3(b, W.l0[0], W.l0[1], W.l0[2]), incb = pick3(b, W.inc[0], W.inc[1], W.inc[2]);
+  const float l0c = pick3(c, W.l0[0], W.l0[1], W.l0[2]), incc = pick3(c, W.inc[0], W.inc[1], W.inc[2]);
+  const Off sa = pick3(a, s0, s1, s2), sb = pick3(b, s0, s1, s2), sc = pick3(c, s0, s1, s2);
   const float L = W.L;
+  const float fNb = (float)Nb, fNc = (float)Nc;
+  float tb = Nb > 0 ? l0b : CUDART_INF_F;
+  float fjb = 1.f;
   float cur = 0.f;
-  for (int it = 0; it < total; ++it) {
-    const float m = fminf(fminf(nx, ny), fminf(nz, L));
-    visit(off, m - cur);
-    cur = m;
-    if (nx <= ny && nx <= nz) {
-      off += sx;
-      ++jx;
-      nx = jx < W.N[0] ? fmaf((float)jx, W.inc[0], W.l0[0]) : CUDART_INF_F;
-    } else if (ny <= nz) {
-      off += sy;
-      ++jy;
-      ny = jy < W.N[1] ? fmaf((float)jy, W.inc[1], W.l0[1]) : CUDART_INF_F;
-    } else {
-      off += sz;
-      ++jz;
-      nz = jz < W.N[2] ? fmaf((float)jz, W.inc[2], W.l0[2]) : CUDART_INF_F;
+  if (Nc == 0) {
+#pragma unroll kLaneWalk2Unroll
+    for (int s = 0; s < Na; ++s) {
+      const float tx = fminf(fmaf((float)s, inca, l0a), L);
+      const bool cb = tb < tx;
+      const float m1 = fmaxf(fminf(tb, tx), cur);
+      const Off o2 = off + (cb ? sb : (Off)0);
+      visit(off, m1 - cur);
+      visit(o2, tx - m1);
+      off = o2 + sa;
+      tb = cb ? (fjb < fNb ? fmaf(fjb, incb, l0b) : CUDART_INF_F) : tb;
+      fjb += cb ? 1.f : 0.f;
+      cur = tx;
+    }
+    const bool cb = tb < L;
+    const float m1 = fmaxf(fminf(tb, L), cur);
+    visit(off, m1 - cur);
+    visit(off + (cb ? sb : (Off)0), L - m1);
+  } else {
+    float tc = l0c;
+    float fjc = 1.f;
+#pragma unroll kWalk3Unroll
+    for (int s = 0; s <= Na; ++s) {
+      const float tx = s < Na ? fminf(fmaf((float)s, inca, l0a), L) : L;
+      const bool cb = tb < tx, cc = tc < tx;
+      const float m1 = fmaxf(fminf(fminf(tb, tc), tx), cur);
+      const float m2 = fmaxf(fminf(fmaxf(tb, tc), tx), m1);
+      const Off db = cb ? sb : (Off)0, dc = cc ? sc : (Off)0;
+      const Off o2 = off + (tb <= tc ? db : dc);
+      const Off o3 = off + db + dc;
+      visit(off, m1 - cur);
+      visit(o2, m2 - m1);
+      visit(o3, tx - m2);
+      tb = cb ? (fjb < fNb ? fmaf(fjb, incb, l0b) : CUDART_INF_F) : tb;
+      fjb += cb ? 1.f : 0.f;
+      tc = cc ? (fjc < fNc ? fmaf(fjc, incc, l0c) : CUDART_INF_F) : tc;
+      fjc += cc ? 1.f : 0.f;
+      off = o3 + sa;
+      cur = tx;
     }
   }
-  visit(off, L - cur);
+}
+
+// FP32 Siddon walk in major-axis slabs, warp-synchronous.
+//
+// The major axis a is the one the ray crosses most often (smallest spacing
+// between crossings), so each slab between two successive a-planes holds at
+// most one crossing of each minor axis b, c: a slab is one, two or three
+// segments, visited in order with predicated (not branched) extra segments.
+// Lanes are aligned on absolute slab positions inside the box: a lane whose
+// ray enters the box further along the major axis waits that many steps, so
+// at every step all lanes of the warp (neighbouring rays) sit in the same
+// slab and touch neighbouring voxels.  visit(offset, physical length) is
+// called for every segment (zero-length ones included); offsets move by the
+// signed strides s0, s1, s2 of axes x, y, z.  Crossings are l0 + j * inc from
+// exact integers j, and the FP64 counts N cap every axis, so offsets never
+// leave the clipped box; a minor crossing that rounds past the exit is
+// dropped (its error is below one ulp of the walk length).
+//
+// All 32 lanes must call this together; lanes without a ray pass active = false.
+template <bool kAlign, typename Off, typename Visit>
+__device__ __forceinline__ void walk(bool active, const Walk& W, const int lo[3], const int hi[3], Off off, Off s0,
+                                     Off s1, Off s2, Visit&& visit) {
+  constexpr unsigned kFull = 0xffffffffu;
+  const float i0 = W.inc[0], i1 = W.inc[1], i2 = W.inc[2];
+  int a, b, c;
+  walk_axes(W, a, b, c);
+  const int Na = active ? pick3(a, W.N[0], W.N[1], W.N[2]) : -1;
+  const int Nb = pick3(b, W.N[0], W.N[1], W.N[2]);
+  const int Nc = pick3(c, W.N[0], W.N[1], W.N[2]);
+  const float l0a = pick3(a, W.l0[0], W.l0[1], W.l0[2]), inca = pick3(a, i0, i1, i2);
+  const float l0b = pick3(b, W.l0[0], W.l0[1], W.l0[2]), incb = pick3(b, i0, i1, i2);
+  const float l0c = pick3(c, W.l0[0], W.l0[1], W.l0[2]), incc = pick3(c, i0, i1, i2);
+  const Off sa = pick3(a, s0, s1, s2), sb = pick3(b, s0, s1, s2), sc = pick3(c, s0, s1, s2);
+
+  // slab alignment: entry position along the major axis in travel direction
+  const int ia = pick3(a, W.i[0], W.i[1], W.i[2]);
+  const int p = pick3(a, W.step[0], W.step[1], W.step[2]) > 0 ? ia - pick3(a, lo[0], lo[1], lo[2])
+                                                               : pick3(a, hi[0], hi[1], hi[2]) - 1 - ia;
+  const int span_plain = __reduce_max_sync(kFull, Na);
+  if (span_plain < 0) return;  // no lane has a ray
+  int d = 0, kmax = span_plain;
+  if (kAlign) {
+    const int pmin = __reduce_min_sync(kFull, active ? p : 0x7fffffff);
+    d = active ? p - pmin : 0;
+    const int span_aligned = __reduce_max_sync(kFull, active ? d + Na : -1);
+    // alignment only pays while it does not stretch the warp's loop much
+    if (span_aligned <= 2 * span_plain + 8) kmax = span_aligned;
+    else d = 0;
+  }
+
+  const float L = W.L;
+  const float fNb = (float)Nb, fNc = (float)Nc;
+  float tb = Nb > 0 ? l0b : CUDART_INF_F;
+  float fjb = 1.f;
+  float cur = 0.f;
+  if (!__any_sync(kFull, active && Nc > 0)) {
+    // no lane crosses a second minor axis: at most two segments per slab
+#pragma unroll kWalk2Unroll
+    for (int k = 0; k <= kmax; ++k) {
+      const int s = k - d;
+      const bool on = s >= 0 && s <= Na;
+      const float tx = s < Na ? fminf(fmaf((float)s, inca, l0a), L) : L;
+      const bool cb = on && tb < tx;
+      const float m1 = fmaxf(fminf(tb, tx), cur);
+      if (on) visit(off, m1 - cur);
+      if (cb) visit(off + sb, tx - m1);
+      if (on) {
+        off += (cb ? sb : (Off)0) + sa;
+        cur = tx;
+      }
+      if (cb) {
+        tb = fjb < fNb ? fmaf(fjb, incb, l0b) : CUDART_INF_F;
+        fjb += 1.f;
+      }
+    }
+  } else {
+    // up to three segments per slab
+    float tc = Nc > 0 ? l0c : CUDART_INF_F;
+    float fjc = 1.f;
+#pragma unroll kWalk3Unroll
+    for (int k = 0; k <= kmax; ++k) {
+      const int s = k - d;
+      const bool on = s >= 0 && s <= Na;
+      const float tx = s < Na ? fminf(fmaf((float)s, inca, l0a), L) : L;
+      const bool cb = on && tb < tx, cc = on && tc < tx;
+      const float m1 = fmaxf(fminf(fminf(tb, tc), tx), cur);
+      const float m2 = fmaxf(fminf(fmaxf(tb, tc), tx), m1);
+      const Off db = cb ? sb : (Off)0, dc = cc ? sc : (Off)0;
+      const Off o2 = off + (tb <= tc ? db : dc);
+      const Off o3 = off + db + dc;
+      if (on) visit(off, m1 - cur);
+      if (cb || cc) visit(o2, m2 - m1);
+      if (cb && cc) visit(o3, tx - m2);
+      if (on) {
+        off = o3 + sa;
+        cur = tx;
+      }
+      if (cb) {
+        tb = fjb < fNb ? fmaf(fjb, incb, l0b) : CUDART_INF_F;
+        fjb += 1.f;
+      }
+      if (cc) {
+        tc = fjc < fNc ? fmaf(fjc, incc, l0c) : CUDART_INF_F;
+        fjc += 1.f;
+      }
+    }
+  }
 }
 
 // ------------------------------------------------------------------ forward --
 
 template <typename Off>
-__global__ void __launch_bounds__(kFwdCols* kFwdRows) forward_kernel(FwdLaunch P, const ViewRec* __restrict__ views,
+__global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_FWD_MIN_BLOCKS) forward_kernel(FwdLaunch P, const ViewRec* __restrict__ views,
                                                                      const double* __restrict__ trig,
                                                                      const float* __restrict__ vol,
                                                                      const float* __restrict__ volT,
@@ -222,29 +418,28 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows) forward_kernel(FwdLaunch P
   const int ct = rem - v * P.n_col_tiles;
   const int c = ct * kFwdCols + threadIdx.x;
   const int r = band * kFwdRows + threadIdx.y;
-  if (c >= P.dims.n_cols || r >= P.dims.n_rows) return;
+  const bool valid = c < P.dims.n_cols && r < P.dims.n_rows;
 
   const ViewRec& V = views[v];
   Ray R;
-  make_ray(V, P.vol, trig, P.dims, v, r, c, R);
+  make_ray(V, P.vol, trig, P.dims, v, valid ? r : 0, valid ? c : 0, R);
   const int lo[3] = {0, 0, 0};
   const int hi[3] = {P.vol.n[0], P.vol.n[1], P.vol.n[2]};
-  double t_in, t_out;
+  double t_in = 0.0, t_out = 0.0;
+  const bool hit = valid && clip(R, lo, hi, t_in, t_out);
+  Walk W = {};
+  if (hit) entry(R, t_in, t_out, lo, hi, W);
+  const Off nx = P.vol.n[0], ny = P.vol.n[1];
+  const bool yfast = V.layout != 0;
+  const float* __restrict__ base = yfast ? volT : vol;
+  const Off sx = yfast ? ny : (Off)1;
+  const Off sy = yfast ? (Off)1 : nx;
+  const Off sz = nx * ny;
+  const Off off = (Off)W.i[2] * sz + (Off)W.i[1] * sy + (Off)W.i[0] * sx;
   float acc = 0.f;
-  if (clip(R, lo, hi, t_in, t_out)) {
-    Walk W;
-    entry(R, t_in, t_out, lo, hi, W);
-    const Off nx = P.vol.n[0], ny = P.vol.n[1];
-    const bool yfast = V.layout != 0;
-    const float* __restrict__ base = yfast ? volT : vol;
-    const Off sx = yfast ? ny : (Off)1;
-    const Off sy = yfast ? (Off)1 : nx;
-    const Off sz = nx * ny;
-    const Off off = (Off)W.i[2] * sz + (Off)W.i[1] * sy + (Off)W.i[0] * sx;
-    walk<Off>(W, off, W.step[0] * sx, W.step[1] * sy, W.step[2] * sz,
-              [&](Off o, float len) { acc = fmaf(len, __ldg(base + o), acc); });
-  }
-  sino[((size_t)v * P.dims.n_rows + r) * P.dims.n_cols + c] = acc;
+  walk<true, Off>(hit, W, lo, hi, off, W.step[0] * sx, W.step[1] * sy, W.step[2] * sz,
+            [&](Off o, float len) { acc = fmaf(len, __ldg(base + o), acc); });
+  if (valid) sino[((size_t)v * P.dims.n_rows + r) * P.dims.n_cols + c] = acc;
 }
 
 // ------------------------------------------------------------------- count --
@@ -259,19 +454,17 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows) count_kernel(FwdLaunch P, 
   const int ct = rem - v * P.n_col_tiles;
   const int c = ct * kFwdCols + threadIdx.x;
   const int r = band * kFwdRows + threadIdx.y;
+  const bool valid = c < P.dims.n_cols && r < P.dims.n_rows;
   unsigned long long n = 0;
-  if (c < P.dims.n_cols && r < P.dims.n_rows) {
-    Ray R;
-    make_ray(views[v], P.vol, trig, P.dims, v, r, c, R);
-    const int lo[3] = {0, 0, 0};
-    const int hi[3] = {P.vol.n[0], P.vol.n[1], P.vol.n[2]};
-    double t_in, t_out;
-    if (clip(R, lo, hi, t_in, t_out)) {
-      Walk W;
-      entry(R, t_in, t_out, lo, hi, W);
-      walk<int>(W, 0, 0, 0, 0, [&](int, float len) { n += len > 0.f ? 1ull : 0ull; });
-    }
-  }
+  Ray R;
+  make_ray(views[v], P.vol, trig, P.dims, v, valid ? r : 0, valid ? c : 0, R);
+  const int lo[3] = {0, 0, 0};
+  const int hi[3] = {P.vol.n[0], P.vol.n[1], P.vol.n[2]};
+  double t_in = 0.0, t_out = 0.0;
+  const bool hit = valid && clip(R, lo, hi, t_in, t_out);
+  Walk W = {};
+  if (hit) entry(R, t_in, t_out, lo, hi, W);
+  walk<false, int>(hit, W, lo, hi, 0, 0, 0, 0, [&](int, float len) { n += len > 0.f ? 1ull : 0ull; });
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
   if ((threadIdx.x & 31) == 0 && n) atomicAdd(counter, n);
@@ -298,13 +491,18 @@ __global__ void __launch_bounds__(256) transpose_xy_kernel(const float* __restri
 // -------------------------------------------------------------- back: brick --
 
 // Detector footprint of the brick [lo, hi) in view V: a rectangle of pixels
-// that contains every pixel whose ray can meet the brick.  Computed by one
-// warp (lanes 0-7 project the eight corners); all lanes return the result.
+// that contains every pixel whose ray can meet the brick.  Also returns
+// nvox, an upper bound on the number of this view's rays that can meet any
+// single voxel of the brick (lattice points inside the bounding rectangle of
+// one voxel's projection, plus slack), used to size the fixed-point scale.
+// Computed by one warp (lanes 0-7 project the eight corners); all lanes
+// return the result.
 __device__ void brick_footprint(const ViewRec& V, const BackLaunch& P, const int lo[3], const int hi[3], int lane,
-                                int& c0, int& c1, int& r0, int& r1) {
+                                int& c0, int& c1, int& r0, int& r1, int& nvox) {
   const int nc = P.dims.n_cols, nr = P.dims.n_rows;
   if (V.full_footprint) {
     c0 = 0, c1 = nc - 1, r0 = 0, r1 = nr - 1;
+    nvox = nc * nr;
     return;
   }
   const int q = lane & 7;
@@ -312,8 +510,10 @@ __device__ void brick_footprint(const ViewRec& V, const BackLaunch& P, const int
   const int cv[3] = {(q & 1) ? hi[0] : lo[0], (q & 2) ? hi[1] : lo[1], (q & 4) ? hi[2] : lo[2]};
 #pragma unroll
   for (int k = 0; k < 3; ++k) X[k] = P.vol.origin[k] + (double)cv[k] * P.vol.spacing[k];
-  double cmin, cmax, rmin, rmax;
+  double cmin, cmax, rmin, rmax, lam_min = 0.0;
   int bad = 0;
+  // cylindrical only: distance of the brick from the source's axis
+  double rho_lo = 0.0, rho_hi = 0.0;
   if (P.dims.beam == CTP_BEAM_PARALLEL) {
     const double d[3] = {X[0] - V.p00[0], X[1] - V.p00[1], X[2] - V.p00[2]};
     cmin = cmax = V.minv[0] * d[0] + V.minv[1] * d[1] + V.minv[2] * d[2];
@@ -323,6 +523,7 @@ __device__ void brick_footprint(const ViewRec& V, const BackLaunch& P, const int
     const double lam = V.minv[0] * d[0] + V.minv[1] * d[1] + V.minv[2] * d[2];
     const double lc = V.minv[3] * d[0] + V.minv[4] * d[1] + V.minv[5] * d[2];
     const double lr = V.minv[6] * d[0] + V.minv[7] * d[1] + V.minv[8] * d[2];
+    lam_min = lam;
     if (!(lam > 1e-12)) {
       bad = 1;
       cmin = cmax = rmin = rmax = 0.0;
@@ -350,7 +551,9 @@ __device__ void brick_footprint(const ViewRec& V, const BackLaunch& P, const int
     cmin = cmax = (phi - V.gam0) / V.dgam;
     rmin = rmax = h;  // reduced below, then converted with the rho bounds
     const double rho_c = sqrt(ac * ac + bc * bc), hd = sqrt(hd2);
-    if (!(rho_c - hd > 1e-9)) bad = 1;
+    rho_lo = rho_c - hd;
+    rho_hi = rho_c + hd;
+    if (!(rho_lo > 1e-9)) bad = 1;
   }
 #pragma unroll
   for (int o = 1; o < 8; o <<= 1) {
@@ -358,24 +561,30 @@ __device__ void brick_footprint(const ViewRec& V, const BackLaunch& P, const int
     cmax = fmax(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
     rmin = fmin(rmin, __shfl_xor_sync(0xffffffffu, rmin, o));
     rmax = fmax(rmax, __shfl_xor_sync(0xffffffffu, rmax, o));
+    lam_min = fmin(lam_min, __shfl_xor_sync(0xffffffffu, lam_min, o));
     bad |= __shfl_xor_sync(0xffffffffu, bad, o);
   }
   if (bad) {
     c0 = 0, c1 = nc - 1, r0 = 0, r1 = nr - 1;
+    nvox = nc * nr;
     return;
   }
-  if (P.dims.beam == CTP_BEAM_CONE && P.dims.det == CTP_DET_CYLINDRICAL) {
-    double Xc[3], hd2 = 0.0;
-#pragma unroll
-    for (int k = 0; k < 3; ++k) {
-      Xc[k] = P.vol.origin[k] + 0.5 * (double)(lo[k] + hi[k]) * P.vol.spacing[k] - V.s[k];
-      const double e = 0.5 * (double)(hi[k] - lo[k]) * P.vol.spacing[k];
-      hd2 += e * e;
-    }
-    const double ac = Xc[0] * V.w[0] + Xc[1] * V.w[1] + Xc[2] * V.w[2];
-    const double bc = Xc[0] * V.du[0] + Xc[1] * V.du[1] + Xc[2] * V.du[2];
-    const double rho_c = sqrt(ac * ac + bc * bc), hd = sqrt(hd2);
-    const double rho_lo = rho_c - hd, rho_hi = rho_c + hd;
+  // extent (in pixels) of one voxel's projection: wc columns by wr rows
+  double wc, wr;
+  const double D = sqrt(P.vol.spacing[0] * P.vol.spacing[0] + P.vol.spacing[1] * P.vol.spacing[1] +
+                        P.vol.spacing[2] * P.vol.spacing[2]);
+  if (P.dims.beam == CTP_BEAM_PARALLEL) {
+    wc = V.vox_ext[0];
+    wr = V.vox_ext[1];
+  } else if (P.dims.det == CTP_DET_FLAT) {
+    // c = lc / lam over a voxel varies by at most (A_c + |c|max A_lam) / lam_min
+    const double cm = fmax(fabs(cmin), fabs(cmax)), rm = fmax(fabs(rmin), fabs(rmax));
+    wc = (V.vox_ext[1] + cm * V.vox_ext[0]) / lam_min;
+    wr = (V.vox_ext[2] + rm * V.vox_ext[0]) / lam_min;
+  } else {
+    const double H = fmax(fabs(rmin), fabs(rmax));
+    wc = 1.5707963267948966 * D / (rho_lo * V.dgam);
+    wr = V.R * D * (1.0 / rho_lo + H / (rho_lo * rho_lo)) / V.vlen;
     const double hmin = rmin, hmax = rmax;
     const double q_lo = hmin >= 0.0 ? hmin / rho_hi : hmin / rho_lo;
     const double q_hi = hmax >= 0.0 ? hmax / rho_lo : hmax / rho_hi;
@@ -388,16 +597,31 @@ __device__ void brick_footprint(const ViewRec& V, const BackLaunch& P, const int
   c1 = min((int)ch, nc - 1);
   r0 = max((int)rl, 0);
   r1 = min((int)rh, nr - 1);
+  const long long fw_ = c1 >= c0 ? c1 - c0 + 1 : 0, fh_ = r1 >= r0 ? r1 - r0 + 1 : 0;
+  const double pc = floor(fmin(wc, 1e6)) + 2.0, pr = floor(fmin(wr, 1e6)) + 2.0;
+  nvox = (int)fmin(pc * pr, (double)(fw_ * fh_));
 }
 
+// Adjoint on one brick.  Ray contributions are accumulated in shared memory
+// as 32-bit fixed point (native integer atomics; shared-memory float atomics
+// are compare-and-swap loops on this hardware).  The views are taken in
+// stages of kBackStage; per stage the scale S is set so that no voxel can
+// overflow: every segment is at most one voxel diagonal long, |y| is at most
+// the stage's largest footprint value, and no voxel meets more than the
+// summed per-view ray bounds.  Each stage is then flushed into the FP32
+// volume.  Integer sums are exact, so the result does not depend on the
+// order in which threads add.
 template <typename Off>
-__global__ void __launch_bounds__(kBackThreads) back_brick_kernel(BackLaunch P, const ViewRec* __restrict__ views,
-                                                                  const double* __restrict__ trig,
-                                                                  const float* __restrict__ sino,
-                                                                  float* __restrict__ vol) {
-  extern __shared__ float acc[];
-  __shared__ int fp[kBackChunk][3];  // c0, r0, width per staged view
-  __shared__ int pre[kBackChunk + 1];
+__global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
+    back_brick_kernel(BackLaunch P, const ViewRec* __restrict__ views, const double* __restrict__ trig,
+                      const float* __restrict__ sino, float* __restrict__ vol) {
+  extern __shared__ int acc[];
+  // per staged view: first column, first row, width, footprint size, ray bound
+  __shared__ int fc0[kBackStage], fr0[kBackStage], fw[kBackStage], cnt[kBackStage], nvb[kBackStage];
+  __shared__ int pre[kBackStage + 1];
+  __shared__ unsigned int s_ymax_bits;
+  __shared__ long long s_nsum;
+  __shared__ float s_scale;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int b = blockIdx.x;
@@ -413,71 +637,173 @@ __global__ void __launch_bounds__(kBackThreads) back_brick_kernel(BackLaunch P, 
   const int pitch = P.pitch_x;
   const int plane = pitch * P.brick[1];
   const int n_acc = plane * P.brick[2];
-  for (int i = tid; i < n_acc; i += kBackThreads) acc[i] = 0.f;
+  for (int i = tid; i < n_acc; i += kBackThreads) acc[i] = 0;
+  const double diag = sqrt(P.vol.spacing[0] * P.vol.spacing[0] + P.vol.spacing[1] * P.vol.spacing[1] +
+                           P.vol.spacing[2] * P.vol.spacing[2]);
+  const int ex = hi[0] - lo[0], ey = hi[1] - lo[1], ez = hi[2] - lo[2];
+  const int n_out = ex * ey * ez;
+  const Off nx = P.vol.n[0], ny = P.vol.n[1];
 
   const int nr = P.dims.n_rows, nc = P.dims.n_cols;
   const int v_begin = g * P.views_per_group;
   const int v_end = min(v_begin + P.views_per_group, P.dims.n_views);
-  for (int vb = v_begin; vb < v_end; vb += kBackChunk) {
-    __syncthreads();  // previous chunk's footprints consumed (and accumulators zeroed)
-    if (warp < kBackChunk) {
-      const int v = vb + warp;
-      int c0 = 0, c1 = -1, r0 = 0, r1 = -1;
-      if (v < v_end) brick_footprint(views[v], P, lo, hi, lane, c0, c1, r0, r1);
+  bool first = true;
+  for (int vb = v_begin; vb < v_end; vb += kBackStage) {
+    const int nvs = min(kBackStage, v_end - vb);
+    __syncthreads();  // previous stage flushed (and accumulators zeroed)
+    for (int s = warp; s < nvs; s += kBackThreads / 32) {
+      int c0 = 0, c1 = -1, r0 = 0, r1 = -1, nv = 0;
+      brick_footprint(views[vb + s], P, lo, hi, lane, c0, c1, r0, r1, nv);
       if (lane == 0) {
         const int w = c1 >= c0 ? c1 - c0 + 1 : 0;
         const int h = r1 >= r0 ? r1 - r0 + 1 : 0;
-        fp[warp][0] = c0;
-        fp[warp][1] = r0;
-        fp[warp][2] = w;
-        pre[warp + 1] = w * h;  // count, turned into a prefix sum below
+        fc0[s] = c0;
+        fr0[s] = r0;
+        fw[s] = w;
+        cnt[s] = w * h;
+        nvb[s] = w * h > 0 ? nv : 0;
       }
+    }
+    if (tid == 0) s_ymax_bits = 0u;
+    __syncthreads();
+    if (warp == 0) {
+      // exclusive scan of cnt[0..nvs) and the sum of the ray bounds
+      constexpr int kPer = kBackStage / 32;
+      int sum = 0;
+      long long nsum = 0;
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        const int i = lane * kPer + j;
+        sum += i < nvs ? cnt[i] : 0;
+        nsum += i < nvs ? nvb[i] : 0;
+      }
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) nsum += __shfl_xor_sync(0xffffffffu, nsum, o);
+      int run = incl - sum;
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        const int i = lane * kPer + j;
+        if (i < nvs) {
+          pre[i] = run;
+          run += cnt[i];
+        }
+      }
+      if (lane == 31) pre[nvs] = incl;
+      if (lane == 0) s_nsum = nsum;
+    }
+    __syncthreads();
+    const int total = pre[nvs];
+    // pass 1: largest |y| of the stage's footprint rays (NaN and inf sort
+    // above every finite value as unsigned bit patterns)
+    {
+      unsigned int mb = 0u;
+      for (int q = tid; q < total; q += kBackThreads) {
+        int sl = 0, sh = nvs;
+        while (sh - sl > 1) {
+          const int mid = (sl + sh) >> 1;
+          if (pre[mid] <= q) sl = mid;
+          else sh = mid;
+        }
+        const int qq = q - pre[sl];
+        const int rr = qq / fw[sl];
+        const int r = fr0[sl] + rr, c = fc0[sl] + (qq - rr * fw[sl]);
+        mb = max(mb, __float_as_uint(fabsf(__ldg(sino + ((size_t)(vb + sl) * nr + r) * nc + c))));
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+      if (lane == 0 && mb) atomicMax(&s_ymax_bits, mb);
     }
     __syncthreads();
     if (tid == 0) {
-      pre[0] = 0;
-      for (int s = 0; s < kBackChunk; ++s) pre[s + 1] += pre[s];
+      const unsigned int bits = s_ymax_bits;
+      float sc = 0.f;
+      if (bits >= 0x7f800000u) {
+        sc = CUDART_NAN_F;  // non-finite input: the brick is written as NaN
+      } else {
+        const double bound = (double)__uint_as_float(bits) * diag * (double)s_nsum;
+        if (bound > 0.0) sc = (float)((2147483647.0 - 4194304.0) / bound);
+      }
+      s_scale = sc;
     }
     __syncthreads();
-    const int total = pre[kBackChunk];
-    for (int q = tid; q < total; q += kBackThreads) {
-      int s = 0;
-      while (q >= pre[s + 1]) ++s;
-      const int qq = q - pre[s];
-      const int w = fp[s][2];
-      const int rr = qq / w;
-      const int r = fp[s][1] + rr, c = fp[s][0] + (qq - rr * w);
-      const int v = vb + s;
-      const float y = __ldg(sino + ((size_t)v * nr + r) * nc + c);
-      if (y == 0.f) continue;
-      Ray R;
-      make_ray(views[v], P.vol, trig, P.dims, v, r, c, R);
-      double t_in, t_out;
-      if (!clip(R, lo, hi, t_in, t_out)) continue;
-      Walk W;
-      entry(R, t_in, t_out, lo, hi, W);
-      const int off = ((W.i[2] - lo[2]) * P.brick[1] + (W.i[1] - lo[1])) * pitch + (W.i[0] - lo[0]);
-      walk<int>(W, off, W.step[0], W.step[1] * pitch, W.step[2] * plane,
-                [&](int o, float len) { atomicAdd(acc + o, len * y); });
+    const float S = s_scale;
+    // pass 2: walk every ray of the stage through the brick.  Each warp takes
+    // 32 consecutive footprint rays (neighbouring columns, similar chords),
+    // sets them up together and reconverges before the next 32.
+    if (S > 0.f) {
+      for (int q0 = warp * 32; q0 < total; q0 += kBackThreads) {
+        const int q = q0 + lane;
+        bool act = q < total;
+        int v = vb, r = 0, c = 0;
+        float y = 0.f;
+        if (act) {
+          int sl = 0, sh = nvs;
+          while (sh - sl > 1) {
+            const int mid = (sl + sh) >> 1;
+            if (pre[mid] <= q) sl = mid;
+            else sh = mid;
+          }
+          const int qq = q - pre[sl];
+          const int w = fw[sl];
+          const int rr = qq / w;
+          r = fr0[sl] + rr;
+          c = fc0[sl] + (qq - rr * w);
+          v = vb + sl;
+          y = __ldg(sino + ((size_t)v * nr + r) * nc + c);
+          act = y != 0.f;
+        }
+        Ray R;
+        double t_in = 0.0, t_out = 0.0;
+        if (act) {
+          make_ray(views[v], P.vol, trig, P.dims, v, r, c, R);
+          act = clip(R, lo, hi, t_in, t_out);
+        }
+        Walk W = {};
+        int off = 0;
+        if (act) {
+          entry(R, t_in, t_out, lo, hi, W);
+          off = ((W.i[2] - lo[2]) * P.brick[1] + (W.i[1] - lo[1])) * pitch + (W.i[0] - lo[0]);
+        }
+        const float yS = y * S;
+#if CTP_BACK_WARP_WALK
+        walk<CTP_BACK_ALIGN != 0, int>(act, W, lo, hi, off, W.step[0], W.step[1] * pitch, W.step[2] * plane,
+                                     [&](int o, float len) { atomicAdd(acc + o, __float2int_rn(len * yS)); });
+#else
+        if (act)
+          walk_lane<int>(W, off, W.step[0], W.step[1] * pitch, W.step[2] * plane,
+                         [&](int o, float len) { atomicAdd(acc + o, __float2int_rn(len * yS)); });
+        __syncwarp();
+#endif
+      }
     }
-  }
-  __syncthreads();
-
-  const int ex = hi[0] - lo[0], ey = hi[1] - lo[1], ez = hi[2] - lo[2];
-  const int n_out = ex * ey * ez;
-  const Off nx = P.vol.n[0], ny = P.vol.n[1];
-  for (int i = tid; i < n_out; i += kBackThreads) {
-    const int x = i % ex;
-    const int t = i / ex;
-    const int yy = t % ey;
-    const int z = t / ey;
-    const float val = acc[(z * P.brick[1] + yy) * pitch + x];
-    const Off gi = ((Off)(lo[2] + z) * ny + (Off)(lo[1] + yy)) * nx + (Off)(lo[0] + x);
-    if (P.view_groups > 1) {
-      if (val != 0.f) atomicAdd(vol + gi, val);
-    } else {
-      vol[gi] = val;
+    __syncthreads();
+    // flush the stage into the volume and clear the accumulators
+    const bool nan_stage = S != S;
+    const float inv = S > 0.f ? 1.f / S : 0.f;
+    for (int i = tid; i < n_out; i += kBackThreads) {
+      const int x = i % ex;
+      const int t = i / ex;
+      const int yy = t % ey;
+      const int z = t / ey;
+      const int ai = (z * P.brick[1] + yy) * pitch + x;
+      const float val = nan_stage ? CUDART_NAN_F : (float)acc[ai] * inv;
+      acc[ai] = 0;
+      const Off gi = ((Off)(lo[2] + z) * ny + (Off)(lo[1] + yy)) * nx + (Off)(lo[0] + x);
+      if (P.view_groups > 1) {
+        if (val != 0.f) atomicAdd(vol + gi, val);
+      } else if (first) {
+        vol[gi] = val;
+      } else {
+        vol[gi] += val;
+      }
     }
+    first = false;
   }
 }
 
@@ -514,7 +840,7 @@ cudaError_t launch_count(const FwdLaunch& p, const ViewRec* views, const double*
 }
 
 size_t back_brick_smem_bytes(const int32_t brick[3]) {
-  return sizeof(float) * (size_t)(brick[0] + 1) * brick[1] * brick[2];
+  return sizeof(int) * (size_t)(brick[0] + 1) * brick[1] * brick[2];
 }
 
 cudaError_t prepare_back_brick(size_t smem_bytes) {

@@ -72,10 +72,13 @@ class CtpError(RuntimeError):
 _lib = None
 
 
-def load(path: str = LIB_PATH):
-    """Load libctp.so (built by ``ray_forward_back_b200.build``)."""
+def load(path: str = None):
+    """Load libctp.so (built by ``ray_forward_back_b200.build``).  The
+    CTP_LIBRARY environment variable selects another build of the library."""
     global _lib
     if _lib is None:
+        if path is None:
+            path = os.environ.get("CTP_LIBRARY") or LIB_PATH
         if not os.path.exists(path):
             raise RuntimeError(f"libctp.so is not built ({path}); run python -m ray_forward_back_b200.build")
         lib = ctypes.CDLL(path)
