@@ -10,11 +10,15 @@
  * each world coordinate by its axis pitch and integrates in physical length
  * units).  Forward and back use the same coefficients ("matched
  * interpolation/traversal coefficients", same section), up to FP32 rounding
- * and summation order; the floating-point scatter order is not deterministic.
+ * and summation order.
  *
  * Precision: per-ray clipping and entry setup in FP64, traversal and data in
- * FP32 (same page, table row backend="numba"; and the paragraph "Segment
- * setup starts from the endpoint nearer the volume center ...").
+ * FP32 (same page, table row backend="numba", and its paragraph on segment
+ * setup from the endpoint nearer the volume centre).  The adjoint sums its
+ * contributions exactly as 32-bit fixed point inside each block of the
+ * volume (scale chosen per stage of views so that no voxel can overflow) and
+ * adds the stages into the FP32 volume, so its result does not depend on
+ * thread scheduling; the forward projection is deterministic as well.
  *
  * Layouts (same page, "Batch dimensions and axis spacing"):
  *   volume    float32 [nz][ny][nx], x fastest, contiguous
@@ -150,7 +154,9 @@ ctp_status ctp_forward(const ctp_geom *geom, const float *vol, float *sino, void
  * coefficients (diffct "Execution": backward applies the matched adjoint).
  * sino: device pointer, float32 [n_views][n_rows][n_cols], read only.
  * vol:  device pointer, float32 [nz][ny][nx], overwritten.
- * Same pointer, stream and synchronisation rules as ctp_forward.
+ * Same pointer, stream and synchronisation rules as ctp_forward.  A
+ * non-finite sinogram value (NaN or infinity) is not dropped: every voxel of
+ * each volume block whose detector footprint holds it is written as NaN.
  */
 ctp_status ctp_back(const ctp_geom *geom, const float *sino, float *vol, void *stream);
 
