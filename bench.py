@@ -106,6 +106,22 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def aggregate_over_ranks(times_ms, world, device=None):
+    """Max over ranks of each timing (barrier semantics: the job is as slow as
+    its slowest rank).  Works with any initialised process group (nccl, gloo)."""
+    import torch
+    t = torch.tensor([float(x) for x in times_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def throughput(updates_per_rank_step, world, ms_per_step):
+    """Whole-job Gupdates/s: every rank's updates over the slowest rank's time."""
+    return world * updates_per_rank_step / (ms_per_step * 1e-3) / 1e9
+
+
 def cpu_oracle_sample(wl, n_views_sample=1):
     """FP64 oracle forward + back over an evenly spaced subset of views, on one
     host core.  Returns (updates/s, seconds, updates, description)."""
@@ -219,12 +235,9 @@ def run_ours(args, rank, world, local_rank):
     total_ms = start.elapsed_time(end)
     fwd_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(args.steps)]
     back_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(args.steps)]
-    t = torch.tensor([total_ms, float(np.mean(fwd_ms)), float(np.mean(back_ms))], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, fwd_avg, back_avg = t.tolist()
+    total_ms, fwd_avg, back_avg = aggregate_over_ranks([total_ms, np.mean(fwd_ms), np.mean(back_ms)], world, dev)
     ms_per_step = total_ms / args.steps
-    value = world * 2 * U / (ms_per_step * 1e-3) / 1e9
+    value = throughput(2 * U, world, ms_per_step)
 
     # end to end through the public API with host buffers (pinned), every step
     e2e = None
@@ -255,11 +268,8 @@ def run_ours(args, rank, world, local_rank):
             e2e_step()
         s1.record(stream)
         torch.cuda.synchronize(dev)
-        et = torch.tensor([s0.elapsed_time(s1) / args.steps], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(et, op=dist.ReduceOp.MAX)
-        e2e_ms = et.item()
-        e2e = {"value": world * 2 * U / (e2e_ms * 1e-3) / 1e9, "unit": UNIT, "ms_per_step": e2e_ms,
+        e2e_ms = aggregate_over_ranks([s0.elapsed_time(s1) / args.steps], world, dev)[0]
+        e2e = {"value": throughput(2 * U, world, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": int(vol_pin.numel() * 4 + sino_pin.numel() * 4),
                "d2h_bytes_per_step": int(sino_res.numel() * 4 + vol_res.numel() * 4)}
 

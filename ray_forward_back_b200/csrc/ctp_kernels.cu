@@ -313,7 +313,11 @@ __device__ __forceinline__ void walk_lane(const Walk& W, Off off, Off s0, Off s1
 // dropped (its error is below one ulp of the walk length).
 //
 // All 32 lanes must call this together; lanes without a ray pass active = false.
-template <bool kAlign, typename Off, typename Visit>
+// With kUniform, every lane calls visit(offset, length, flag) at every segment
+// slot, flag telling whether the segment exists for that lane (so the visitor
+// may use warp collectives); a slot that no lane of the warp has is skipped.
+// Without it, visit(offset, length, true) is called for existing segments only.
+template <bool kAlign, bool kUniform, typename Off, typename Visit>
 __device__ __forceinline__ void walk(bool active, const Walk& W, const int lo[3], const int hi[3], Off off, Off s0,
                                      Off s1, Off s2, Visit&& visit) {
   constexpr unsigned kFull = 0xffffffffu;
@@ -358,8 +362,13 @@ __device__ __forceinline__ void walk(bool active, const Walk& W, const int lo[3]
       const float tx = s < Na ? fminf(fmaf((float)s, inca, l0a), L) : L;
       const bool cb = on && tb < tx;
       const float m1 = fmaxf(fminf(tb, tx), cur);
-      if (on) visit(off, m1 - cur);
-      if (cb) visit(off + sb, tx - m1);
+      if (kUniform) {
+        visit(off, m1 - cur, on);
+        if (__any_sync(kFull, cb)) visit(off + sb, tx - m1, cb);
+      } else {
+        if (on) visit(off, m1 - cur, true);
+        if (cb) visit(off + sb, tx - m1, true);
+      }
       if (on) {
         off += (cb ? sb : (Off)0) + sa;
         cur = tx;
@@ -384,9 +393,15 @@ __device__ __forceinline__ void walk(bool active, const Walk& W, const int lo[3]
       const Off db = cb ? sb : (Off)0, dc = cc ? sc : (Off)0;
       const Off o2 = off + (tb <= tc ? db : dc);
       const Off o3 = off + db + dc;
-      if (on) visit(off, m1 - cur);
-      if (cb || cc) visit(o2, m2 - m1);
-      if (cb && cc) visit(o3, tx - m2);
+      if (kUniform) {
+        visit(off, m1 - cur, on);
+        if (__any_sync(kFull, cb || cc)) visit(o2, m2 - m1, cb || cc);
+        if (__any_sync(kFull, cb && cc)) visit(o3, tx - m2, cb && cc);
+      } else {
+        if (on) visit(off, m1 - cur, true);
+        if (cb || cc) visit(o2, m2 - m1, true);
+        if (cb && cc) visit(o3, tx - m2, true);
+      }
       if (on) {
         off = o3 + sa;
         cur = tx;
@@ -437,8 +452,8 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_FWD_MIN_BLOCKS) forwar
   const Off sz = nx * ny;
   const Off off = (Off)W.i[2] * sz + (Off)W.i[1] * sy + (Off)W.i[0] * sx;
   float acc = 0.f;
-  walk<true, Off>(hit, W, lo, hi, off, W.step[0] * sx, W.step[1] * sy, W.step[2] * sz,
-            [&](Off o, float len) { acc = fmaf(len, __ldg(base + o), acc); });
+  walk<true, false, Off>(hit, W, lo, hi, off, W.step[0] * sx, W.step[1] * sy, W.step[2] * sz,
+                         [&](Off o, float len, bool) { acc = fmaf(len, __ldg(base + o), acc); });
   if (valid) sino[((size_t)v * P.dims.n_rows + r) * P.dims.n_cols + c] = acc;
 }
 
@@ -464,7 +479,7 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows) count_kernel(FwdLaunch P, 
   const bool hit = valid && clip(R, lo, hi, t_in, t_out);
   Walk W = {};
   if (hit) entry(R, t_in, t_out, lo, hi, W);
-  walk<false, int>(hit, W, lo, hi, 0, 0, 0, 0, [&](int, float len) { n += len > 0.f ? 1ull : 0ull; });
+  walk<false, false, int>(hit, W, lo, hi, 0, 0, 0, 0, [&](int, float len, bool) { n += len > 0.f ? 1ull : 0ull; });
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
   if ((threadIdx.x & 31) == 0 && n) atomicAdd(counter, n);
@@ -772,8 +787,8 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
         }
         const float yS = y * S;
 #if CTP_BACK_WARP_WALK
-        walk<CTP_BACK_ALIGN != 0, int>(act, W, lo, hi, off, W.step[0], W.step[1] * pitch, W.step[2] * plane,
-                                     [&](int o, float len) { atomicAdd(acc + o, __float2int_rn(len * yS)); });
+        walk<CTP_BACK_ALIGN != 0, false, int>(act, W, lo, hi, off, W.step[0], W.step[1] * pitch, W.step[2] * plane,
+                                            [&](int o, float len, bool) { atomicAdd(acc + o, __float2int_rn(len * yS)); });
 #else
         if (act)
           walk_lane<int>(W, off, W.step[0], W.step[1] * pitch, W.step[2] * plane,
@@ -807,6 +822,114 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
   }
 }
 
+// ------------------------------------------------------ back: sort / reduce --
+
+// Bitonic sort of one (key, value) pair per lane across the warp, ascending
+// by key; pairs move together and equal keys are never split or duplicated.
+template <typename Key>
+__device__ __forceinline__ void warp_sort_pairs(Key& key, float& val, int lane) {
+  constexpr unsigned kFull = 0xffffffffu;
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const Key pk = __shfl_xor_sync(kFull, key, j);
+      const float pv = __shfl_xor_sync(kFull, val, j);
+      const bool ascending = (lane & k) == 0;
+      const bool lower = (lane & j) == 0;
+      const bool take = (lower == ascending) ? (pk < key) : (key < pk);
+      if (take) {
+        key = pk;
+        val = pv;
+      }
+    }
+  }
+}
+
+// One warp-wide batch of the sort / segment-reduce adjoint: the 32 lanes'
+// (voxel key, contribution) pairs are grouped by key (a warp sort, skipped
+// when the keys are already monotone across the lanes, which the aligned
+// walk of neighbouring rays usually gives), each run of equal keys is summed
+// with a segmented scan, and its last lane adds the run's sum to the volume
+// with one global atomic.  With kCount nothing is written; instead the
+// numbers of contributions and of runs are added to n_upd and n_runs.
+template <bool kCount, typename Key>
+__device__ __forceinline__ void warp_segment_reduce(Key key, float val, bool valid, float* __restrict__ vol,
+                                                    unsigned long long& n_upd, unsigned long long& n_runs) {
+  constexpr unsigned kFull = 0xffffffffu;
+  const Key kNone = (Key)(~(unsigned long long)0 >> 1);
+  const int lane = threadIdx.x & 31;
+  if (!valid || !(val != 0.f)) {
+    key = kNone;
+    val = 0.f;
+  }
+  const Key kn = __shfl_down_sync(kFull, key, 1);
+  const bool nondec = lane == 31 || key <= kn, noninc = lane == 31 || key >= kn;
+  if (!__all_sync(kFull, nondec) && !__all_sync(kFull, noninc)) warp_sort_pairs(key, val, lane);
+  const Key kp = __shfl_up_sync(kFull, key, 1);
+  const Key kq = __shfl_down_sync(kFull, key, 1);
+  const bool head = lane == 0 || kp != key;
+  const bool tail = lane == 31 || kq != key;
+  const unsigned heads = __ballot_sync(kFull, head);
+  const int start = 31 - __clz(heads & (kFull >> (31 - lane)));
+  float sum = val;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float t = __shfl_up_sync(kFull, sum, o);
+    if (lane - o >= start) sum += t;
+  }
+  if (kCount) {
+    const unsigned u = __ballot_sync(kFull, key != kNone);
+    const unsigned r = __ballot_sync(kFull, tail && key != kNone);
+    if (lane == 0) {
+      n_upd += __popc(u);
+      n_runs += __popc(r);
+    }
+  } else if (tail && key != kNone) {
+    atomicAdd(vol + key, sum);
+  }
+}
+
+// Sort / segment-reduce adjoint: one thread per ray as in the forward
+// kernel (same block order and aligned slab walk over the whole volume), the
+// contributions of each warp step grouped and reduced before one global add
+// per distinct voxel.  Needs the volume zeroed first.  With kCount it writes
+// nothing and counts contributions and runs (the collision ratio) instead,
+// treating every ray value as 1.
+template <bool kCount, typename Off>
+__global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_FWD_MIN_BLOCKS)
+    back_sort_kernel(FwdLaunch P, const ViewRec* __restrict__ views, const double* __restrict__ trig,
+                     const float* __restrict__ sino, float* __restrict__ vol,
+                     unsigned long long* __restrict__ counters) {
+  const int per_band = P.dims.n_views * P.n_col_tiles;
+  const int band = blockIdx.x / per_band;
+  const int rem = blockIdx.x - band * per_band;
+  const int v = rem / P.n_col_tiles;
+  const int ct = rem - v * P.n_col_tiles;
+  const int c = ct * kFwdCols + threadIdx.x;
+  const int r = band * kFwdRows + threadIdx.y;
+  const bool valid = c < P.dims.n_cols && r < P.dims.n_rows;
+  float y = 1.f;
+  if (!kCount) y = valid ? __ldg(sino + ((size_t)v * P.dims.n_rows + r) * P.dims.n_cols + c) : 0.f;
+  Ray R;
+  make_ray(views[v], P.vol, trig, P.dims, v, valid ? r : 0, valid ? c : 0, R);
+  const int lo[3] = {0, 0, 0};
+  const int hi[3] = {P.vol.n[0], P.vol.n[1], P.vol.n[2]};
+  double t_in = 0.0, t_out = 0.0;
+  const bool hit = valid && y != 0.f && clip(R, lo, hi, t_in, t_out);
+  Walk W = {};
+  if (hit) entry(R, t_in, t_out, lo, hi, W);
+  const Off nx = P.vol.n[0], sz = (Off)P.vol.n[0] * P.vol.n[1];
+  const Off off = (Off)W.i[2] * sz + (Off)W.i[1] * nx + (Off)W.i[0];
+  unsigned long long n_upd = 0, n_runs = 0;
+  walk<true, true, Off>(hit, W, lo, hi, off, (Off)W.step[0], W.step[1] * nx, W.step[2] * sz,
+                        [&](Off o, float len, bool f) { warp_segment_reduce<kCount, Off>(o, len * y, f, vol, n_upd, n_runs); });
+  if (kCount && (threadIdx.x & 31) == 0 && (n_upd | n_runs)) {
+    atomicAdd(counters, n_upd);
+    atomicAdd(counters + 1, n_runs);
+  }
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------- launchers --
@@ -836,6 +959,33 @@ cudaError_t launch_count(const FwdLaunch& p, const ViewRec* views, const double*
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   count_kernel<<<(unsigned)blocks, dim3(kFwdCols, kFwdRows), 0, stream>>>(p, views, trig, counter);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_back_sort(const FwdLaunch& p, const ViewRec* views, const double* trig, const float* sino,
+                             float* vol, bool wide_index, cudaStream_t stream) {
+  const long long blocks = (long long)p.n_row_bands * p.dims.n_views * p.n_col_tiles;
+  if (blocks <= 0) return cudaSuccess;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  dim3 block(kFwdCols, kFwdRows);
+  if (wide_index)
+    back_sort_kernel<false, long long><<<(unsigned)blocks, block, 0, stream>>>(p, views, trig, sino, vol, nullptr);
+  else
+    back_sort_kernel<false, int><<<(unsigned)blocks, block, 0, stream>>>(p, views, trig, sino, vol, nullptr);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_collision_count(const FwdLaunch& p, const ViewRec* views, const double* trig,
+                                   unsigned long long* counters, bool wide_index, cudaStream_t stream) {
+  const long long blocks = (long long)p.n_row_bands * p.dims.n_views * p.n_col_tiles;
+  if (blocks <= 0) return cudaSuccess;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  dim3 block(kFwdCols, kFwdRows);
+  if (wide_index)
+    back_sort_kernel<true, long long><<<(unsigned)blocks, block, 0, stream>>>(p, views, trig, nullptr, nullptr,
+                                                                             counters);
+  else
+    back_sort_kernel<true, int><<<(unsigned)blocks, block, 0, stream>>>(p, views, trig, nullptr, nullptr, counters);
   return cudaGetLastError();
 }
 

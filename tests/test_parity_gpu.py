@@ -271,3 +271,56 @@ def test_host_pointer_is_rejected():
     with pytest.raises(ctp.CtpError) as ei:
         ctp.ctp_forward(P.handle, host.data_ptr(), dev.data_ptr())
     assert ei.value.status == ctp.CTP_ERR_INVALID_ARGUMENT
+
+
+# ------------------------------------------ sort / segment-reduce adjoint ---
+
+@pytest.mark.parametrize("name", sorted(ragged_geometries()))
+def test_back_sort_variant_matches_oracle_small(name):
+    """The sort / segment-reduce adjoint meets the same tolerances."""
+    g = ragged_geometries()[name]
+    rng = np.random.default_rng(12)
+    sino = rng.random(g.sino_shape).astype(np.float32)
+    P = projector(g, {"adjoint_variant": 2})
+    assert P.info()["adjoint_variant"] == 2
+    x = gpu_back(P, sino)
+    check_back(x, oracle.back(g, sino), oracle.back(g, np.abs(sino), power=0), float(np.linalg.norm(
+        np.array([g.nx, g.ny, g.nz]) * np.array(g.spacing))), name)
+    assert adjoint_mismatch(P, g) <= 1e-5
+
+
+@pytest.mark.parametrize("index", [0, 1])
+def test_back_sort_variant_workloads(index):
+    wl = W.workload(index)
+    g = wl.geom
+    sino = wl.sinogram()
+    P = projector(g, {"adjoint_variant": 2})
+    x = gpu_back(P, sino)
+    check_back(x, oracle.back(g, sino), oracle.back(g, sino, power=0),
+               float(np.linalg.norm(np.array([g.nx, g.ny, g.nz]) * np.array(g.spacing))), wl.name)
+
+
+def high_magnification_cone():
+    """Cone beam whose rays are ten times denser than the voxels at the centre."""
+    return W.make_cone(40, 40, 24, 8, 48, 160, sid=60.0, sdd=600.0, pitch_u=1.0, pitch_v=1.0, start=0.15)
+
+
+def test_collision_ratio_measured_and_dispatch_consistent():
+    """The ratio measured at create is >= 1 and grows with ray density; the
+    automatic choice is the sort adjoint for dense rays (ratio >= 3.4) and
+    the brick adjoint otherwise, and both results meet the tolerances."""
+    dense = high_magnification_cone()
+    sparse = ragged_geometries()["parallel_ragged"]
+    Pd, Ps = projector(dense), projector(sparse)
+    rd, rs = Pd.info()["collision_ratio"], Ps.info()["collision_ratio"]
+    assert rs >= 1.0 and rd >= 1.0
+    assert rd > 2.0 * rs, (rd, rs)
+    assert Pd.info()["adjoint_variant"] == (2 if rd >= 3.4 else 1)
+    assert Ps.info()["adjoint_variant"] == (2 if rs >= 3.4 else 1)
+    assert Pd.info()["adjoint_variant"] == 2 and Ps.info()["adjoint_variant"] == 1
+    for P, g in ((Pd, dense), (Ps, sparse)):
+        rng = np.random.default_rng(3)
+        sino = rng.random(g.sino_shape).astype(np.float32)
+        ref = oracle.back(g, sino)
+        check_back(gpu_back(P, sino), ref, oracle.back(g, sino, power=0),
+                   float(np.linalg.norm(np.array([g.nx, g.ny, g.nz]) * np.array(g.spacing))), "auto")
