@@ -167,6 +167,38 @@ ctp_status ctp_back(const ctp_geom *geom, const float *sino, float *vol, void *s
  */
 ctp_status ctp_count_updates(const ctp_geom *geom, int64_t *host_out, void *stream);
 
+/*
+ * ctp_forward_noalloc — the forward projection sino = A vol for callers that
+ * cannot allocate device memory: code running where cudaMalloc is not
+ * allowed (a real-time loop with a fixed memory budget, an allocator-free
+ * embedded runtime, a process whose device memory is owned by another
+ * framework) and so cannot create a geometry handle either.  The pages have
+ * no counterpart; this is a library convenience.
+ *
+ * It takes the acquisition description itself (same fields and guards as
+ * ctp_geom_create) plus the caller's device buffers, and computes exactly
+ * what ctp_forward computes, with the same kernels.  It calls no cudaMalloc,
+ * cudaFree or other allocating routine, and uses no host heap: its per-view
+ * records, the cylindrical column table and the y-fastest copy of the volume
+ * live in one fixed device array of CTP_NOALLOC_SCRATCH_BYTES, which every
+ * GPU that loads this library holds until the process exits.  A description
+ * whose records + column table + volume copy (4 bytes per voxel, needed when
+ * some view's detector columns run mostly along y) exceed that size is
+ * rejected with CTP_ERR_OUT_OF_RANGE and a detail message giving the sizes.
+ *
+ * The first call on a device looks the array's device address up
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * The records are copied from host stack memory with cudaMemcpyAsync, so the
+ * call may wait for earlier work on `stream` before returning.  All calls on a
+ * device share the one array and it keeps the last call's contents: calls
+ * that overlap on the GPU (different streams, or different host threads) race
+ * and corrupt each other's results; serialise them on one stream.
+ * vol, sino: as for ctp_forward.  The plan's forward_layout is honoured; the
+ * other plan fields do not apply.
+ */
+#define CTP_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+ctp_status ctp_forward_noalloc(const ctp_geom_desc *desc, const float *vol, float *sino, void *stream);
+
 /* Static description of a status code. */
 const char *ctp_status_string(ctp_status status);
 

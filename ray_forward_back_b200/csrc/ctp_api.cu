@@ -160,152 +160,162 @@ ctp_status validate_desc(const ctp_geom_desc *d) {
   return CTP_OK;
 }
 
-// Per-view records and per-view guards.  Host FP64 throughout.
-ctp_status build_views(const ctp_geom_desc *d, std::vector<ViewRec> &views, std::vector<double> &trig) {
-  const int64_t nv = d->n_views, nr = d->n_rows, nc = d->n_cols;
+// One view's FP64 record and its guards; for a cylindrical detector also
+// the row of column cos/sin values (2 * n_cols doubles at trig_row).
+ctp_status build_view(const ctp_geom_desc *d, int64_t v, ViewRec &V, double *trig_row) {
+  const int64_t nr = d->n_rows, nc = d->n_cols;
   const double cc = 0.5 * (double)(nc - 1), rc = 0.5 * (double)(nr - 1);
   const double n3[3] = {(double)d->nx, (double)d->ny, (double)d->nz};
   double centre_w[3];
   for (int k = 0; k < 3; ++k) centre_w[k] = d->origin[k] + 0.5 * n3[k] * d->spacing[k];
   const double smin = std::fmin(d->spacing[0], std::fmin(d->spacing[1], d->spacing[2]));
+  V = ViewRec{};
+  const double *s = d->src + 3 * v, *dc = d->det_c + 3 * v, *du = d->det_u + 3 * v, *dv = d->det_v + 3 * v;
+  if (!finite3(s) || !finite3(dc) || !finite3(du) || !finite3(dv))
+    return fail(CTP_ERR_INVALID_ARGUMENT, "view %lld: a vector is not finite", (long long)v);
+  const double nu = norm(du), nvl = norm(dv);
+  if (!(nu > 0.0) || !(nvl > 0.0))
+    return fail(CTP_ERR_INVALID_ARGUMENT, "view %lld: det_u and det_v must be non-zero", (long long)v);
+  V.vlen = nvl;
+  for (int k = 0; k < 3; ++k) V.vhat[k] = dv[k] / nvl;
+  for (int k = 0; k < 3; ++k) V.dv[k] = dv[k];
+  if (d->beam == CTP_BEAM_PARALLEL) {
+    const double ns = norm(s);
+    if (!(ns > 0.0)) return fail(CTP_ERR_DEGENERATE_RAY, "view %lld: zero ray direction", (long long)v);
+    for (int k = 0; k < 3; ++k) {
+      V.s[k] = s[k] / ns;
+      V.p00[k] = dc[k] - cc * du[k] - rc * dv[k];
+      V.du[k] = du[k];
+      const double dvox = V.s[k] / d->spacing[k];
+      V.rcp_dir[k] = dvox != 0.0 ? 1.0 / dvox : HUGE_VAL;
+    }
+    if (!invert_columns(du, dv, V.s, V.minv))
+      return fail(CTP_ERR_DEGENERATE_RAY, "view %lld: ray direction lies in the detector plane", (long long)v);
+  } else if (d->detector == CTP_DET_FLAT) {
+    double n[3];
+    cross(du, dv, n);
+    const double nn = norm(n);
+    if (!(nn > 1e-12 * nu * nvl))
+      return fail(CTP_ERR_INVALID_ARGUMENT, "view %lld: det_u and det_v are parallel", (long long)v);
+    for (int k = 0; k < 3; ++k) {
+      V.s[k] = s[k];
+      V.p00[k] = dc[k] - cc * du[k] - rc * dv[k];
+      V.du[k] = du[k];
+    }
+    // Source / pixel coincidence: only possible if the source lies in the detector plane.
+    double rel[3] = {s[0] - dc[0], s[1] - dc[1], s[2] - dc[2]};
+    const double h = std::fabs(dot(rel, n)) / nn;
+    const double scale = std::fmax(norm(rel), std::fmax(nu, nvl));
+    double sp00[3] = {V.p00[0] - s[0], V.p00[1] - s[1], V.p00[2] - s[2]};
+    if (!(h > 1e-12 * scale)) {
+      // coordinates of the source in the pixel lattice
+      double inv[9];
+      double a[3] = {s[0] - V.p00[0], s[1] - V.p00[1], s[2] - V.p00[2]};
+      if (invert_columns(du, dv, n, inv)) {
+        const double cs = inv[0] * a[0] + inv[1] * a[1] + inv[2] * a[2];
+        const double rs = inv[3] * a[0] + inv[4] * a[1] + inv[5] * a[2];
+        const double ci = std::round(cs), ri = std::round(rs);
+        if (std::fabs(cs - ci) < 1e-9 && std::fabs(rs - ri) < 1e-9 && ci >= 0 && ci < (double)nc && ri >= 0 &&
+            ri < (double)nr)
+          return fail(CTP_ERR_DEGENERATE_RAY, "view %lld: the source coincides with pixel (%g, %g)", (long long)v,
+                      ri, ci);
+      }
+      V.full_footprint = 1;
+    } else if (!invert_columns(sp00, du, dv, V.minv)) {
+      V.full_footprint = 1;
+    }
+    // distance guards at the detector corners (pixel distance is convex over the plane)
+    const double ds = vox_dist(s, centre_w, d->spacing);
+    double dp_max = 0.0;
+    for (int corner = 0; corner < 4; ++corner) {
+      double p[3];
+      host_pixel(V, CTP_DET_FLAT, (corner & 1) ? nr - 1 : 0, (corner & 2) ? nc - 1 : 0, p);
+      dp_max = std::fmax(dp_max, vox_dist(p, centre_w, d->spacing));
+    }
+    if (!(ds <= kFarLimit && dp_max <= kFarLimit))
+      return fail(CTP_ERR_OUT_OF_RANGE, "view %lld: an endpoint is beyond 1e15 voxels", (long long)v);
+    if (!(ds <= kNearLimit || dp_max <= kNearLimit))
+      return fail(CTP_ERR_OUT_OF_RANGE, "view %lld: no endpoint within 1e6 voxels of the volume centre",
+                  (long long)v);
+  } else {
+    // cylindrical detector centred on the source's axis
+    const double uhat[3] = {du[0] / nu, du[1] / nu, du[2] / nu};
+    double w0[3] = {dc[0] - s[0], dc[1] - s[1], dc[2] - s[2]};
+    const double axial = dot(w0, V.vhat);
+    double wp[3];
+    for (int k = 0; k < 3; ++k) wp[k] = w0[k] - axial * V.vhat[k];
+    const double R = norm(wp);
+    if (!(R > 1e-9 * std::fmax(norm(w0), 1.0)))
+      return fail(CTP_ERR_DEGENERATE_RAY, "view %lld: the detector centre lies on the source's axis", (long long)v);
+    if (std::fabs(dot(uhat, V.vhat)) > 1e-9)
+      return fail(CTP_ERR_INVALID_ARGUMENT, "view %lld: det_u must be orthogonal to det_v", (long long)v);
+    if (std::fabs(dot(uhat, wp)) > 1e-9 * R)
+      return fail(CTP_ERR_INVALID_ARGUMENT, "view %lld: det_u must be orthogonal to det_c - src", (long long)v);
+    V.R = R;
+    for (int k = 0; k < 3; ++k) {
+      V.s[k] = s[k];
+      V.w[k] = wp[k] / R;
+      V.du[k] = uhat[k];
+    }
+    V.dgam = nu / R;
+    V.gam0 = -cc * V.dgam;
+    V.axial0 = axial - rc * nvl;
+    for (int k = 0; k < 3; ++k) V.p00[k] = s[k] + V.axial0 * V.vhat[k];
+    if (trig_row)
+      for (int64_t c = 0; c < nc; ++c) {
+        const double g = V.gam0 + (double)c * V.dgam;
+        trig_row[2 * c] = std::cos(g);
+        trig_row[2 * c + 1] = std::sin(g);
+      }
+    // distance guards: a bound first, the exact per-pixel check only if it fails
+    const double ds = vox_dist(s, centre_w, d->spacing);
+    const double row_ext = std::fmax(std::fabs(V.axial0), std::fabs(V.axial0 + (double)(nr - 1) * nvl));
+    const double bound = ds + (R + row_ext) / smin;
+    double dp_max = bound;
+    if (!(ds <= kNearLimit || bound <= kNearLimit) || !(bound <= kFarLimit)) {
+      dp_max = 0.0;
+      for (int64_t r = 0; r < nr; ++r)
+        for (int64_t c = 0; c < nc; ++c) {
+          double p[3];
+          const double g = V.gam0 + (double)c * V.dgam;
+          for (int k = 0; k < 3; ++k)
+            p[k] = V.p00[k] + (double)r * V.dv[k] + R * (std::cos(g) * V.w[k] + std::sin(g) * V.du[k]);
+          dp_max = std::fmax(dp_max, vox_dist(p, centre_w, d->spacing));
+        }
+    }
+    if (!(ds <= kFarLimit && dp_max <= kFarLimit))
+      return fail(CTP_ERR_OUT_OF_RANGE, "view %lld: an endpoint is beyond 1e15 voxels", (long long)v);
+    if (!(ds <= kNearLimit || dp_max <= kNearLimit))
+      return fail(CTP_ERR_OUT_OF_RANGE, "view %lld: no endpoint within 1e6 voxels of the volume centre",
+                  (long long)v);
+  }
+  // extent of one voxel's projection, used to bound the rays per voxel
+  if (d->beam == CTP_BEAM_PARALLEL) {
+    for (int i = 0; i < 2; ++i)
+      V.vox_ext[i] = std::fabs(V.minv[3 * i]) * d->spacing[0] + std::fabs(V.minv[3 * i + 1]) * d->spacing[1] +
+                     std::fabs(V.minv[3 * i + 2]) * d->spacing[2];
+  } else if (d->detector == CTP_DET_FLAT) {
+    for (int i = 0; i < 3; ++i)
+      V.vox_ext[i] = std::fabs(V.minv[3 * i]) * d->spacing[0] + std::fabs(V.minv[3 * i + 1]) * d->spacing[1] +
+                     std::fabs(V.minv[3 * i + 2]) * d->spacing[2];
+  }
+  // forward gather layout: y-fastest copy when the column step runs mostly along y
+  const double ux = std::fabs(du[0] / d->spacing[0]), uy = std::fabs(du[1] / d->spacing[1]),
+               uz = std::fabs(du[2] / d->spacing[2]);
+  V.layout = (uy > ux && uy >= uz) ? 1 : 0;
+  if (d->plan && d->plan->forward_layout == 1) V.layout = 0;
+  if (d->plan && d->plan->forward_layout == 2) V.layout = 1;
+  return CTP_OK;
+}
+
+// Per-view records and per-view guards of all views.  Host FP64 throughout.
+ctp_status build_views(const ctp_geom_desc *d, std::vector<ViewRec> &views, std::vector<double> &trig) {
+  const int64_t nv = d->n_views, nc = d->n_cols;
   views.assign((size_t)nv, ViewRec{});
   if (d->detector == CTP_DET_CYLINDRICAL) trig.assign((size_t)(2 * nv * nc), 0.0);
   for (int64_t v = 0; v < nv; ++v) {
-    const double *s = d->src + 3 * v, *dc = d->det_c + 3 * v, *du = d->det_u + 3 * v, *dv = d->det_v + 3 * v;
-    if (!finite3(s) || !finite3(dc) || !finite3(du) || !finite3(dv))
-      return fail(CTP_ERR_INVALID_ARGUMENT, "view %lld: a vector is not finite", (long long)v);
-    const double nu = norm(du), nvl = norm(dv);
-    if (!(nu > 0.0) || !(nvl > 0.0))
-      return fail(CTP_ERR_INVALID_ARGUMENT, "view %lld: det_u and det_v must be non-zero", (long long)v);
-    ViewRec &V = views[(size_t)v];
-    V.vlen = nvl;
-    for (int k = 0; k < 3; ++k) V.vhat[k] = dv[k] / nvl;
-    for (int k = 0; k < 3; ++k) V.dv[k] = dv[k];
-    if (d->beam == CTP_BEAM_PARALLEL) {
-      const double ns = norm(s);
-      if (!(ns > 0.0)) return fail(CTP_ERR_DEGENERATE_RAY, "view %lld: zero ray direction", (long long)v);
-      for (int k = 0; k < 3; ++k) {
-        V.s[k] = s[k] / ns;
-        V.p00[k] = dc[k] - cc * du[k] - rc * dv[k];
-        V.du[k] = du[k];
-        const double dvox = V.s[k] / d->spacing[k];
-        V.rcp_dir[k] = dvox != 0.0 ? 1.0 / dvox : HUGE_VAL;
-      }
-      if (!invert_columns(du, dv, V.s, V.minv))
-        return fail(CTP_ERR_DEGENERATE_RAY, "view %lld: ray direction lies in the detector plane", (long long)v);
-    } else if (d->detector == CTP_DET_FLAT) {
-      double n[3];
-      cross(du, dv, n);
-      const double nn = norm(n);
-      if (!(nn > 1e-12 * nu * nvl))
-        return fail(CTP_ERR_INVALID_ARGUMENT, "view %lld: det_u and det_v are parallel", (long long)v);
-      for (int k = 0; k < 3; ++k) {
-        V.s[k] = s[k];
-        V.p00[k] = dc[k] - cc * du[k] - rc * dv[k];
-        V.du[k] = du[k];
-      }
-      // Source / pixel coincidence: only possible if the source lies in the detector plane.
-      double rel[3] = {s[0] - dc[0], s[1] - dc[1], s[2] - dc[2]};
-      const double h = std::fabs(dot(rel, n)) / nn;
-      const double scale = std::fmax(norm(rel), std::fmax(nu, nvl));
-      double sp00[3] = {V.p00[0] - s[0], V.p00[1] - s[1], V.p00[2] - s[2]};
-      if (!(h > 1e-12 * scale)) {
-        // coordinates of the source in the pixel lattice
-        double inv[9];
-        double a[3] = {s[0] - V.p00[0], s[1] - V.p00[1], s[2] - V.p00[2]};
-        if (invert_columns(du, dv, n, inv)) {
-          const double cs = inv[0] * a[0] + inv[1] * a[1] + inv[2] * a[2];
-          const double rs = inv[3] * a[0] + inv[4] * a[1] + inv[5] * a[2];
-          const double ci = std::round(cs), ri = std::round(rs);
-          if (std::fabs(cs - ci) < 1e-9 && std::fabs(rs - ri) < 1e-9 && ci >= 0 && ci < (double)nc && ri >= 0 &&
-              ri < (double)nr)
-            return fail(CTP_ERR_DEGENERATE_RAY, "view %lld: the source coincides with pixel (%g, %g)", (long long)v,
-                        ri, ci);
-        }
-        V.full_footprint = 1;
-      } else if (!invert_columns(sp00, du, dv, V.minv)) {
-        V.full_footprint = 1;
-      }
-      // distance guards at the detector corners (pixel distance is convex over the plane)
-      const double ds = vox_dist(s, centre_w, d->spacing);
-      double dp_max = 0.0;
-      for (int corner = 0; corner < 4; ++corner) {
-        double p[3];
-        host_pixel(V, CTP_DET_FLAT, (corner & 1) ? nr - 1 : 0, (corner & 2) ? nc - 1 : 0, p);
-        dp_max = std::fmax(dp_max, vox_dist(p, centre_w, d->spacing));
-      }
-      if (!(ds <= kFarLimit && dp_max <= kFarLimit))
-        return fail(CTP_ERR_OUT_OF_RANGE, "view %lld: an endpoint is beyond 1e15 voxels", (long long)v);
-      if (!(ds <= kNearLimit || dp_max <= kNearLimit))
-        return fail(CTP_ERR_OUT_OF_RANGE, "view %lld: no endpoint within 1e6 voxels of the volume centre",
-                    (long long)v);
-    } else {
-      // cylindrical detector centred on the source's axis
-      const double uhat[3] = {du[0] / nu, du[1] / nu, du[2] / nu};
-      double w0[3] = {dc[0] - s[0], dc[1] - s[1], dc[2] - s[2]};
-      const double axial = dot(w0, V.vhat);
-      double wp[3];
-      for (int k = 0; k < 3; ++k) wp[k] = w0[k] - axial * V.vhat[k];
-      const double R = norm(wp);
-      if (!(R > 1e-9 * std::fmax(norm(w0), 1.0)))
-        return fail(CTP_ERR_DEGENERATE_RAY, "view %lld: the detector centre lies on the source's axis", (long long)v);
-      if (std::fabs(dot(uhat, V.vhat)) > 1e-9)
-        return fail(CTP_ERR_INVALID_ARGUMENT, "view %lld: det_u must be orthogonal to det_v", (long long)v);
-      if (std::fabs(dot(uhat, wp)) > 1e-9 * R)
-        return fail(CTP_ERR_INVALID_ARGUMENT, "view %lld: det_u must be orthogonal to det_c - src", (long long)v);
-      V.R = R;
-      for (int k = 0; k < 3; ++k) {
-        V.s[k] = s[k];
-        V.w[k] = wp[k] / R;
-        V.du[k] = uhat[k];
-      }
-      V.dgam = nu / R;
-      V.gam0 = -cc * V.dgam;
-      V.axial0 = axial - rc * nvl;
-      for (int k = 0; k < 3; ++k) V.p00[k] = s[k] + V.axial0 * V.vhat[k];
-      for (int64_t c = 0; c < nc; ++c) {
-        const double g = V.gam0 + (double)c * V.dgam;
-        trig[(size_t)(2 * (v * nc + c))] = std::cos(g);
-        trig[(size_t)(2 * (v * nc + c) + 1)] = std::sin(g);
-      }
-      // distance guards: a bound first, the exact per-pixel check only if it fails
-      const double ds = vox_dist(s, centre_w, d->spacing);
-      const double row_ext = std::fmax(std::fabs(V.axial0), std::fabs(V.axial0 + (double)(nr - 1) * nvl));
-      const double bound = ds + (R + row_ext) / smin;
-      double dp_max = bound;
-      if (!(ds <= kNearLimit || bound <= kNearLimit) || !(bound <= kFarLimit)) {
-        dp_max = 0.0;
-        for (int64_t r = 0; r < nr; ++r)
-          for (int64_t c = 0; c < nc; ++c) {
-            double p[3];
-            const double g = V.gam0 + (double)c * V.dgam;
-            for (int k = 0; k < 3; ++k)
-              p[k] = V.p00[k] + (double)r * V.dv[k] + R * (std::cos(g) * V.w[k] + std::sin(g) * V.du[k]);
-            dp_max = std::fmax(dp_max, vox_dist(p, centre_w, d->spacing));
-          }
-      }
-      if (!(ds <= kFarLimit && dp_max <= kFarLimit))
-        return fail(CTP_ERR_OUT_OF_RANGE, "view %lld: an endpoint is beyond 1e15 voxels", (long long)v);
-      if (!(ds <= kNearLimit || dp_max <= kNearLimit))
-        return fail(CTP_ERR_OUT_OF_RANGE, "view %lld: no endpoint within 1e6 voxels of the volume centre",
-                    (long long)v);
-    }
-    // extent of one voxel's projection, used to bound the rays per voxel
-    if (d->beam == CTP_BEAM_PARALLEL) {
-      for (int i = 0; i < 2; ++i)
-        V.vox_ext[i] = std::fabs(V.minv[3 * i]) * d->spacing[0] + std::fabs(V.minv[3 * i + 1]) * d->spacing[1] +
-                       std::fabs(V.minv[3 * i + 2]) * d->spacing[2];
-    } else if (d->detector == CTP_DET_FLAT) {
-      for (int i = 0; i < 3; ++i)
-        V.vox_ext[i] = std::fabs(V.minv[3 * i]) * d->spacing[0] + std::fabs(V.minv[3 * i + 1]) * d->spacing[1] +
-                       std::fabs(V.minv[3 * i + 2]) * d->spacing[2];
-    }
-    // forward gather layout: y-fastest copy when the column step runs mostly along y
-    const double ux = std::fabs(du[0] / d->spacing[0]), uy = std::fabs(du[1] / d->spacing[1]),
-                 uz = std::fabs(du[2] / d->spacing[2]);
-    V.layout = (uy > ux && uy >= uz) ? 1 : 0;
-    if (d->plan && d->plan->forward_layout == 1) V.layout = 0;
-    if (d->plan && d->plan->forward_layout == 2) V.layout = 1;
+    const ctp_status st = build_view(d, v, views[(size_t)v], trig.empty() ? nullptr : trig.data() + 2 * v * nc);
+    if (st != CTP_OK) return st;
   }
   return CTP_OK;
 }
@@ -430,6 +440,19 @@ ctp_status measure_collision_ratio(ctp_geom *g, const std::vector<ViewRec> &view
 }
 
 }  // namespace
+
+// Host helpers shared with the entry point that allocates nothing
+// (ctp_noalloc.cu); thin wrappers over the functions above.
+namespace ctp {
+ctp_status host_validate(const ctp_geom_desc *d) { return validate_desc(d); }
+ctp_status host_view_record(const ctp_geom_desc *d, int64_t v, ViewRec &V, double *trig_row) {
+  return build_view(d, v, V, trig_row);
+}
+ctp_status host_error(ctp_status s, const char *msg) { return fail(s, "%s", msg); }
+ctp_status host_cuda_error(cudaError_t e, const char *where) { return cuda_fail(e, where); }
+bool host_is_device_pointer(const void *ptr, int device) { return is_device_pointer(ptr, device); }
+void host_clear_error() { g_detail[0] = '\0'; }
+}  // namespace ctp
 
 extern "C" {
 

@@ -80,6 +80,14 @@ cudaError_t launch_back_sort(const FwdLaunch& p, const ViewRec* views, const dou
 cudaError_t launch_collision_count(const FwdLaunch& p, const ViewRec* views, const double* trig,
                                    unsigned long long* counters, bool wide_index, cudaStream_t stream);
 size_t back_brick_smem_bytes(const int32_t brick[3]);
+
+// Host helpers (ctp_api.cu).
+ctp_status host_validate(const ctp_geom_desc* d);
+ctp_status host_view_record(const ctp_geom_desc* d, int64_t v, ViewRec& V, double* trig_row);
+ctp_status host_error(ctp_status s, const char* msg);
+ctp_status host_cuda_error(cudaError_t e, const char* where);
+bool host_is_device_pointer(const void* ptr, int device);
+void host_clear_error();
 cudaError_t prepare_back_brick(size_t smem_bytes);
 
 }  // namespace ctp

@@ -35,7 +35,8 @@ CTP_ADJOINT_BRICK = 1
 CTP_ADJOINT_SORT = 2
 
 EXPORTED = ["ctp_geom_create", "ctp_geom_destroy", "ctp_geom_query", "ctp_forward", "ctp_back",
-            "ctp_count_updates", "ctp_status_string", "ctp_last_error_detail", "ctp_version"]
+            "ctp_count_updates", "ctp_forward_noalloc", "ctp_status_string", "ctp_last_error_detail",
+            "ctp_version"]
 
 
 class ctp_plan(ctypes.Structure):
@@ -95,6 +96,8 @@ def load(path: str = None):
         lib.ctp_back.restype = ctypes.c_int
         lib.ctp_count_updates.argtypes = [vp, ctypes.POINTER(i64), vp]
         lib.ctp_count_updates.restype = ctypes.c_int
+        lib.ctp_forward_noalloc.argtypes = [ctypes.POINTER(ctp_geom_desc), vp, vp, vp]
+        lib.ctp_forward_noalloc.restype = ctypes.c_int
         lib.ctp_status_string.argtypes = [ctypes.c_int]
         lib.ctp_status_string.restype = ctypes.c_char_p
         lib.ctp_last_error_detail.argtypes = []
@@ -198,6 +201,17 @@ def ctp_count_updates(handle: int, stream=None) -> int:
     n = ctypes.c_int64()
     _check(load().ctp_count_updates(handle, ctypes.byref(n), _stream_handle(stream)))
     return int(n.value)
+
+
+def ctp_forward_noalloc(geom, vol, sino, device: int = 0, plan: Optional[dict] = None, stream=None) -> None:
+    """Forward projection without any allocation by the library: the
+    geometry is passed as a description, scratch is the library's fixed
+    device array (see include/ctp.h)."""
+    desc = _Desc(geom, device, plan)
+    _check(load().ctp_forward_noalloc(ctypes.byref(desc.desc), _ptr(vol), _ptr(sino), _stream_handle(stream)))
+
+
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 def ctp_version() -> str:
