@@ -324,3 +324,24 @@ def test_collision_ratio_measured_and_dispatch_consistent():
         ref = oracle.back(g, sino)
         check_back(gpu_back(P, sino), ref, oracle.back(g, sino, power=0),
                    float(np.linalg.norm(np.array([g.nx, g.ny, g.nz]) * np.array(g.spacing))), "auto")
+
+
+def _stored_counts():
+    rows = {}
+    path = __file__.replace("test_parity_gpu.py", "golden/update_counts.txt")
+    for line in open(path):
+        if line.strip() and not line.startswith("#"):
+            i, n = line.split()
+            rows[int(i)] = int(n)
+    return rows
+
+
+@pytest.mark.parametrize("index", [0, 1, 2, 3])
+def test_device_update_count_matches_oracle_fixture(index):
+    """The device's count of positive-length segments for each full workload
+    equals the oracle's exact count (stored by tests/golden/make_update_counts.py)
+    up to segments whose length rounds across zero (ties at voxel corners)."""
+    ref = _stored_counts()[index]
+    P = projector(W.workload(index).geom)
+    got = P.count_updates()
+    assert abs(got - ref) <= 1e-4 * ref, (got, ref)
