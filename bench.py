@@ -51,6 +51,25 @@ def workload_config(wl):
             "seed": wl.seed, "l2": "inputs larger than L2 (volume and sinogram each > 126 MB)"}
 
 
+def measured_traffic(kernel, workload_index):
+    """Per-launch DRAM bytes of `kernel` from the committed one-pass ncu
+    capture, or None when the capture is for another workload or the kernel
+    source has changed since it was taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "dram_traffic_parallel512_900views.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        with open(os.path.join(ROOT, rec["kernel_source"]), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except Exception:
+        return None
+    if sha != rec.get("kernel_source_sha256") or workload_index != 4:
+        return None
+    k = rec["kernels"].get(kernel)
+    return int(k["dram_bytes_per_launch"]) if k else None
+
+
 def algorithmic_bytes(U, n_vox, n_rays):
     """4 B per ray-voxel update (one FP32 voxel read or accumulation) plus the
     compulsory read/write of every voxel and every sinogram element once."""
@@ -176,6 +195,75 @@ def run_reference(args, rank, world):
     return 0
 
 
+def run_e2e(args, P, g, wl, vol_host, U, world, dev):
+    """End-to-end steps through the public API from and to pinned host
+    memory: every step copies its volume and sinogram in and its sinogram and
+    volume results out.  Copies run on their own streams with double-buffered
+    device buffers, so step k's transfers overlap the neighbouring steps'
+    projections; the timed region spans the first copy-in to the last
+    copy-out, CUDA events, max over ranks."""
+    import torch
+    vol_pin = torch.from_numpy(vol_host).pin_memory()
+    sino_pin = torch.from_numpy(wl.sinogram()).pin_memory()
+    sino_res = torch.empty(g.sino_shape, dtype=torch.float32).pin_memory()
+    vol_res = torch.empty(g.vol_shape, dtype=torch.float32).pin_memory()
+    s_in, s_comp, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
+    vol_d = [torch.empty(g.vol_shape, dtype=torch.float32, device=dev) for _ in range(2)]
+    sino_d = [torch.empty(g.sino_shape, dtype=torch.float32, device=dev) for _ in range(2)]
+    y_d = [torch.empty(g.sino_shape, dtype=torch.float32, device=dev) for _ in range(2)]
+    x_d = [torch.empty(g.vol_shape, dtype=torch.float32, device=dev) for _ in range(2)]
+    done_out = [torch.cuda.Event() for _ in range(2)]   # buffer b free again
+    done_comp = [torch.cuda.Event() for _ in range(2)]
+
+    def step(k):
+        b = k & 1
+        ev_in = torch.cuda.Event()
+        s_in.wait_event(done_comp[b])          # inputs of buffer b no longer read
+        with torch.cuda.stream(s_in):
+            vol_d[b].copy_(vol_pin, non_blocking=True)
+            sino_d[b].copy_(sino_pin, non_blocking=True)
+        ev_in.record(s_in)
+        s_comp.wait_event(ev_in)
+        s_comp.wait_event(done_out[b])         # outputs of buffer b already copied out
+        P.forward(vol_d[b], out=y_d[b], stream=s_comp)
+        ev_y = torch.cuda.Event()
+        ev_y.record(s_comp)
+        P.back(sino_d[b], out=x_d[b], stream=s_comp)
+        done_comp[b].record(s_comp)
+        s_out.wait_event(ev_y)
+        with torch.cuda.stream(s_out):
+            sino_res.copy_(y_d[b], non_blocking=True)
+        s_out.wait_event(done_comp[b])
+        with torch.cuda.stream(s_out):
+            vol_res.copy_(x_d[b], non_blocking=True)
+        done_out[b].record(s_out)
+
+    for b in range(2):
+        done_out[b].record(s_out)
+        done_comp[b].record(s_comp)
+    for k in range(max(1, min(args.warmup, 2))):
+        step(k)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(s_in)
+    s_comp.wait_event(t0)
+    s_out.wait_event(t0)
+    for k in range(args.steps):
+        step(k)
+    s_in.wait_event(done_out[(args.steps - 1) & 1])
+    t1.record(s_in)
+    torch.cuda.synchronize(dev)
+    e2e_ms = aggregate_over_ranks([t0.elapsed_time(t1) / args.steps], world, dev)[0]
+    return {"value": throughput(2 * U, world, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
+            "h2d_bytes_per_step": int(vol_pin.numel() * 4 + sino_pin.numel() * 4),
+            "d2h_bytes_per_step": int(sino_res.numel() * 4 + vol_res.numel() * 4),
+            "pipelining": "copies on separate streams, double-buffered device buffers"}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -242,42 +330,16 @@ def run_ours(args, rank, world, local_rank):
     # end to end through the public API with host buffers (pinned), every step
     e2e = None
     if not args.no_e2e:
-        vol_pin = torch.from_numpy(vol_host).pin_memory()
-        sino_pin = torch.from_numpy(wl.sinogram()).pin_memory()
-        sino_res = torch.empty(g.sino_shape, dtype=torch.float32).pin_memory()
-        vol_res = torch.empty(g.vol_shape, dtype=torch.float32).pin_memory()
-
-        def e2e_step():
-            with torch.cuda.stream(stream):
-                vol_d = vol_pin.to(dev, non_blocking=True)
-                y = P.forward(vol_d, stream=stream)
-                sino_res.copy_(y, non_blocking=True)
-                sino_d = sino_pin.to(dev, non_blocking=True)
-                x = P.back(sino_d, stream=stream)
-                vol_res.copy_(x, non_blocking=True)
-
-        for _ in range(max(1, min(args.warmup, 2))):
-            e2e_step()
-        stream.synchronize()
-        if world > 1:
-            dist.barrier()
-        s0 = torch.cuda.Event(enable_timing=True)
-        s1 = torch.cuda.Event(enable_timing=True)
-        s0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        s1.record(stream)
-        torch.cuda.synchronize(dev)
-        e2e_ms = aggregate_over_ranks([s0.elapsed_time(s1) / args.steps], world, dev)[0]
-        e2e = {"value": throughput(2 * U, world, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
-               "h2d_bytes_per_step": int(vol_pin.numel() * 4 + sino_pin.numel() * 4),
-               "d2h_bytes_per_step": int(sino_res.numel() * 4 + vol_res.numel() * 4)}
-
+        e2e = run_e2e(args, P, g, wl, vol_host, U, world, dev)
     if rank != 0:
         return 0
     peak, peak_kind = measured_hbm_peak()
     B = algorithmic_bytes(U, g.n_vox, g.n_rays)
     dominant = "back" if back_avg >= fwd_avg else "forward"
+    if dominant == "back":
+        dom_kernel = "back_sort_kernel" if info["adjoint_variant"] == 2 else "back_brick_kernel"
+    else:
+        dom_kernel = "forward_kernel"
     dom_ms = max(back_avg, fwd_avg)
     achieved = B / (dom_ms * 1e-3) / 1e9
     cpu = None
@@ -300,9 +362,10 @@ def run_ours(args, rank, world, local_rank):
                  "effective_gbs": B / (back_avg * 1e-3) / 1e9,
                  "frac_of_hbm": B / (back_avg * 1e-3) / 1e9 / peak,
                  "variant": info["adjoint_variant"], "brick": info["brick"], "view_groups": info["view_groups"]},
-        "roofline": {"kernel": "back_brick_kernel" if dominant == "back" else "forward_kernel",
+        "roofline": {"kernel": dom_kernel,
                      "bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs",
-                     "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                     "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": measured_traffic(dom_kernel, wl.index) if not args.views else None,
                      "algorithmic_bytes_per_launch": B},
         "clocks": clk,
         "e2e": e2e,

@@ -161,6 +161,18 @@ ctp_status ctp_forward(const ctp_geom *geom, const float *vol, float *sino, void
 ctp_status ctp_back(const ctp_geom *geom, const float *sino, float *vol, void *stream);
 
 /*
+ * ctp_back_power — vol = (A∘A)^T sino for power 2 (every coefficient squared)
+ * or A^T sino for power 1 (identical to ctp_back).  Back projection with
+ * squared weights gives the diagonal of the normal operator used for
+ * Hessian-diagonal preconditioning (MBIRJAX "Projector kernels", paragraph
+ * "Gradient and Hessian can take different paths": back projection with the
+ * weights unchanged for the gradient and squared for the Hessian diagonal).
+ * Same pointer, stream and synchronisation rules as ctp_back; other powers
+ * give CTP_ERR_INVALID_ARGUMENT.
+ */
+ctp_status ctp_back_power(const ctp_geom *geom, const float *sino, float *vol, int power, void *stream);
+
+/*
  * ctp_count_updates — the number of positive-length ray-voxel segments of the
  * whole acquisition (the work measure of both projectors), computed on the
  * device.  Synchronous: waits for the count and writes it to *host_out.

@@ -618,8 +618,13 @@ ctp_status ctp_forward(const ctp_geom *g, const float *vol, float *sino, void *s
 }
 
 ctp_status ctp_back(const ctp_geom *g, const float *sino, float *vol, void *stream) {
+  return ctp_back_power(g, sino, vol, 1, stream);
+}
+
+ctp_status ctp_back_power(const ctp_geom *g, const float *sino, float *vol, int power, void *stream) {
   g_detail[0] = '\0';
   if (!g) return fail(CTP_ERR_INVALID_ARGUMENT, "geometry is NULL");
+  if (power != 1 && power != 2) return fail(CTP_ERR_INVALID_ARGUMENT, "power %d is not 1 or 2", power);
   DeviceGuard dg(g->device);
   if (dg.err != cudaSuccess) return cuda_fail(dg.err, "cudaSetDevice");
   if (!is_device_pointer(sino, g->device))
@@ -635,9 +640,9 @@ ctp_status ctp_back(const ctp_geom *g, const float *sino, float *vol, void *stre
     if (e != cudaSuccess) return cuda_fail(e, "volume zero-fill");
   }
   if (sorted)
-    e = ctp::launch_back_sort(g->fwd, g->d_views, g->d_trig, sino, vol, g->wide_index, s);
+    e = ctp::launch_back_sort(g->fwd, g->d_views, g->d_trig, sino, vol, power, g->wide_index, s);
   else
-    e = ctp::launch_back_brick(g->back, g->d_views, g->d_trig, sino, vol, g->wide_index, s);
+    e = ctp::launch_back_brick(g->back, g->d_views, g->d_trig, sino, vol, power, g->wide_index, s);
   if (e != cudaSuccess) return cuda_fail(e, "adjoint launch");
   return CTP_OK;
 }

@@ -72,11 +72,11 @@ cudaError_t launch_transpose_xy(const float* vol, float* volT, const VolDesc& vd
 cudaError_t launch_forward(const FwdLaunch& p, const ViewRec* views, const double* trig, const float* vol,
                            const float* volT, float* sino, bool wide_index, cudaStream_t stream);
 cudaError_t launch_back_brick(const BackLaunch& p, const ViewRec* views, const double* trig, const float* sino,
-                              float* vol, bool wide_index, cudaStream_t stream);
+                              float* vol, int power, bool wide_index, cudaStream_t stream);
 cudaError_t launch_count(const FwdLaunch& p, const ViewRec* views, const double* trig,
                          unsigned long long* counter, cudaStream_t stream);
 cudaError_t launch_back_sort(const FwdLaunch& p, const ViewRec* views, const double* trig, const float* sino,
-                             float* vol, bool wide_index, cudaStream_t stream);
+                             float* vol, int power, bool wide_index, cudaStream_t stream);
 cudaError_t launch_collision_count(const FwdLaunch& p, const ViewRec* views, const double* trig,
                                    unsigned long long* counters, bool wide_index, cudaStream_t stream);
 size_t back_brick_smem_bytes(const int32_t brick[3]);

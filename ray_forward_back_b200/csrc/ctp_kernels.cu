@@ -61,12 +61,6 @@ constexpr int kWalk3Unroll = CTP_WALK3_UNROLL;
 constexpr int kFwdCols = 32;  // threads along detector columns per block
 constexpr int kFwdRows = 8;   // detector rows per block (row band height)
 constexpr int kBackThreads = 256;
-#ifndef CTP_BACK_WARP_WALK
-#define CTP_BACK_WARP_WALK 0
-#endif
-#ifndef CTP_BACK_ALIGN
-#define CTP_BACK_ALIGN 0
-#endif
 #ifndef CTP_BACK_STAGE
 #define CTP_BACK_STAGE 64
 #endif
@@ -505,6 +499,14 @@ __global__ void __launch_bounds__(256) transpose_xy_kernel(const float* __restri
 
 // -------------------------------------------------------------- back: brick --
 
+// Adjoint coefficient of a segment of physical length len: len (the
+// transpose of the forward projection) or len^2 (squared weights, the
+// diagonal of the normal operator used for Hessian preconditioning).
+template <int kPower>
+__device__ __forceinline__ float coef(float len) {
+  return kPower == 2 ? len * len : len;
+}
+
 // Detector footprint of the brick [lo, hi) in view V: a rectangle of pixels
 // that contains every pixel whose ray can meet the brick.  Also returns
 // nvox, an upper bound on the number of this view's rays that can meet any
@@ -626,7 +628,7 @@ __device__ void brick_footprint(const ViewRec& V, const BackLaunch& P, const int
 // summed per-view ray bounds.  Each stage is then flushed into the FP32
 // volume.  Integer sums are exact, so the result does not depend on the
 // order in which threads add.
-template <typename Off>
+template <int kPower, typename Off>
 __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
     back_brick_kernel(BackLaunch P, const ViewRec* __restrict__ views, const double* __restrict__ trig,
                       const float* __restrict__ sino, float* __restrict__ vol) {
@@ -741,7 +743,8 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
       if (bits >= 0x7f800000u) {
         sc = CUDART_NAN_F;  // non-finite input: the brick is written as NaN
       } else {
-        const double bound = (double)__uint_as_float(bits) * diag * (double)s_nsum;
+        const double seg_max = kPower == 2 ? diag * diag : diag;
+        const double bound = (double)__uint_as_float(bits) * seg_max * (double)s_nsum;
         if (bound > 0.0) sc = (float)((2147483647.0 - 4194304.0) / bound);
       }
       s_scale = sc;
@@ -786,15 +789,10 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
           off = ((W.i[2] - lo[2]) * P.brick[1] + (W.i[1] - lo[1])) * pitch + (W.i[0] - lo[0]);
         }
         const float yS = y * S;
-#if CTP_BACK_WARP_WALK
-        walk<CTP_BACK_ALIGN != 0, false, int>(act, W, lo, hi, off, W.step[0], W.step[1] * pitch, W.step[2] * plane,
-                                            [&](int o, float len, bool) { atomicAdd(acc + o, __float2int_rn(len * yS)); });
-#else
         if (act)
           walk_lane<int>(W, off, W.step[0], W.step[1] * pitch, W.step[2] * plane,
-                         [&](int o, float len) { atomicAdd(acc + o, __float2int_rn(len * yS)); });
+                         [&](int o, float len) { atomicAdd(acc + o, __float2int_rn(coef<kPower>(len) * yS)); });
         __syncwarp();
-#endif
       }
     }
     __syncthreads();
@@ -896,7 +894,7 @@ __device__ __forceinline__ void warp_segment_reduce(Key key, float val, bool val
 // per distinct voxel.  Needs the volume zeroed first.  With kCount it writes
 // nothing and counts contributions and runs (the collision ratio) instead,
 // treating every ray value as 1.
-template <bool kCount, typename Off>
+template <bool kCount, int kPower, typename Off>
 __global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_FWD_MIN_BLOCKS)
     back_sort_kernel(FwdLaunch P, const ViewRec* __restrict__ views, const double* __restrict__ trig,
                      const float* __restrict__ sino, float* __restrict__ vol,
@@ -923,7 +921,9 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_FWD_MIN_BLOCKS)
   const Off off = (Off)W.i[2] * sz + (Off)W.i[1] * nx + (Off)W.i[0];
   unsigned long long n_upd = 0, n_runs = 0;
   walk<true, true, Off>(hit, W, lo, hi, off, (Off)W.step[0], W.step[1] * nx, W.step[2] * sz,
-                        [&](Off o, float len, bool f) { warp_segment_reduce<kCount, Off>(o, len * y, f, vol, n_upd, n_runs); });
+                        [&](Off o, float len, bool f) {
+                          warp_segment_reduce<kCount, Off>(o, coef<kPower>(len) * y, f, vol, n_upd, n_runs);
+                        });
   if (kCount && (threadIdx.x & 31) == 0 && (n_upd | n_runs)) {
     atomicAdd(counters, n_upd);
     atomicAdd(counters + 1, n_runs);
@@ -963,15 +963,19 @@ cudaError_t launch_count(const FwdLaunch& p, const ViewRec* views, const double*
 }
 
 cudaError_t launch_back_sort(const FwdLaunch& p, const ViewRec* views, const double* trig, const float* sino,
-                             float* vol, bool wide_index, cudaStream_t stream) {
+                             float* vol, int power, bool wide_index, cudaStream_t stream) {
   const long long blocks = (long long)p.n_row_bands * p.dims.n_views * p.n_col_tiles;
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   dim3 block(kFwdCols, kFwdRows);
-  if (wide_index)
-    back_sort_kernel<false, long long><<<(unsigned)blocks, block, 0, stream>>>(p, views, trig, sino, vol, nullptr);
-  else
-    back_sort_kernel<false, int><<<(unsigned)blocks, block, 0, stream>>>(p, views, trig, sino, vol, nullptr);
+  const unsigned nb = (unsigned)blocks;
+  if (power == 2) {
+    if (wide_index) back_sort_kernel<false, 2, long long><<<nb, block, 0, stream>>>(p, views, trig, sino, vol, nullptr);
+    else back_sort_kernel<false, 2, int><<<nb, block, 0, stream>>>(p, views, trig, sino, vol, nullptr);
+  } else {
+    if (wide_index) back_sort_kernel<false, 1, long long><<<nb, block, 0, stream>>>(p, views, trig, sino, vol, nullptr);
+    else back_sort_kernel<false, 1, int><<<nb, block, 0, stream>>>(p, views, trig, sino, vol, nullptr);
+  }
   return cudaGetLastError();
 }
 
@@ -982,10 +986,10 @@ cudaError_t launch_collision_count(const FwdLaunch& p, const ViewRec* views, con
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   dim3 block(kFwdCols, kFwdRows);
   if (wide_index)
-    back_sort_kernel<true, long long><<<(unsigned)blocks, block, 0, stream>>>(p, views, trig, nullptr, nullptr,
-                                                                             counters);
+    back_sort_kernel<true, 1, long long><<<(unsigned)blocks, block, 0, stream>>>(p, views, trig, nullptr, nullptr,
+                                                                                counters);
   else
-    back_sort_kernel<true, int><<<(unsigned)blocks, block, 0, stream>>>(p, views, trig, nullptr, nullptr, counters);
+    back_sort_kernel<true, 1, int><<<(unsigned)blocks, block, 0, stream>>>(p, views, trig, nullptr, nullptr, counters);
   return cudaGetLastError();
 }
 
@@ -994,25 +998,33 @@ size_t back_brick_smem_bytes(const int32_t brick[3]) {
 }
 
 cudaError_t prepare_back_brick(size_t smem_bytes) {
-  cudaError_t e = cudaFuncSetAttribute(back_brick_kernel<int>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem_bytes);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(back_brick_kernel<long long>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)smem_bytes);
+  const int b = (int)smem_bytes;
+  cudaError_t e = cudaFuncSetAttribute(back_brick_kernel<1, int>, cudaFuncAttributeMaxDynamicSharedMemorySize, b);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(back_brick_kernel<1, long long>, cudaFuncAttributeMaxDynamicSharedMemorySize, b);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(back_brick_kernel<2, int>, cudaFuncAttributeMaxDynamicSharedMemorySize, b);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(back_brick_kernel<2, long long>, cudaFuncAttributeMaxDynamicSharedMemorySize, b);
+  return e;
 }
 
 cudaError_t launch_back_brick(const BackLaunch& p, const ViewRec* views, const double* trig, const float* sino,
-                              float* vol, bool wide_index, cudaStream_t stream) {
+                              float* vol, int power, bool wide_index, cudaStream_t stream) {
   const long long blocks = (long long)p.nbrick[0] * p.nbrick[1] * p.nbrick[2] * p.view_groups;
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   const size_t smem = back_brick_smem_bytes(p.brick);
   cudaError_t e = prepare_back_brick(smem);
   if (e != cudaSuccess) return e;
-  if (wide_index)
-    back_brick_kernel<long long><<<(unsigned)blocks, kBackThreads, smem, stream>>>(p, views, trig, sino, vol);
-  else
-    back_brick_kernel<int><<<(unsigned)blocks, kBackThreads, smem, stream>>>(p, views, trig, sino, vol);
+  const unsigned nb = (unsigned)blocks;
+  if (power == 2) {
+    if (wide_index) back_brick_kernel<2, long long><<<nb, kBackThreads, smem, stream>>>(p, views, trig, sino, vol);
+    else back_brick_kernel<2, int><<<nb, kBackThreads, smem, stream>>>(p, views, trig, sino, vol);
+  } else {
+    if (wide_index) back_brick_kernel<1, long long><<<nb, kBackThreads, smem, stream>>>(p, views, trig, sino, vol);
+    else back_brick_kernel<1, int><<<nb, kBackThreads, smem, stream>>>(p, views, trig, sino, vol);
+  }
   return cudaGetLastError();
 }
 

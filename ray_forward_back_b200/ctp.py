@@ -35,7 +35,7 @@ CTP_ADJOINT_BRICK = 1
 CTP_ADJOINT_SORT = 2
 
 EXPORTED = ["ctp_geom_create", "ctp_geom_destroy", "ctp_geom_query", "ctp_forward", "ctp_back",
-            "ctp_count_updates", "ctp_forward_noalloc", "ctp_status_string", "ctp_last_error_detail",
+            "ctp_back_power", "ctp_count_updates", "ctp_forward_noalloc", "ctp_status_string", "ctp_last_error_detail",
             "ctp_version"]
 
 
@@ -94,6 +94,8 @@ def load(path: str = None):
         lib.ctp_forward.restype = ctypes.c_int
         lib.ctp_back.argtypes = [vp, vp, vp, vp]
         lib.ctp_back.restype = ctypes.c_int
+        lib.ctp_back_power.argtypes = [vp, vp, vp, ctypes.c_int, vp]
+        lib.ctp_back_power.restype = ctypes.c_int
         lib.ctp_count_updates.argtypes = [vp, ctypes.POINTER(i64), vp]
         lib.ctp_count_updates.restype = ctypes.c_int
         lib.ctp_forward_noalloc.argtypes = [ctypes.POINTER(ctp_geom_desc), vp, vp, vp]
@@ -197,6 +199,10 @@ def ctp_back(handle: int, sino, vol, stream=None) -> None:
     _check(load().ctp_back(handle, _ptr(sino), _ptr(vol), _stream_handle(stream)))
 
 
+def ctp_back_power(handle: int, sino, vol, power: int, stream=None) -> None:
+    _check(load().ctp_back_power(handle, _ptr(sino), _ptr(vol), int(power), _stream_handle(stream)))
+
+
 def ctp_count_updates(handle: int, stream=None) -> int:
     n = ctypes.c_int64()
     _check(load().ctp_count_updates(handle, ctypes.byref(n), _stream_handle(stream)))
@@ -275,6 +281,16 @@ class Projector:
             out = torch.empty(self.geom.vol_shape, dtype=torch.float32, device=sino.device)
         self._check_tensor(out, self.geom.vol_shape, "out")
         ctp_back(self.handle, sino, out, stream)
+        return out
+
+    def back_power(self, sino, power: int, out=None, stream=None):
+        """Back projection with every coefficient raised to ``power`` (1 or 2)."""
+        import torch
+        self._check_tensor(sino, self.geom.sino_shape, "sino")
+        if out is None:
+            out = torch.empty(self.geom.vol_shape, dtype=torch.float32, device=sino.device)
+        self._check_tensor(out, self.geom.vol_shape, "out")
+        ctp_back_power(self.handle, sino, out, power, stream)
         return out
 
     def count_updates(self, stream=None) -> int:

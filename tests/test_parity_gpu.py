@@ -345,3 +345,61 @@ def test_device_update_count_matches_oracle_fixture(index):
     P = projector(W.workload(index).geom)
     got = P.count_updates()
     assert abs(got - ref) <= 1e-4 * ref, (got, ref)
+
+
+# ------------------------------------------------ coefficient powers (NEXT) ---
+
+@pytest.mark.parametrize("variant", [1, 2])
+@pytest.mark.parametrize("name", ["parallel_ragged", "cone_ragged", "helical_ragged", "parallel_tilted"])
+def test_back_squared_coefficients(name, variant):
+    """Back projection with squared weights (the normal operator's diagonal)
+    against the oracle's power-2 back projection.  A segment error d in len
+    becomes 2 len d in len^2, so the per-segment term of the tolerance is
+    scaled by 2 x the voxel diagonal."""
+    g = ragged_geometries()[name]
+    rng = np.random.default_rng(21)
+    sino = rng.random(g.sino_shape).astype(np.float32)
+    P = projector(g, {"adjoint_variant": variant})
+    import torch
+    x = P.back_power(torch.from_numpy(sino).cuda(), 2)
+    torch.cuda.synchronize()
+    diag = float(np.linalg.norm(g.spacing))
+    local = _local_len(P, g) if variant == 1 else float(np.linalg.norm(np.array([g.nx, g.ny, g.nz]) * np.array(g.spacing)))
+    check_back(x.cpu().numpy(), oracle.back(g, sino, power=2), oracle.back(g, np.abs(sino), power=0),
+               2.0 * diag * local, f"{name} power 2")
+
+
+def test_back_power_one_is_back():
+    import torch
+    g = ragged_geometries()["cone_ragged"]
+    P = projector(g)
+    sino = torch.rand(g.sino_shape, device="cuda")
+    a = P.back(sino)
+    b = P.back_power(sino, 1)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_sirt_normalisers_are_projections_of_ones():
+    """Row sums A 1 (ray lengths through the volume) and column sums A^T 1
+    (total ray length per voxel) against the oracle."""
+    import torch
+    g = ragged_geometries()["helical_ragged"]
+    P = projector(g)
+    rows = P.forward(torch.ones(g.vol_shape, device="cuda"))
+    cols = P.back(torch.ones(g.sino_shape, device="cuda"))
+    torch.cuda.synchronize()
+    ones_v = np.ones(g.vol_shape, np.float32)
+    ones_s = np.ones(g.sino_shape, np.float32)
+    check_forward(rows.cpu().numpy(), oracle.forward(g, ones_v), oracle_chords(g), min(g.spacing), "A 1")
+    check_back(cols.cpu().numpy(), oracle.back(g, ones_s), oracle.back(g, ones_s, power=0), _local_len(P, g), "A^T 1")
+
+
+def test_back_power_rejects_other_powers():
+    import torch
+    from ray_forward_back_b200 import ctp
+    g = small_geometries()["parallel"]
+    P = projector(g)
+    with pytest.raises(ctp.CtpError) as ei:
+        P.back_power(torch.zeros(g.sino_shape, device="cuda"), 3)
+    assert ei.value.status == ctp.CTP_ERR_INVALID_ARGUMENT
