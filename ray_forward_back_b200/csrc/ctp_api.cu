@@ -324,7 +324,7 @@ void plan_back(ctp_geom *g, const ctp_plan *plan, int sm_count) {
   int b[3];
   // measured on B200: flat, wide bricks amortise the per-ray FP64 entry best
   if (g->beam == CTP_BEAM_PARALLEL) {
-    b[0] = 128, b[1] = 64, b[2] = 2;
+    b[0] = 128, b[1] = 128, b[2] = 1;
   } else {
     b[0] = 64, b[1] = 64, b[2] = 4;
   }

@@ -507,6 +507,14 @@ __device__ __forceinline__ float coef(float len) {
   return kPower == 2 ? len * len : len;
 }
 
+// Column of the t-th ray of a footprint row of width w taken from both ends
+// inwards (0, w-1, 1, w-2, ...).  With parallel rays a brick's chord profile
+// along a footprint row is a trapezoid symmetric about the row centre, so 32
+// consecutive rays in this order sit at two mirrored distances from the
+// centre and have nearly equal chords: the lanes of a warp finish their
+// walks together.  (Cone footprints are not symmetric; they keep plain order.)
+__device__ __forceinline__ int mirror_order(int t, int w) { return (t & 1) ? w - 1 - (t >> 1) : (t >> 1); }
+
 // Detector footprint of the brick [lo, hi) in view V: a rectangle of pixels
 // that contains every pixel whose ray can meet the brick.  Also returns
 // nvox, an upper bound on the number of this view's rays that can meet any
@@ -752,8 +760,9 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
     __syncthreads();
     const float S = s_scale;
     // pass 2: walk every ray of the stage through the brick.  Each warp takes
-    // 32 consecutive footprint rays (neighbouring columns, similar chords),
-    // sets them up together and reconverges before the next 32.
+    // 32 consecutive footprint rays (parallel beams: in mirror order, rays
+    // with similar chords through the brick), sets them up together and
+    // reconverges before the next 32.
     if (S > 0.f) {
       for (int q0 = warp * 32; q0 < total; q0 += kBackThreads) {
         const int q = q0 + lane;
@@ -771,7 +780,7 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
           const int w = fw[sl];
           const int rr = qq / w;
           r = fr0[sl] + rr;
-          c = fc0[sl] + (qq - rr * w);
+          c = fc0[sl] + (P.dims.beam == CTP_BEAM_PARALLEL ? mirror_order(qq - rr * w, w) : qq - rr * w);
           v = vb + sl;
           y = __ldg(sino + ((size_t)v * nr + r) * nc + c);
           act = y != 0.f;
