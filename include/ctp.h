@@ -52,6 +52,7 @@
 #ifndef CTP_H
 #define CTP_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -210,6 +211,48 @@ ctp_status ctp_count_updates(const ctp_geom *geom, int64_t *host_out, void *stre
  */
 #define CTP_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 ctp_status ctp_forward_noalloc(const ctp_geom_desc *desc, const float *vol, float *sino, void *stream);
+
+/* Iterative solvers (diffct "Execution", section "Numerical solver API"). */
+enum { CTP_SOLVER_CGLS = 1, CTP_SOLVER_SIRT = 2 };
+
+typedef struct {
+  int32_t method;       /* CTP_SOLVER_CGLS | CTP_SOLVER_SIRT */
+  int32_t iterations;   /* run at most this many iterations */
+  double atol, rtol;    /* stop when ||y - A x|| <= atol + rtol ||y||, the initial iterate included */
+  double relaxation;    /* SIRT step factor lambda (1 = plain SIRT); ignored by CGLS */
+  int32_t nonnegative;  /* SIRT: clamp x >= 0 after every step; ignored by CGLS */
+  int32_t use_x0;       /* 1: vol holds the initial iterate; 0: start from zero */
+} ctp_solver_options;
+
+typedef struct {
+  int32_t iterations;   /* completed iterations (history holds iterations + 1 entries) */
+  int32_t converged;    /* 1 if the tolerance was met (possibly by the initial iterate) */
+} ctp_solver_result;
+
+/* Device workspace ctp_solve needs for this geometry and method, in bytes
+ * (0 for a NULL geometry or an unknown method). */
+size_t ctp_solver_workspace_bytes(const ctp_geom *geom, int32_t method);
+
+/*
+ * ctp_solve — least-squares reconstruction of vol from sino with the matched
+ * pair, following diffct "Execution", section "Numerical solver API":
+ *   CGLS: conjugate gradients on the normal equations (least-squares form);
+ *   SIRT: x <- x + lambda C A^T R (y - A x), R and C the reciprocal row and
+ *         column sums of A (0 where a sum is 0), optionally clamped at 0; the
+ *         residual of each history entry is reused for the next update.
+ * history (HOST, at least iterations + 1 doubles) receives ||y - A x|| of the
+ * initial iterate and of every completed iteration; *result the count and
+ * whether the tolerance was met.  workspace: DEVICE memory of at least
+ * ctp_solver_workspace_bytes(geom, method), 256-byte aligned, owned by the
+ * caller and overwritten.  sino, vol: device pointers as for ctp_forward;
+ * vol is overwritten with the final iterate.
+ * Synchronous: every iteration reads one block of norms back to the host
+ * (the residual norm, and for CGLS the two norms of its step), so the call
+ * returns when the solve is finished.
+ */
+ctp_status ctp_solve(const ctp_geom *geom, const float *sino, float *vol, const ctp_solver_options *opts,
+                     void *workspace, size_t workspace_bytes, double *history, ctp_solver_result *result,
+                     void *stream);
 
 /* Static description of a status code. */
 const char *ctp_status_string(ctp_status status);

@@ -35,8 +35,10 @@ CTP_ADJOINT_BRICK = 1
 CTP_ADJOINT_SORT = 2
 
 EXPORTED = ["ctp_geom_create", "ctp_geom_destroy", "ctp_geom_query", "ctp_forward", "ctp_back",
-            "ctp_back_power", "ctp_count_updates", "ctp_forward_noalloc", "ctp_status_string", "ctp_last_error_detail",
-            "ctp_version"]
+            "ctp_back_power", "ctp_count_updates", "ctp_forward_noalloc", "ctp_solve", "ctp_solver_workspace_bytes",
+            "ctp_status_string", "ctp_last_error_detail", "ctp_version"]
+CTP_SOLVER_CGLS = 1
+CTP_SOLVER_SIRT = 2
 
 
 class ctp_plan(ctypes.Structure):
@@ -61,6 +63,16 @@ class ctp_geom_info(ctypes.Structure):
                 ("adjoint_variant", ctypes.c_int32), ("brick", ctypes.c_int32 * 3),
                 ("view_groups", ctypes.c_int32), ("n_transposed_views", ctypes.c_int32),
                 ("collision_ratio", ctypes.c_double)]
+
+
+class ctp_solver_options(ctypes.Structure):
+    _fields_ = [("method", ctypes.c_int32), ("iterations", ctypes.c_int32), ("atol", ctypes.c_double),
+                ("rtol", ctypes.c_double), ("relaxation", ctypes.c_double), ("nonnegative", ctypes.c_int32),
+                ("use_x0", ctypes.c_int32)]
+
+
+class ctp_solver_result(ctypes.Structure):
+    _fields_ = [("iterations", ctypes.c_int32), ("converged", ctypes.c_int32)]
 
 
 class CtpError(RuntimeError):
@@ -100,6 +112,11 @@ def load(path: str = None):
         lib.ctp_count_updates.restype = ctypes.c_int
         lib.ctp_forward_noalloc.argtypes = [ctypes.POINTER(ctp_geom_desc), vp, vp, vp]
         lib.ctp_forward_noalloc.restype = ctypes.c_int
+        lib.ctp_solver_workspace_bytes.argtypes = [vp, ctypes.c_int32]
+        lib.ctp_solver_workspace_bytes.restype = ctypes.c_size_t
+        lib.ctp_solve.argtypes = [vp, vp, vp, ctypes.POINTER(ctp_solver_options), vp, ctypes.c_size_t,
+                                  ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctp_solver_result), vp]
+        lib.ctp_solve.restype = ctypes.c_int
         lib.ctp_status_string.argtypes = [ctypes.c_int]
         lib.ctp_status_string.restype = ctypes.c_char_p
         lib.ctp_last_error_detail.argtypes = []
@@ -220,6 +237,31 @@ def ctp_forward_noalloc(geom, vol, sino, device: int = 0, plan: Optional[dict] =
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
+def ctp_solver_workspace_bytes(handle: int, method: int) -> int:
+    return int(load().ctp_solver_workspace_bytes(handle, int(method)))
+
+
+def ctp_solve(handle: int, sino, vol, method: int, iterations: int, atol=0.0, rtol=0.0, relaxation=1.0,
+              nonnegative=True, use_x0=False, workspace=None, stream=None):
+    """Run CGLS or SIRT; returns (history list, converged).  ``workspace`` is
+    a device buffer of at least ctp_solver_workspace_bytes bytes (allocated
+    here from torch when omitted)."""
+    import torch
+    need = ctp_solver_workspace_bytes(handle, method)
+    if workspace is None:
+        workspace = torch.empty(need + 256, dtype=torch.uint8, device=sino.device)
+    base = _ptr(workspace)
+    base_aligned = (base + 255) & ~255
+    size = int(workspace.numel() * workspace.element_size()) - (base_aligned - base)
+    opts = ctp_solver_options(int(method), int(iterations), float(atol), float(rtol), float(relaxation),
+                              1 if nonnegative else 0, 1 if use_x0 else 0)
+    hist = (ctypes.c_double * (int(iterations) + 1))()
+    res = ctp_solver_result()
+    _check(load().ctp_solve(handle, _ptr(sino), _ptr(vol), ctypes.byref(opts), base_aligned, size, hist,
+                            ctypes.byref(res), _stream_handle(stream)))
+    return [hist[i] for i in range(res.iterations + 1)], bool(res.converged)
+
+
 def ctp_version() -> str:
     return load().ctp_version().decode()
 
@@ -292,6 +334,19 @@ class Projector:
         self._check_tensor(out, self.geom.vol_shape, "out")
         ctp_back_power(self.handle, sino, out, power, stream)
         return out
+
+    def solve(self, sino, method="cgls", iterations=10, atol=0.0, rtol=0.0, relaxation=1.0, nonnegative=True,
+              x0=None, stream=None):
+        """CGLS or SIRT reconstruction; returns (volume, residual history, converged)."""
+        import torch
+        self._check_tensor(sino, self.geom.sino_shape, "sino")
+        m = {"cgls": CTP_SOLVER_CGLS, "sirt": CTP_SOLVER_SIRT}[method]
+        vol = torch.empty(self.geom.vol_shape, dtype=torch.float32, device=sino.device)
+        if x0 is not None:
+            vol.copy_(x0)
+        hist, conv = ctp_solve(self.handle, sino, vol, m, iterations, atol, rtol, relaxation, nonnegative,
+                               x0 is not None, stream=stream)
+        return vol, hist, conv
 
     def count_updates(self, stream=None) -> int:
         return ctp_count_updates(self.handle, stream)
