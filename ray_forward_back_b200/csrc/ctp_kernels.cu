@@ -318,7 +318,9 @@ __device__ __forceinline__ void walk(bool active, const Walk& W, const int lo[3]
   const float i0 = W.inc[0], i1 = W.inc[1], i2 = W.inc[2];
   int a, b, c;
   walk_axes(W, a, b, c);
-  const int Na = active ? pick3(a, W.N[0], W.N[1], W.N[2]) : -1;
+  // Rayless lanes get Na = 0 and, below, an unreachable slab window, so the
+  // window test is one unsigned compare.
+  const int Na = active ? pick3(a, W.N[0], W.N[1], W.N[2]) : 0;
   const int Nb = pick3(b, W.N[0], W.N[1], W.N[2]);
   const int Nc = pick3(c, W.N[0], W.N[1], W.N[2]);
   const float l0a = pick3(a, W.l0[0], W.l0[1], W.l0[2]), inca = pick3(a, i0, i1, i2);
@@ -330,7 +332,7 @@ __device__ __forceinline__ void walk(bool active, const Walk& W, const int lo[3]
   const int ia = pick3(a, W.i[0], W.i[1], W.i[2]);
   const int p = pick3(a, W.step[0], W.step[1], W.step[2]) > 0 ? ia - pick3(a, lo[0], lo[1], lo[2])
                                                                : pick3(a, hi[0], hi[1], hi[2]) - 1 - ia;
-  const int span_plain = __reduce_max_sync(kFull, Na);
+  const int span_plain = __reduce_max_sync(kFull, active ? Na : -1);
   if (span_plain < 0) return;  // no lane has a ray
   int d = 0, kmax = span_plain;
   if (kAlign) {
@@ -341,6 +343,7 @@ __device__ __forceinline__ void walk(bool active, const Walk& W, const int lo[3]
     if (span_aligned <= 2 * span_plain + 8) kmax = span_aligned;
     else d = 0;
   }
+  if (!active) d = 1 << 30;  // s = k - d stays negative: never inside [0, Na]
 
   const float L = W.L;
   const float fNb = (float)Nb, fNc = (float)Nc;
@@ -352,8 +355,10 @@ __device__ __forceinline__ void walk(bool active, const Walk& W, const int lo[3]
 #pragma unroll kWalk2Unroll
     for (int k = 0; k <= kmax; ++k) {
       const int s = k - d;
-      const bool on = s >= 0 && s <= Na;
-      const float tx = s < Na ? fminf(fmaf((float)s, inca, l0a), L) : L;
+      const bool on = (unsigned)s <= (unsigned)Na;
+      // the (Na+1)-th major crossing lies at or past the exit: clamping to L
+      // ends the last slab there (to within rounding of the walk length)
+      const float tx = fminf(fmaf((float)s, inca, l0a), L);
       const bool cb = on && tb < tx;
       const float m1 = fmaxf(fminf(tb, tx), cur);
       if (kUniform) {
@@ -379,8 +384,8 @@ __device__ __forceinline__ void walk(bool active, const Walk& W, const int lo[3]
 #pragma unroll kWalk3Unroll
     for (int k = 0; k <= kmax; ++k) {
       const int s = k - d;
-      const bool on = s >= 0 && s <= Na;
-      const float tx = s < Na ? fminf(fmaf((float)s, inca, l0a), L) : L;
+      const bool on = (unsigned)s <= (unsigned)Na;
+      const float tx = fminf(fmaf((float)s, inca, l0a), L);
       const bool cb = on && tb < tx, cc = on && tc < tx;
       const float m1 = fmaxf(fminf(fminf(tb, tc), tx), cur);
       const float m2 = fmaxf(fminf(fmaxf(tb, tc), tx), m1);
