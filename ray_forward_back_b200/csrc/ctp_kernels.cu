@@ -290,6 +290,79 @@ __device__ __forceinline__ void walk_lane(const Walk& W, Off off, Off s0, Off s1
   }
 }
 
+// Branch-free FP32 Siddon walk in major-axis slabs with a warp-uniform trip
+// count: every lane steps slab s = 0, 1, ... up to the warp's longest walk
+// and lanes past their own last slab are predicated off, so the loop needs
+// no reconvergence and unrolls cleanly.  Every slab makes the same visit
+// calls (a segment absent from that slab is visited with length 0 at a valid
+// offset).  The last slab of a ray ends at its exit: the (Na+1)-th major
+// crossing lies at or past it, so clamping to L closes the walk (to within
+// rounding of the walk length).  All 32 lanes must call this; lanes without
+// a ray pass active = false.  Offsets as in walk_lane.
+template <typename Off, typename Visit>
+__device__ __forceinline__ void walk_warp_bf(bool active, const Walk& W, Off off, Off s0, Off s1, Off s2,
+                                             Visit&& visit) {
+  constexpr unsigned kFull = 0xffffffffu;
+  int a, b, c;
+  walk_axes(W, a, b, c);
+  const int Na = active ? pick3(a, W.N[0], W.N[1], W.N[2]) : -1;
+  const int Nb = pick3(b, W.N[0], W.N[1], W.N[2]);
+  const int Nc = pick3(c, W.N[0], W.N[1], W.N[2]);
+  const float l0a = pick3(a, W.l0[0], W.l0[1], W.l0[2]), inca = pick3(a, W.inc[0], W.inc[1], W.inc[2]);
+  const float l0b = pick3(b, W.l0[0], W.l0[1], W.l0[2]), incb = pick3(b, W.inc[0], W.inc[1], W.inc[2]);
+  const float l0c = pick3(c, W.l0[0], W.l0[1], W.l0[2]), incc = pick3(c, W.inc[0], W.inc[1], W.inc[2]);
+  const Off sa = pick3(a, s0, s1, s2), sb = pick3(b, s0, s1, s2), sc = pick3(c, s0, s1, s2);
+  const float L = W.L;
+  const float fNb = (float)Nb, fNc = (float)Nc;
+  const int kmax = __reduce_max_sync(kFull, Na);
+  if (kmax < 0) return;
+  float tb = Nb > 0 ? l0b : CUDART_INF_F;
+  float fjb = 1.f, cur = 0.f;
+  if (!__any_sync(kFull, active && Nc > 0)) {
+#pragma unroll kLaneWalk2Unroll
+    for (int s = 0; s <= kmax; ++s) {
+      const bool on = s <= Na;
+      const float tx = fminf(fmaf((float)s, inca, l0a), L);
+      const bool cb = tb < tx;
+      const float m1 = fmaxf(fminf(tb, tx), cur);
+      const Off o2 = off + (cb ? sb : (Off)0);
+      if (on) {
+        visit(off, m1 - cur);
+        visit(o2, tx - m1);
+        off = o2 + sa;
+        tb = cb ? (fjb < fNb ? fmaf(fjb, incb, l0b) : CUDART_INF_F) : tb;
+        fjb += cb ? 1.f : 0.f;
+        cur = tx;
+      }
+    }
+  } else {
+    float tc = Nc > 0 ? l0c : CUDART_INF_F;
+    float fjc = 1.f;
+#pragma unroll kWalk3Unroll
+    for (int s = 0; s <= kmax; ++s) {
+      const bool on = s <= Na;
+      const float tx = fminf(fmaf((float)s, inca, l0a), L);
+      const bool cb = tb < tx, cc = tc < tx;
+      const float m1 = fmaxf(fminf(fminf(tb, tc), tx), cur);
+      const float m2 = fmaxf(fminf(fmaxf(tb, tc), tx), m1);
+      const Off db = cb ? sb : (Off)0, dc = cc ? sc : (Off)0;
+      const Off o2 = off + (tb <= tc ? db : dc);
+      const Off o3 = off + db + dc;
+      if (on) {
+        visit(off, m1 - cur);
+        visit(o2, m2 - m1);
+        visit(o3, tx - m2);
+        off = o3 + sa;
+        tb = cb ? (fjb < fNb ? fmaf(fjb, incb, l0b) : CUDART_INF_F) : tb;
+        fjb += cb ? 1.f : 0.f;
+        tc = cc ? (fjc < fNc ? fmaf(fjc, incc, l0c) : CUDART_INF_F) : tc;
+        fjc += cc ? 1.f : 0.f;
+        cur = tx;
+      }
+    }
+  }
+}
+
 // FP32 Siddon walk in major-axis slabs, warp-synchronous.
 //
 // The major axis a is the one the ray crosses most often (smallest spacing
@@ -803,10 +876,16 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
           off = ((W.i[2] - lo[2]) * P.brick[1] + (W.i[1] - lo[1])) * pitch + (W.i[0] - lo[0]);
         }
         const float yS = y * S;
-        if (act)
-          walk_lane<int>(W, off, W.step[0], W.step[1] * pitch, W.step[2] * plane,
-                         [&](int o, float len) { atomicAdd(acc + o, __float2int_rn(coef<kPower>(len) * yS)); });
-        __syncwarp();
+        auto visit = [&](int o, float len) { atomicAdd(acc + o, __float2int_rn(coef<kPower>(len) * yS)); };
+        // measured on B200: parallel rays (mirror-ordered, near-equal chords)
+        // walk fastest with independent lane loops, cone rays with the
+        // warp-uniform trip count
+        if (P.dims.beam == CTP_BEAM_PARALLEL) {
+          if (act) walk_lane<int>(W, off, W.step[0], W.step[1] * pitch, W.step[2] * plane, visit);
+          __syncwarp();
+        } else {
+          walk_warp_bf<int>(act, W, off, W.step[0], W.step[1] * pitch, W.step[2] * plane, visit);
+        }
       }
     }
     __syncthreads();
