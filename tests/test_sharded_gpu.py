@@ -1,0 +1,45 @@
+"""The view-sharded projector on the GPU path: the CUDA library per rank and
+NCCL for the reductions.  Only one GPU is available to a test, so the group
+has one rank; the multi-rank logic is covered by the gloo tests."""
+import os
+import socket
+
+import numpy as np
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+
+def _port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def test_single_rank_nccl_sharded_equals_projector():
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from ray_forward_back_b200 import workloads as W
+    from ray_forward_back_b200.sharded import ShardedProjector
+    from tests.gpu_helpers import projector
+    g = W.make_cone(40, 36, 24, 9, 20, 30, sid=80.0, sdd=140.0, pitch_u=1.5, pitch_v=1.5, start=0.3)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(_port())
+    dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=60), device_id=dev)
+    try:
+        S = ShardedProjector(g, device=dev.index)
+        P = projector(g)
+        vol = torch.rand(g.vol_shape, device=dev)
+        sino = torch.rand(g.sino_shape, device=dev)
+        assert torch.equal(S.forward(vol), P.forward(vol))
+        x_ref = P.back(sino)
+        assert torch.equal(S.back(sino), x_ref)
+        z0, z1, slab = S.back_slab(sino)
+        assert (z0, z1) == (0, g.nz) and torch.equal(slab, x_ref)
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
