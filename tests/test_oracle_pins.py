@@ -338,3 +338,35 @@ def test_view_ranges_compose():
     np.testing.assert_array_equal(np.concatenate([oracle.forward(g, x, (0, 3)), oracle.forward(g, x, (3, 7))]), full)
     np.testing.assert_allclose(oracle.back(g, y[:3], (0, 3)) + oracle.back(g, y[3:], (3, 7)), oracle.back(g, y),
                                atol=1e-12)
+
+
+# ------------------------------------------- geometry gradient reference ---
+
+def test_fd_geometry_gradient_matches_rectangle_chord_slope():
+    """Uniform W x H box, one in-plane parallel ray at offset q: the chord is
+    a trapezoid in q; shifting det_c along the detector's column direction by
+    e moves the ray by e, so dy/d(det_c . u_hat) is the trapezoid's slope,
+    computed from the rectangle's edge lines (closed form), and shifting
+    det_c along the ray direction changes nothing."""
+    from oracle.geometry_grad import geometry_gradient_fd
+    theta = 0.41
+    g = _box_geom(theta)
+    vol = np.ones(g.vol_shape, np.float32)
+    Wd, Hd = g.nx * g.spacing[0], g.ny * g.spacing[1]
+    d = np.array([math.cos(theta), math.sin(theta)])
+    n = np.array([-math.sin(theta), math.cos(theta)])
+
+    def chord(q):
+        p = q * n
+        ts = sorted([(-Wd / 2 - p[0]) / d[0], (Wd / 2 - p[0]) / d[0]])
+        us = sorted([(-Hd / 2 - p[1]) / d[1], (Hd / 2 - p[1]) / d[1]])
+        return max(0.0, min(ts[1], us[1]) - max(ts[0], us[0]))
+
+    for c in (0, 2, 6, 8):   # rays on the sloped part of the trapezoid
+        q = (c - (g.n_cols - 1) / 2) * 0.77
+        slope = (chord(q + 1e-4) - chord(q - 1e-4)) / 2e-4
+        up = np.zeros(g.sino_shape)
+        up[0, 1, c] = 1.0
+        grad = geometry_gradient_fd(g, vol, up)
+        assert grad[0, 1] @ np.array([n[0], n[1], 0.0]) == pytest.approx(slope, rel=1e-6, abs=1e-7)
+        assert grad[0, 1] @ np.array([d[0], d[1], 0.0]) == pytest.approx(0.0, abs=1e-6)
