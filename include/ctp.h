@@ -174,6 +174,29 @@ ctp_status ctp_back(const ctp_geom *geom, const float *sino, float *vol, void *s
 ctp_status ctp_back_power(const ctp_geom *geom, const float *sino, float *vol, int power, void *stream);
 
 /*
+ * ctp_geometry_gradient — gradients of a scalar loss with respect to the
+ * acquisition geometry, given the loss's gradient on the sinogram:
+ *   grad[v][f][k] = sum over the rays (r, c) of view v of
+ *                   sino_grad[v][r][c] * d(A vol)[v][r][c] / d(vector f)_k,
+ * f = 0 src, 1 det_c, 2 det_u, 3 det_v (the vectors of ctp_geom_desc; for
+ * a parallel beam src is the ray direction, whose length does not matter).
+ * diffct "Execution", section "Streaming analytical reconstruction": geometry
+ * gradients of the projection at the cost of one extra traversal.  The line
+ * integral is piecewise linear in the geometry; where a ray passes through a
+ * voxel edge or an endpoint lies on a voxel face it has a kink and the result
+ * is one of the one-sided derivatives.
+ * vol:       device pointer, float32 [nz][ny][nx] (the forward's input), read only.
+ * sino_grad: device pointer, float32 [n_views][n_rows][n_cols], read only.
+ * grad:      device pointer, float64 [n_views][4][3], overwritten (zeroed,
+ *            then accumulated; contents are undefined if the call fails).
+ * Flat detectors only: a cylindrical detector gives CTP_ERR_UNSUPPORTED.
+ * Asynchronous on `stream`; summation order across blocks is not fixed, so
+ * results can differ between calls in the last bits.
+ */
+ctp_status ctp_geometry_gradient(const ctp_geom *geom, const float *vol, const float *sino_grad, double *grad,
+                                 void *stream);
+
+/*
  * ctp_count_updates — the number of positive-length ray-voxel segments of the
  * whole acquisition (the work measure of both projectors), computed on the
  * device.  Synchronous: waits for the count and writes it to *host_out.

@@ -179,6 +179,7 @@ ctp_status build_view(const ctp_geom_desc *d, int64_t v, ViewRec &V, double *tri
   V.vlen = nvl;
   for (int k = 0; k < 3; ++k) V.vhat[k] = dv[k] / nvl;
   for (int k = 0; k < 3; ++k) V.dv[k] = dv[k];
+  V.src_norm = norm(s);
   if (d->beam == CTP_BEAM_PARALLEL) {
     const double ns = norm(s);
     if (!(ns > 0.0)) return fail(CTP_ERR_DEGENERATE_RAY, "view %lld: zero ray direction", (long long)v);
@@ -644,6 +645,27 @@ ctp_status ctp_back_power(const ctp_geom *g, const float *sino, float *vol, int 
   else
     e = ctp::launch_back_brick(g->back, g->d_views, g->d_trig, sino, vol, power, g->wide_index, s);
   if (e != cudaSuccess) return cuda_fail(e, "adjoint launch");
+  return CTP_OK;
+}
+
+ctp_status ctp_geometry_gradient(const ctp_geom *g, const float *vol, const float *sino_grad, double *grad,
+                                 void *stream) {
+  g_detail[0] = '\0';
+  if (!g) return fail(CTP_ERR_INVALID_ARGUMENT, "geometry is NULL");
+  if (g->det != CTP_DET_FLAT)
+    return fail(CTP_ERR_UNSUPPORTED, "geometry gradients are available for flat detectors only");
+  DeviceGuard dg(g->device);
+  if (dg.err != cudaSuccess) return cuda_fail(dg.err, "cudaSetDevice");
+  if (!is_device_pointer(vol, g->device) || !is_device_pointer(sino_grad, g->device) ||
+      !is_device_pointer(grad, g->device))
+    return fail(CTP_ERR_INVALID_ARGUMENT, "vol, sino_grad and grad must be device memory of device %d", g->device);
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "pending error before ctp_geometry_gradient");
+  e = cudaMemsetAsync(grad, 0, sizeof(double) * 12 * (size_t)g->n_views, s);
+  if (e == cudaSuccess)
+    e = ctp::launch_geometry_gradient(g->fwd, g->d_views, g->d_trig, vol, sino_grad, grad, g->wide_index, s);
+  if (e != cudaSuccess) return cuda_fail(e, "geometry gradient launch");
   return CTP_OK;
 }
 

@@ -30,6 +30,7 @@ struct ViewRec {
   double vox_ext[3];  // one voxel's projected extent: parallel (columns, rows, -);
                       // cone flat: sum_k |minv row i, k| * spacing_k for rows i = 0, 1, 2
   double R, gam0, dgam, axial0, vlen;
+  double src_norm;    // |src| as given (parallel beam: the direction's length)
   int32_t layout;     // forward gather: 0 = x-fastest volume, 1 = y-fastest copy
   int32_t full_footprint;  // 1: the footprint test cannot bound this view; scan all pixels
 };
@@ -80,6 +81,8 @@ cudaError_t launch_back_sort(const FwdLaunch& p, const ViewRec* views, const dou
 cudaError_t launch_collision_count(const FwdLaunch& p, const ViewRec* views, const double* trig,
                                    unsigned long long* counters, bool wide_index, cudaStream_t stream);
 size_t back_brick_smem_bytes(const int32_t brick[3]);
+cudaError_t launch_geometry_gradient(const FwdLaunch& p, const ViewRec* views, const double* trig, const float* vol,
+                                     const float* gsino, double* grad, bool wide_index, cudaStream_t stream);
 
 // Host helpers (ctp_api.cu).
 ctp_status host_validate(const ctp_geom_desc* d);

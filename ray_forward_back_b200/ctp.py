@@ -35,7 +35,7 @@ CTP_ADJOINT_BRICK = 1
 CTP_ADJOINT_SORT = 2
 
 EXPORTED = ["ctp_geom_create", "ctp_geom_destroy", "ctp_geom_query", "ctp_forward", "ctp_back",
-            "ctp_back_power", "ctp_count_updates", "ctp_forward_noalloc", "ctp_solve", "ctp_solver_workspace_bytes",
+            "ctp_back_power", "ctp_geometry_gradient", "ctp_count_updates", "ctp_forward_noalloc", "ctp_solve", "ctp_solver_workspace_bytes",
             "ctp_status_string", "ctp_last_error_detail", "ctp_version"]
 CTP_SOLVER_CGLS = 1
 CTP_SOLVER_SIRT = 2
@@ -108,6 +108,8 @@ def load(path: str = None):
         lib.ctp_back.restype = ctypes.c_int
         lib.ctp_back_power.argtypes = [vp, vp, vp, ctypes.c_int, vp]
         lib.ctp_back_power.restype = ctypes.c_int
+        lib.ctp_geometry_gradient.argtypes = [vp, vp, vp, vp, vp]
+        lib.ctp_geometry_gradient.restype = ctypes.c_int
         lib.ctp_count_updates.argtypes = [vp, ctypes.POINTER(i64), vp]
         lib.ctp_count_updates.restype = ctypes.c_int
         lib.ctp_forward_noalloc.argtypes = [ctypes.POINTER(ctp_geom_desc), vp, vp, vp]
@@ -218,6 +220,10 @@ def ctp_back(handle: int, sino, vol, stream=None) -> None:
 
 def ctp_back_power(handle: int, sino, vol, power: int, stream=None) -> None:
     _check(load().ctp_back_power(handle, _ptr(sino), _ptr(vol), int(power), _stream_handle(stream)))
+
+
+def ctp_geometry_gradient(handle: int, vol, sino_grad, grad, stream=None) -> None:
+    _check(load().ctp_geometry_gradient(handle, _ptr(vol), _ptr(sino_grad), _ptr(grad), _stream_handle(stream)))
 
 
 def ctp_count_updates(handle: int, stream=None) -> int:
@@ -333,6 +339,20 @@ class Projector:
             out = torch.empty(self.geom.vol_shape, dtype=torch.float32, device=sino.device)
         self._check_tensor(out, self.geom.vol_shape, "out")
         ctp_back_power(self.handle, sino, out, power, stream)
+        return out
+
+    def geometry_gradient(self, vol, sino_grad, out=None, stream=None):
+        """d(loss)/d(src, det_c, det_u, det_v) per view, float64 [n_views, 4, 3],
+        given the volume and the loss's gradient on the sinogram."""
+        import torch
+        self._check_tensor(vol, self.geom.vol_shape, "vol")
+        self._check_tensor(sino_grad, self.geom.sino_shape, "sino_grad")
+        shape = (self.geom.n_views, 4, 3)
+        if out is None:
+            out = torch.empty(shape, dtype=torch.float64, device=vol.device)
+        if out.dtype != torch.float64 or not out.is_cuda or tuple(out.shape) != shape or not out.is_contiguous():
+            raise ValueError(f"out must be a contiguous float64 CUDA tensor of shape {shape}")
+        ctp_geometry_gradient(self.handle, vol, sino_grad, out, stream)
         return out
 
     def solve(self, sino, method="cgls", iterations=10, atol=0.0, rtol=0.0, relaxation=1.0, nonnegative=True,

@@ -1,0 +1,111 @@
+"""Geometry gradients on the GPU (ctp_geometry_gradient) against central
+finite differences of the FP64 oracle's forward projection.
+
+The line integral is piecewise linear in the geometry, so away from kinks
+the finite difference is exact up to rounding; the seeded geometries are
+perturbed off the voxel lattice so that no ray sits within the step of a
+kink.  The GPU walks in FP32 (crossing distances to a few ulp of the ray
+length) and sums in FP64, so the bound is relative to the largest entry."""
+import numpy as np
+import pytest
+
+from oracle.geometry_grad import geometry_gradient_fd
+from ray_forward_back_b200 import ctp
+from ray_forward_back_b200 import workloads as W
+from tests.gpu_helpers import projector
+
+pytestmark = pytest.mark.gpu
+
+REL = 2e-4
+
+
+def _jitter(g, seed, scale=0.03):
+    """Move every vector off the lattice by a small seeded amount."""
+    rng = np.random.default_rng(seed)
+    for name in ("src", "det_c", "det_u", "det_v"):
+        a = getattr(g, name).copy()
+        ref = np.abs(a).max()
+        setattr(g, name, a + scale * max(ref, 1.0) * 0.01 * rng.standard_normal(a.shape))
+    return g
+
+
+def _gpu_grad(g, vol, gs):
+    import torch
+    P = projector(g)
+    out = P.geometry_gradient(torch.from_numpy(vol).cuda(), torch.from_numpy(gs).cuda())
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+def _check(g, seed, vol=None):
+    rng = np.random.default_rng(seed)
+    if vol is None:
+        vol = rng.random(g.vol_shape).astype(np.float32)
+    gs = rng.standard_normal(g.sino_shape).astype(np.float32)
+    ref = geometry_gradient_fd(g, vol, gs.astype(np.float64))
+    got = _gpu_grad(g, vol, gs)
+    assert got.shape == (g.n_views, 4, 3)
+    scale = np.abs(ref).max()
+    assert scale > 0
+    err = np.abs(got - ref).max()
+    assert err <= REL * scale, (err, scale)
+    return ref, got
+
+
+CASES = {
+    # cone, source and detector outside the volume; ragged detector tiles
+    "cone_outside": lambda: _jitter(W.make_cone(10, 9, 7, 4, 6, 37, sid=30.0, sdd=55.0, pitch_u=1.3,
+                                                pitch_v=1.4, start=0.2), 1),
+    # detector plane through the volume: pixels inside, the t = 1 endpoint term
+    "cone_pixels_inside": lambda: _jitter(W.make_cone(10, 9, 7, 3, 9, 11, sid=20.0, sdd=21.5, pitch_u=1.1,
+                                                      pitch_v=0.9, start=0.4), 2),
+    # source inside the volume: the source is the parameter origin
+    "cone_source_inside": lambda: _jitter(W.make_cone(10, 9, 7, 3, 7, 9, sid=2.5, sdd=30.0, pitch_u=2.1,
+                                                      pitch_v=1.7, start=0.7), 3),
+    # helical source path, anisotropic voxels and a shifted volume
+    "helical_flat": lambda: _jitter(W.make_cone(8, 10, 6, 5, 5, 9, sid=25.0, sdd=45.0, pitch_u=1.6, pitch_v=1.5,
+                                                spacing=(1.1, 0.9, 1.3), z_start=-3.0, z_end=2.0, start=0.1,
+                                                origin=(-4.7, -4.1, -3.3)), 4),
+    "parallel": lambda: _jitter(W.make_parallel(9, 8, 7, 5, 6, 35, pitch_u=0.8, pitch_v=0.9, start=0.13), 5),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_geometry_gradient_matches_finite_differences(name):
+    g = CASES[name]()
+    if name == "parallel":
+        src = g.src.copy()
+        src[:, 2] += 0.3     # rays oblique to the z planes
+        src *= 1.7           # a direction that is not unit length
+        g.src = src
+    ref, got = _check(g, 10)
+    if name == "parallel":
+        # the length of the direction does not matter: no gradient along it
+        for v in range(g.n_views):
+            assert abs(got[v, 0] @ g.src[v]) <= 1e-5 * np.abs(got[v, 0]).max() * np.linalg.norm(g.src[v])
+
+
+def test_geometry_gradient_on_workload1_phantom():
+    """Cone 64^3 phantom of the 16-view workload, two views off the lattice,
+    128x128 detector: a piecewise-constant object with many edges."""
+    wl = W.workload(1)
+    g = _jitter(wl.geom.subset_views([3, 11]), 6)
+    _check(g, 11, vol=wl.phantom())
+
+
+def test_zero_inputs_give_zero_and_cylindrical_is_unsupported():
+    import torch
+    g = CASES["cone_outside"]()
+    P = projector(g)
+    vol = torch.rand(g.vol_shape, device="cuda")
+    gs = torch.zeros(g.sino_shape, device="cuda")
+    out = torch.full((g.n_views, 4, 3), 7.0, dtype=torch.float64, device="cuda")
+    P.geometry_gradient(vol, gs, out=out)
+    assert torch.count_nonzero(out).item() == 0
+    P.geometry_gradient(torch.zeros_like(vol), torch.randn_like(gs), out=out)
+    assert torch.count_nonzero(out).item() == 0
+    cyl = W.make_cone(10, 9, 7, 2, 4, 5, sid=30.0, sdd=55.0, pitch_u=0.1, detector=W.DET_CYLINDRICAL)
+    Pc = projector(cyl)
+    with pytest.raises(ctp.CtpError) as ei:
+        Pc.geometry_gradient(torch.zeros(cyl.vol_shape, device="cuda"), torch.zeros(cyl.sino_shape, device="cuda"))
+    assert ei.value.status == ctp.CTP_ERR_UNSUPPORTED
