@@ -37,10 +37,10 @@
 // one of the one-sided values.
 //
 // Kernel: one thread per ray on the forward's grid (a block is 32 columns x 8
-// rows of one view), FP64 setup shared with the projectors, a merged Siddon
-// walk that visits every crossing in order (FP32 crossing distances from
-// exact integers, FP64 sums), then a block reduction and 12 FP64 atomics per
-// block into grad[view][4][3].
+// rows of one view), FP64 setup shared with the projectors, an FP32
+// major-axis slab walk for the per-axis crossing sums, the per-ray gradient
+// in FP64, then a block reduction and 12 FP64 atomics per block into
+// grad[view][4][3].
 #include "ctp_ray.cuh"
 
 namespace ctp {
@@ -79,10 +79,135 @@ __device__ __forceinline__ bool clip_faces(const Ray& R, const int hi[3], double
   return t_out > t_in;
 }
 
-__device__ __forceinline__ void add_axis(int k, double v, double& s0, double& s1, double& s2) {
-  s0 += k == 0 ? v : 0.0;
-  s1 += k == 1 ? v : 0.0;
-  s2 += k == 2 ? v : 0.0;
+// Per-axis crossing sums of one ray in FP32:
+//   S0_k = sum of dx over the crossings of axis k,
+//   Sl_k = sum of dx * (distance of the crossing from the entry),
+// dx = value before - value after, for the crossings strictly inside the
+// clipped segment (the faces at its ends are added by the caller).  Walks
+// major-axis slabs as the forward projector does: a slab between two
+// successive planes of the major axis a holds at most one crossing of each
+// minor axis, so it is two to four neighbouring voxels, read only where the
+// crossing exists.  The warp's lanes are aligned on their entry position
+// along the major axis (slab k of the loop is slab k - d of the lane), so
+// neighbouring rays read the same plane in the same iteration.  Crossing
+// distances are l0 + j * inc from exact integers j and the FP64 counts N
+// bound every index, as in the projectors.  All 32 lanes call this; lanes
+// without a ray pass active = false.  Returns the value of the voxel the
+// segment ends in.
+template <typename Off>
+__device__ __forceinline__ float crossing_sums(bool active, const Walk& W, const int hi[3],
+                                               const float* __restrict__ vol, Off off, Off s0, Off s1, Off s2,
+                                               float x0, float S0[3], float Sl[3]) {
+  constexpr unsigned kFull = 0xffffffffu;
+  int a, b, c;
+  walk_axes(W, a, b, c);
+  const int Na = active ? pick3(a, W.N[0], W.N[1], W.N[2]) : 0;
+  const int Nb = pick3(b, W.N[0], W.N[1], W.N[2]);
+  const int Nc = pick3(c, W.N[0], W.N[1], W.N[2]);
+  const float l0a = pick3(a, W.l0[0], W.l0[1], W.l0[2]), inca = pick3(a, W.inc[0], W.inc[1], W.inc[2]);
+  const float l0b = pick3(b, W.l0[0], W.l0[1], W.l0[2]), incb = pick3(b, W.inc[0], W.inc[1], W.inc[2]);
+  const float l0c = pick3(c, W.l0[0], W.l0[1], W.l0[2]), incc = pick3(c, W.inc[0], W.inc[1], W.inc[2]);
+  const Off sa = pick3(a, s0, s1, s2), sb = pick3(b, s0, s1, s2), sc = pick3(c, s0, s1, s2);
+
+  // slab alignment on the entry position along the major axis (travel direction)
+  const int ia = pick3(a, W.i[0], W.i[1], W.i[2]);
+  const int p = pick3(a, W.step[0], W.step[1], W.step[2]) > 0 ? ia : pick3(a, hi[0], hi[1], hi[2]) - 1 - ia;
+  const int span_plain = __reduce_max_sync(kFull, active ? Na : -1);
+  float S0a = 0.f, S0b = 0.f, S0c = 0.f, Sla = 0.f, Slb = 0.f, Slc = 0.f;
+  float xe = x0;
+  if (span_plain >= 0) {
+    const int pmin = __reduce_min_sync(kFull, active ? p : 0x7fffffff);
+    int d = active ? p - pmin : 0;
+    int kmax = __reduce_max_sync(kFull, active ? d + Na : -1);
+    if (kmax > 2 * span_plain + 8) {  // alignment would stretch the warp's loop too much
+      d = 0;
+      kmax = span_plain;
+    }
+    if (!active) d = 1 << 30;  // s = k - d stays negative: never inside [0, Na]
+    const float L = W.L;
+    const float fNb = (float)Nb, fNc = (float)Nc;
+    float tb = Nb > 0 ? l0b : CUDART_INF_F, tc = Nc > 0 ? l0c : CUDART_INF_F;
+    float fjb = 1.f, fjc = 1.f, cur = 0.f;
+    if (!__any_sync(kFull, active && Nc > 0)) {
+#pragma unroll 4
+      for (int k = 0; k <= kmax; ++k) {
+        const int s = k - d;
+        const bool on = (unsigned)s <= (unsigned)Na;
+        const bool ona = (unsigned)s < (unsigned)Na;  // a major plane ends this slab
+        const float tx = ona ? fminf(fmaf((float)s, inca, l0a), L) : L;
+        const bool cb = on && tb < tx;
+        const float m1 = fmaxf(fminf(tb, tx), cur);
+        const Off o2 = off + (cb ? sb : (Off)0);
+        float x1 = x0;
+        if (cb) x1 = __ldg(vol + o2);
+        float x2 = x1;
+        if (ona) x2 = __ldg(vol + o2 + sa);
+        const float d1 = x0 - x1, d2 = x1 - x2;
+        S0b += d1;
+        Slb = fmaf(d1, m1, Slb);
+        S0a += d2;
+        Sla = fmaf(d2, tx, Sla);
+        if (on) {
+          xe = x1;
+          x0 = x2;
+          off = o2 + sa;
+          cur = tx;
+        }
+        if (cb) {
+          tb = fjb < fNb ? fmaf(fjb, incb, l0b) : CUDART_INF_F;
+          fjb += 1.f;
+        }
+      }
+    } else {
+#pragma unroll 2
+      for (int k = 0; k <= kmax; ++k) {
+        const int s = k - d;
+        const bool on = (unsigned)s <= (unsigned)Na;
+        const bool ona = (unsigned)s < (unsigned)Na;
+        const float tx = ona ? fminf(fmaf((float)s, inca, l0a), L) : L;
+        const bool cb = on && tb < tx, cc = on && tc < tx;
+        const bool bfirst = tb <= tc;
+        const float m1 = fmaxf(fminf(fminf(tb, tc), tx), cur);
+        const float m2 = fmaxf(fminf(fmaxf(tb, tc), tx), m1);
+        const Off db = cb ? sb : (Off)0, dc = cc ? sc : (Off)0;
+        const Off o2 = off + (bfirst ? db : dc);
+        const Off o3 = off + db + dc;
+        float x1 = x0;
+        if (cb || cc) x1 = __ldg(vol + o2);
+        float x2 = x1;
+        if (cb && cc) x2 = __ldg(vol + o3);
+        float x3 = x2;
+        if (ona) x3 = __ldg(vol + o3 + sa);
+        const float d1 = x0 - x1, d2 = x1 - x2, d3 = x2 - x3;
+        S0b += bfirst ? d1 : d2;
+        S0c += bfirst ? d2 : d1;
+        Slb = fmaf(bfirst ? d1 : d2, bfirst ? m1 : m2, Slb);
+        Slc = fmaf(bfirst ? d2 : d1, bfirst ? m2 : m1, Slc);
+        S0a += d3;
+        Sla = fmaf(d3, tx, Sla);
+        if (on) {
+          xe = x2;
+          x0 = x3;
+          off = o3 + sa;
+          cur = tx;
+        }
+        if (cb) {
+          tb = fjb < fNb ? fmaf(fjb, incb, l0b) : CUDART_INF_F;
+          fjb += 1.f;
+        }
+        if (cc) {
+          tc = fjc < fNc ? fmaf(fjc, incc, l0c) : CUDART_INF_F;
+          fjc += 1.f;
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    S0[k] = k == a ? S0a : (k == b ? S0b : S0c);
+    Sl[k] = k == a ? Sla : (k == b ? Slb : Slc);
+  }
+  return xe;
 }
 
 template <typename Off>
@@ -90,6 +215,7 @@ __global__ void __launch_bounds__(kGradThreads) geometry_gradient_kernel(FwdLaun
                                                                          const ViewRec* __restrict__ views,
                                                                          const double* __restrict__ trig,
                                                                          const float* __restrict__ vol,
+                                                                         const float* __restrict__ volT,
                                                                          const float* __restrict__ gsino,
                                                                          double* __restrict__ grad) {
   const int per_band = P.dims.n_views * P.n_col_tiles;
@@ -112,55 +238,31 @@ __global__ void __launch_bounds__(kGradThreads) geometry_gradient_kernel(FwdLaun
   const bool hit = valid && gr != 0.f && clip_faces(R, hi, t_in, t_out, k_in, k_out);
 
   // per-axis sums S0_k and sum of dx * (local distance from the entry)
-  double S0x = 0.0, S0y = 0.0, S0z = 0.0, Slx = 0.0, Sly = 0.0, Slz = 0.0, x_end = 0.0;
-  if (hit) {
-    Walk W;
-    entry(R, t_in, t_out, lo, hi, W);
-    const Off nx = P.vol.n[0], ny = P.vol.n[1];
-    const Off sx = W.step[0], sy = W.step[1] * nx, sz = W.step[2] * nx * ny;
-    Off off = (Off)W.i[2] * nx * ny + (Off)W.i[1] * nx + (Off)W.i[0];
-    float cur = __ldg(vol + off);
-    if (k_in >= 0) add_axis(k_in, -(double)cur, S0x, S0y, S0z);  // enters through a face at local distance 0
-    // merged walk: every crossing in order of distance; an axis takes part
-    // only while it has crossings left, so each axis moves exactly N_k times
-    int jx = 0, jy = 0, jz = 0;
-    float lx = W.l0[0], ly = W.l0[1], lz = W.l0[2];
-    const int total = W.N[0] + W.N[1] + W.N[2];
-    for (int n = 0; n < total; ++n) {
-      const bool ex = jx < W.N[0], ey = jy < W.N[1], ez = jz < W.N[2];
-      const int k = (ex && (!ey || lx <= ly) && (!ez || lx <= lz)) ? 0 : ((ey && (!ez || ly <= lz)) ? 1 : 2);
-      const float l = k == 0 ? lx : (k == 1 ? ly : lz);
-      off += k == 0 ? sx : (k == 1 ? sy : sz);
-      const float nxt = __ldg(vol + off);
-      const double dx = (double)cur - (double)nxt;
-      add_axis(k, dx, S0x, S0y, S0z);
-      add_axis(k, dx * (double)l, Slx, Sly, Slz);
-      cur = nxt;
-      if (k == 0) {
-        ++jx;
-        lx = fmaf((float)jx, W.inc[0], W.l0[0]);
-      } else if (k == 1) {
-        ++jy;
-        ly = fmaf((float)jy, W.inc[1], W.l0[1]);
-      } else {
-        ++jz;
-        lz = fmaf((float)jz, W.inc[2], W.l0[2]);
-      }
-    }
-    if (k_out >= 0) {  // leaves through a face at local distance L
-      const double L = (t_out - t_in) * R.len;
-      add_axis(k_out, (double)cur, S0x, S0y, S0z);
-      add_axis(k_out, (double)cur * L, Slx, Sly, Slz);
-    } else {
-      x_end = (double)cur;
-    }
+  Walk W = {};
+  if (hit) entry(R, t_in, t_out, lo, hi, W);
+  // gather from the x-fastest volume or its y-fastest copy, as the forward does
+  const Off nx = P.vol.n[0], ny = P.vol.n[1];
+  const bool yfast = V.layout != 0;
+  const float* __restrict__ base = yfast ? volT : vol;
+  const Off sx = yfast ? ny : (Off)1, sy = yfast ? (Off)1 : nx, sz = nx * ny;
+  const Off off = (Off)W.i[2] * sz + (Off)W.i[1] * sy + (Off)W.i[0] * sx;
+  const float first = hit ? __ldg(base + off) : 0.f;
+  float f0[3], fl[3];
+  const float last =
+      crossing_sums<Off>(hit, W, hi, base, off, W.step[0] * sx, W.step[1] * sy, W.step[2] * sz, first, f0, fl);
+  double S0[3], Sl[3];
+  // the faces: entering at local distance 0, leaving at the segment's length
+  const double Lseg = (t_out - t_in) * R.len;
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    S0[k] = (double)f0[k] - (k == k_in ? (double)first : 0.0) + (k == k_out ? (double)last : 0.0);
+    Sl[k] = (double)fl[k] + (k == k_out ? (double)last * Lseg : 0.0);
   }
+  const double x_end = k_out < 0 ? (double)last : 0.0;
 
   // per-ray gradients: G_src (3) and G_pix (3), weighted by g
   double gs[3] = {0.0, 0.0, 0.0}, gp[3] = {0.0, 0.0, 0.0};
   if (hit) {
-    const double S0[3] = {S0x, S0y, S0z};
-    const double Sl[3] = {Slx, Sly, Slz};
     const double len = R.len, g = (double)gr;
     double S1[3], Dw[3];
 #pragma unroll
@@ -229,15 +331,16 @@ __global__ void __launch_bounds__(kGradThreads) geometry_gradient_kernel(FwdLaun
 }  // namespace
 
 cudaError_t launch_geometry_gradient(const FwdLaunch& p, const ViewRec* views, const double* trig, const float* vol,
-                                     const float* gsino, double* grad, bool wide_index, cudaStream_t stream) {
+                                     const float* volT, const float* gsino, double* grad, bool wide_index,
+                                     cudaStream_t stream) {
   const long long blocks = (long long)p.n_row_bands * p.dims.n_views * p.n_col_tiles;
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   dim3 block(kGradCols, kGradRows);
   if (wide_index)
-    geometry_gradient_kernel<long long><<<(unsigned)blocks, block, 0, stream>>>(p, views, trig, vol, gsino, grad);
+    geometry_gradient_kernel<long long><<<(unsigned)blocks, block, 0, stream>>>(p, views, trig, vol, volT, gsino, grad);
   else
-    geometry_gradient_kernel<int><<<(unsigned)blocks, block, 0, stream>>>(p, views, trig, vol, gsino, grad);
+    geometry_gradient_kernel<int><<<(unsigned)blocks, block, 0, stream>>>(p, views, trig, vol, volT, gsino, grad);
   return cudaGetLastError();
 }
 

@@ -82,7 +82,8 @@ cudaError_t launch_collision_count(const FwdLaunch& p, const ViewRec* views, con
                                    unsigned long long* counters, bool wide_index, cudaStream_t stream);
 size_t back_brick_smem_bytes(const int32_t brick[3]);
 cudaError_t launch_geometry_gradient(const FwdLaunch& p, const ViewRec* views, const double* trig, const float* vol,
-                                     const float* gsino, double* grad, bool wide_index, cudaStream_t stream);
+                                     const float* volT, const float* gsino, double* grad, bool wide_index,
+                                     cudaStream_t stream);
 
 // Host helpers (ctp_api.cu).
 ctp_status host_validate(const ctp_geom_desc* d);

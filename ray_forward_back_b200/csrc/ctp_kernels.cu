@@ -64,28 +64,6 @@ constexpr int kBackThreads = 256;
 #endif
 constexpr int kBackStage = CTP_BACK_STAGE;  // views per fixed-point accumulation stage of the adjoint
 
-template <typename T>
-__device__ __forceinline__ T pick3(int k, T a0, T a1, T a2) {
-  return k == 0 ? a0 : (k == 1 ? a1 : a2);
-}
-
-// Axis roles of a walk: a = major (crossed most often, smallest spacing
-// between crossings), c = the minor axis crossed least often, b = the other.
-__device__ __forceinline__ void walk_axes(const Walk& W, int& a, int& b, int& c) {
-  const float i0 = W.inc[0], i1 = W.inc[1], i2 = W.inc[2];
-  a = (i0 <= i1 && i0 <= i2) ? 0 : (i1 <= i2 ? 1 : 2);
-  if (a == 0) {
-    b = i1 <= i2 ? 1 : 2;
-    c = 3 - b;
-  } else if (a == 1) {
-    b = i0 <= i2 ? 0 : 2;
-    c = 2 - b;
-  } else {
-    b = i0 <= i1 ? 0 : 1;
-    c = 1 - b;
-  }
-}
-
 // FP32 Siddon walk in major-axis slabs, one lane per ray (lanes run
 // independently).  Each slab between two successive planes of the major axis
 // a holds at most one crossing of each minor axis, so it is one, two or three
