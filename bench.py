@@ -7,7 +7,9 @@ A step is one forward projection and one back projection of the workload
 resident in HBM.  value = (forward updates + back updates) / step time, in
 Gupdates/s (ray-voxel updates), summed over ranks; with N > 1 every rank runs
 its own copy of the workload (independent problems, weak scaling, no
-collective on the data path).  Rank 0 prints one JSON line.
+collective on the data path).  Rank 0 prints one JSON line.  The geometry
+gradient (flat detectors) is timed on its own after the step and reported
+under "geometry_gradient"; it is not part of the step.
 
 --impl reference times the FP64 CPU oracle on a bounded sample of the same
 workload (the reference arm; slow by design).
@@ -59,15 +61,16 @@ def measured_traffic(kernel, workload_index):
     path = os.path.join(ROOT, "profiles", "dram_traffic_parallel512_900views.json")
     try:
         with open(path) as f:
-            rec = json.load(f)
-        with open(os.path.join(ROOT, rec["kernel_source"]), "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()
+            k = json.load(f)["kernels"][kernel]
+        h = hashlib.sha256()
+        for src in k["sources"]:
+            with open(os.path.join(ROOT, src), "rb") as f:
+                h.update(f.read())
     except Exception:
         return None
-    if sha != rec.get("kernel_source_sha256") or workload_index != 4:
+    if h.hexdigest() != k.get("sources_sha256") or workload_index != 4:
         return None
-    k = rec["kernels"].get(kernel)
-    return int(k["dram_bytes_per_launch"]) if k else None
+    return int(k["dram_bytes_per_launch"])
 
 
 def algorithmic_bytes(U, n_vox, n_rays):
@@ -264,6 +267,27 @@ def run_e2e(args, P, g, wl, vol_host, U, world, dev):
             "pipelining": "copies on separate streams, double-buffered device buffers"}
 
 
+def time_geometry_gradient(args, P, g, vol, sino_grad, stream, U, world, dev):
+    """Device time of ctp_geometry_gradient (one traversal of every ray,
+    reading the volume and an upstream sinogram gradient), CUDA events on the
+    launching stream after warm-up, max over ranks."""
+    import torch
+    out = torch.empty((g.n_views, 4, 3), dtype=torch.float64, device=dev)
+    for _ in range(max(1, args.warmup)):
+        P.geometry_gradient(vol, sino_grad, out=out, stream=stream)
+    stream.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        P.geometry_gradient(vol, sino_grad, out=out, stream=stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = aggregate_over_ranks([t0.elapsed_time(t1) / args.steps], world, dev)[0]
+    return {"ms": ms, "gupdates_s": U / (ms * 1e-3) / 1e9, "kernel": "geometry_gradient_kernel",
+            "launches_per_call": 1 + (1 if P.info()["n_transposed_views"] > 0 else 0)}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -331,9 +355,17 @@ def run_ours(args, rank, world, local_rank):
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, P, g, wl, vol_host, U, world, dev)
+    # geometry gradients (flat detectors): timed on their own after the step
+    grad = None
+    if not args.no_extras and g.detector == W.DET_FLAT:
+        grad = time_geometry_gradient(args, P, g, vol, sino_in, stream, U, world, dev)
     if rank != 0:
         return 0
     peak, peak_kind = measured_hbm_peak()
+    if grad is not None:
+        gb = algorithmic_bytes(U, g.n_vox, g.n_rays) / (grad["ms"] * 1e-3) / 1e9
+        grad.update({"effective_gbs": gb, "frac_of_hbm": gb / peak,
+                     "traffic": measured_traffic("geometry_gradient_kernel", wl.index) if not args.views else None})
     B = algorithmic_bytes(U, g.n_vox, g.n_rays)
     dominant = "back" if back_avg >= fwd_avg else "forward"
     if dominant == "back":
@@ -367,6 +399,7 @@ def run_ours(args, rank, world, local_rank):
                      "unit": "GB/s", "frac": achieved / peak,
                      "traffic": measured_traffic(dom_kernel, wl.index) if not args.views else None,
                      "algorithmic_bytes_per_launch": B},
+        "geometry_gradient": grad,
         "clocks": clk,
         "e2e": e2e,
         "gpu_launches": args.steps * (2 + (1 if info["n_transposed_views"] > 0 else 0)),
@@ -387,6 +420,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip the geometry-gradient timing")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -46,6 +46,19 @@
 namespace ctp {
 namespace {
 
+// Tuning knobs (compile-time; the defaults are the measured choices: 4 CTAs
+// per SM with the setup recomputed after the walk, 2 / 1 slab unroll).
+#ifndef CTP_GRAD_MIN_BLOCKS
+#define CTP_GRAD_MIN_BLOCKS 4
+#endif
+#ifndef CTP_GRAD_UNROLL2
+#define CTP_GRAD_UNROLL2 2
+#endif
+#ifndef CTP_GRAD_UNROLL3
+#define CTP_GRAD_UNROLL3 1
+#endif
+constexpr int kGradUnroll2 = CTP_GRAD_UNROLL2;
+constexpr int kGradUnroll3 = CTP_GRAD_UNROLL3;
 constexpr int kGradCols = 32;
 constexpr int kGradRows = 8;
 constexpr int kGradThreads = kGradCols * kGradRows;
@@ -129,7 +142,7 @@ __device__ __forceinline__ float crossing_sums(bool active, const Walk& W, const
     float tb = Nb > 0 ? l0b : CUDART_INF_F, tc = Nc > 0 ? l0c : CUDART_INF_F;
     float fjb = 1.f, fjc = 1.f, cur = 0.f;
     if (!__any_sync(kFull, active && Nc > 0)) {
-#pragma unroll 4
+#pragma unroll kGradUnroll2
       for (int k = 0; k <= kmax; ++k) {
         const int s = k - d;
         const bool on = (unsigned)s <= (unsigned)Na;
@@ -159,7 +172,7 @@ __device__ __forceinline__ float crossing_sums(bool active, const Walk& W, const
         }
       }
     } else {
-#pragma unroll 2
+#pragma unroll kGradUnroll3
       for (int k = 0; k <= kmax; ++k) {
         const int s = k - d;
         const bool on = (unsigned)s <= (unsigned)Na;
@@ -211,7 +224,7 @@ __device__ __forceinline__ float crossing_sums(bool active, const Walk& W, const
 }
 
 template <typename Off>
-__global__ void __launch_bounds__(kGradThreads) geometry_gradient_kernel(FwdLaunch P,
+__global__ void __launch_bounds__(kGradThreads, CTP_GRAD_MIN_BLOCKS) geometry_gradient_kernel(FwdLaunch P,
                                                                          const ViewRec* __restrict__ views,
                                                                          const double* __restrict__ trig,
                                                                          const float* __restrict__ vol,
@@ -227,22 +240,27 @@ __global__ void __launch_bounds__(kGradThreads) geometry_gradient_kernel(FwdLaun
   const int r = band * kGradRows + threadIdx.y;
   const bool valid = c < P.dims.n_cols && r < P.dims.n_rows;
 
-  const ViewRec& V = views[v];
-  Ray R;
-  const bool from_pixel = make_ray(V, P.vol, trig, P.dims, v, valid ? r : 0, valid ? c : 0, R);
   const int lo[3] = {0, 0, 0};
   const int hi[3] = {P.vol.n[0], P.vol.n[1], P.vol.n[2]};
-  double t_in = 0.0, t_out = 0.0;
-  int k_in = -1, k_out = -1;
   const float gr = valid ? gsino[((size_t)v * P.dims.n_rows + r) * P.dims.n_cols + c] : 0.f;
-  const bool hit = valid && gr != 0.f && clip_faces(R, hi, t_in, t_out, k_in, k_out);
+  const int rr = valid ? r : 0, cc = valid ? c : 0;
 
-  // per-axis sums S0_k and sum of dx * (local distance from the entry)
+  // Pass 1: FP64 setup, then the FP32 walk for the per-axis crossing sums.
   Walk W = {};
-  if (hit) entry(R, t_in, t_out, lo, hi, W);
+  bool hit;
+  bool yfast;
+  {
+    const ViewRec& V = views[v];
+    Ray R;
+    make_ray(V, P.vol, trig, P.dims, v, rr, cc, R);
+    double t_in = 0.0, t_out = 0.0;
+    int k_in, k_out;
+    hit = valid && gr != 0.f && clip_faces(R, hi, t_in, t_out, k_in, k_out);
+    if (hit) entry(R, t_in, t_out, lo, hi, W);
+    yfast = V.layout != 0;
+  }
   // gather from the x-fastest volume or its y-fastest copy, as the forward does
   const Off nx = P.vol.n[0], ny = P.vol.n[1];
-  const bool yfast = V.layout != 0;
   const float* __restrict__ base = yfast ? volT : vol;
   const Off sx = yfast ? ny : (Off)1, sy = yfast ? (Off)1 : nx, sz = nx * ny;
   const Off off = (Off)W.i[2] * sz + (Off)W.i[1] * sy + (Off)W.i[0] * sx;
@@ -250,6 +268,19 @@ __global__ void __launch_bounds__(kGradThreads) geometry_gradient_kernel(FwdLaun
   float f0[3], fl[3];
   const float last =
       crossing_sums<Off>(hit, W, hi, base, off, W.step[0] * sx, W.step[1] * sy, W.step[2] * sz, first, f0, fl);
+
+  // Pass 2: the same FP64 setup again (bit-identical), recomputed rather than
+  // kept live through the walk so the walk runs with fewer registers; the
+  // opaque copy of the record pointer keeps the compiler from merging the
+  // two setups.
+  const ViewRec* vp = views + v;
+  asm volatile("" : "+l"(vp));
+  const ViewRec& V = *vp;
+  Ray R;
+  const bool from_pixel = make_ray(V, P.vol, trig, P.dims, v, rr, cc, R);
+  double t_in = 0.0, t_out = 0.0;
+  int k_in = -1, k_out = -1;
+  if (hit) clip_faces(R, hi, t_in, t_out, k_in, k_out);
   double S0[3], Sl[3];
   // the faces: entering at local distance 0, leaving at the segment's length
   const double Lseg = (t_out - t_in) * R.len;
