@@ -83,7 +83,9 @@ typedef struct {
   int32_t brick[3];          /* adjoint brick (bx, by, bz) in voxels; 0 = automatic */
   int32_t view_groups;       /* adjoint: split the views over this many CTA groups; 0 = automatic */
   int32_t forward_layout;    /* 0 = automatic per view, 1 = always x-fastest volume, 2 = always y-fastest */
-  int32_t reserved[10];
+  int32_t batch_chunk;       /* ctp_forward_batch: volumes per fused launch, 1, 2 or 4; 0 = 1.  The
+                                y-fastest scratch copy (if any view uses it) grows by this factor. */
+  int32_t reserved[9];
 } ctp_plan;
 
 /* Acquisition and volume description.  All pointers are HOST pointers; the
@@ -113,6 +115,8 @@ typedef struct {
   int32_t view_groups;
   int32_t n_transposed_views;   /* views whose forward gathers from the y-fastest copy */
   double collision_ratio;       /* updates / distinct voxels per sort batch, measured at create */
+  int32_t batch_chunk;          /* volumes per fused ctp_forward_batch launch */
+  int32_t reserved;
 } ctp_geom_info;
 
 /*
@@ -160,6 +164,24 @@ ctp_status ctp_forward(const ctp_geom *geom, const float *vol, float *sino, void
  * each volume block whose detector footprint holds it is written as NaN.
  */
 ctp_status ctp_back(const ctp_geom *geom, const float *sino, float *vol, void *stream);
+
+/*
+ * ctp_forward_batch / ctp_back_batch — the projections of n_batch volumes
+ * (sinograms) that share one geometry, laid out one after the other:
+ *   vol:  device pointer, float32 [n_batch][nz][ny][nx]
+ *   sino: device pointer, float32 [n_batch][n_views][n_rows][n_cols]
+ * Member b's output is exactly what ctp_forward / ctp_back give for member b
+ * alone (leading batch dimensions are preserved, diffct "Execution", section
+ * "Batch dimensions and axis spacing"; empty batches included: n_batch = 0
+ * does nothing and returns CTP_OK without looking at the pointers).
+ * The forward walks every ray once per chunk of plan.batch_chunk members and
+ * gathers from all of them, so the per-ray set-up and walk control are shared
+ * across the chunk; the adjoint runs member by member.  n_batch < 0, or a
+ * batch whose element count exceeds 2^62, gives CTP_ERR_INVALID_ARGUMENT.
+ * Same pointer, stream and synchronisation rules as ctp_forward / ctp_back.
+ */
+ctp_status ctp_forward_batch(const ctp_geom *geom, const float *vol, float *sino, int64_t n_batch, void *stream);
+ctp_status ctp_back_batch(const ctp_geom *geom, const float *sino, float *vol, int64_t n_batch, void *stream);
 
 /*
  * ctp_back_power — vol = (A∘A)^T sino for power 2 (every coefficient squared)

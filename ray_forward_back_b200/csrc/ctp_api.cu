@@ -34,6 +34,7 @@ struct ctp_geom {
   float *d_volT = nullptr;
   unsigned long long *d_counter = nullptr;
   int64_t scratch_bytes = 0;
+  int batch_chunk = 1;  // volumes per fused batched forward launch (y-fastest copies held)
 };
 
 namespace {
@@ -156,6 +157,8 @@ ctp_status validate_desc(const ctp_geom_desc *d) {
       if (p->brick[k] < 0 || p->brick[k] > 1024) return fail(CTP_ERR_INVALID_ARGUMENT, "plan.brick[%d]", k);
     if (p->view_groups < 0) return fail(CTP_ERR_INVALID_ARGUMENT, "plan.view_groups");
     if (p->forward_layout < 0 || p->forward_layout > 2) return fail(CTP_ERR_INVALID_ARGUMENT, "plan.forward_layout");
+    if (p->batch_chunk != 0 && p->batch_chunk != 1 && p->batch_chunk != 2 && p->batch_chunk != 4)
+      return fail(CTP_ERR_INVALID_ARGUMENT, "plan.batch_chunk %d is not 0, 1, 2 or 4", p->batch_chunk);
   }
   return CTP_OK;
 }
@@ -523,6 +526,7 @@ ctp_status ctp_geom_create(const ctp_geom_desc *desc, ctp_geom **out) {
   f.any_transposed = g->n_transposed > 0;
   const ctp_plan *plan = desc->plan;
   g->adjoint_variant = CTP_ADJOINT_BRICK;
+  g->batch_chunk = plan && plan->batch_chunk > 0 ? plan->batch_chunk : 1;
 
   DeviceGuard dg(g->device);
   int sm_count = 0;
@@ -552,7 +556,8 @@ ctp_status ctp_geom_create(const ctp_geom_desc *desc, ctp_geom **out) {
   st = alloc((void **)&g->d_views, vbytes, "view records");
   if (st == CTP_OK && !trig.empty()) st = alloc((void **)&g->d_trig, sizeof(double) * trig.size(), "column angles");
   if (st == CTP_OK && f.any_transposed)
-    st = alloc((void **)&g->d_volT, sizeof(float) * (size_t)g->n_vox, "y-fastest volume copy");
+    st = alloc((void **)&g->d_volT, sizeof(float) * (size_t)g->n_vox * (size_t)g->batch_chunk,
+               "y-fastest volume copies");
   if (st == CTP_OK) st = alloc((void **)&g->d_counter, sizeof(unsigned long long), "counter");
   cudaError_t e = cudaSuccess;
   if (st == CTP_OK) {
@@ -594,6 +599,8 @@ ctp_status ctp_geom_query(const ctp_geom *g, ctp_geom_info *info) {
   info->view_groups = g->back.view_groups;
   info->n_transposed_views = g->n_transposed;
   info->collision_ratio = g->collision_ratio;
+  info->batch_chunk = g->batch_chunk;
+  info->reserved = 0;
   return CTP_OK;
 }
 
@@ -613,8 +620,62 @@ ctp_status ctp_forward(const ctp_geom *g, const float *vol, float *sino, void *s
     e = ctp::launch_transpose_xy(vol, g->d_volT, g->vol, s);
     if (e != cudaSuccess) return cuda_fail(e, "transpose launch");
   }
-  e = ctp::launch_forward(g->fwd, g->d_views, g->d_trig, vol, g->d_volT, sino, g->wide_index, s);
+  e = ctp::launch_forward(g->fwd, g->d_views, g->d_trig, vol, g->d_volT, sino, 1, g->wide_index, s);
   if (e != cudaSuccess) return cuda_fail(e, "forward launch");
+  return CTP_OK;
+}
+
+namespace {
+// n_batch >= 0 and the batch's largest array below 2^62 elements.
+ctp_status check_batch(const ctp_geom *g, int64_t n_batch) {
+  if (n_batch < 0) return fail(CTP_ERR_INVALID_ARGUMENT, "n_batch %lld is negative", (long long)n_batch);
+  const double most = (double)n_batch * (double)(g->n_vox > g->n_rays ? g->n_vox : g->n_rays);
+  if (most >= 4.6e18) return fail(CTP_ERR_INVALID_ARGUMENT, "batch of %lld is too large", (long long)n_batch);
+  return CTP_OK;
+}
+}  // namespace
+
+ctp_status ctp_forward_batch(const ctp_geom *g, const float *vol, float *sino, int64_t n_batch, void *stream) {
+  g_detail[0] = '\0';
+  if (!g) return fail(CTP_ERR_INVALID_ARGUMENT, "geometry is NULL");
+  ctp_status st = check_batch(g, n_batch);
+  if (st != CTP_OK || n_batch == 0) return st;
+  DeviceGuard dg(g->device);
+  if (dg.err != cudaSuccess) return cuda_fail(dg.err, "cudaSetDevice");
+  if (!is_device_pointer(vol, g->device))
+    return fail(CTP_ERR_INVALID_ARGUMENT, "vol is not device memory of device %d", g->device);
+  if (!is_device_pointer(sino, g->device))
+    return fail(CTP_ERR_INVALID_ARGUMENT, "sino is not device memory of device %d", g->device);
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "pending error before ctp_forward_batch");
+  for (int64_t b0 = 0; b0 < n_batch;) {
+    // the largest supported chunk that fits the remaining members
+    int kb = g->batch_chunk;
+    while (kb > 1 && b0 + kb > n_batch) kb >>= 1;
+    const float *v0 = vol + (size_t)b0 * (size_t)g->n_vox;
+    if (g->fwd.any_transposed)
+      for (int j = 0; j < kb && e == cudaSuccess; ++j)
+        e = ctp::launch_transpose_xy(v0 + (size_t)j * (size_t)g->n_vox, g->d_volT + (size_t)j * (size_t)g->n_vox,
+                                     g->vol, s);
+    if (e == cudaSuccess)
+      e = ctp::launch_forward(g->fwd, g->d_views, g->d_trig, v0, g->d_volT, sino + (size_t)b0 * (size_t)g->n_rays,
+                              kb, g->wide_index, s);
+    if (e != cudaSuccess) return cuda_fail(e, "batched forward launch");
+    b0 += kb;
+  }
+  return CTP_OK;
+}
+
+ctp_status ctp_back_batch(const ctp_geom *g, const float *sino, float *vol, int64_t n_batch, void *stream) {
+  g_detail[0] = '\0';
+  if (!g) return fail(CTP_ERR_INVALID_ARGUMENT, "geometry is NULL");
+  ctp_status st = check_batch(g, n_batch);
+  if (st != CTP_OK || n_batch == 0) return st;
+  for (int64_t b = 0; b < n_batch; ++b) {
+    st = ctp_back_power(g, sino + (size_t)b * (size_t)g->n_rays, vol + (size_t)b * (size_t)g->n_vox, 1, stream);
+    if (st != CTP_OK) return st;
+  }
   return CTP_OK;
 }
 

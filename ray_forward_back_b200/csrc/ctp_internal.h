@@ -70,8 +70,10 @@ struct BackLaunch {
 
 // Launchers (ctp_kernels.cu).  All enqueue on `stream` and return the launch error.
 cudaError_t launch_transpose_xy(const float* vol, float* volT, const VolDesc& vd, cudaStream_t stream);
+// Forward of kb (1, 2 or 4) volumes at vol, vol + n_vox, ... (their y-fastest
+// copies at volT, volT + n_vox, ...) into kb sinograms at sino, sino + n_rays, ...
 cudaError_t launch_forward(const FwdLaunch& p, const ViewRec* views, const double* trig, const float* vol,
-                           const float* volT, float* sino, bool wide_index, cudaStream_t stream);
+                           const float* volT, float* sino, int kb, bool wide_index, cudaStream_t stream);
 cudaError_t launch_back_brick(const BackLaunch& p, const ViewRec* views, const double* trig, const float* sino,
                               float* vol, int power, bool wide_index, cudaStream_t stream);
 cudaError_t launch_count(const FwdLaunch& p, const ViewRec* views, const double* trig,

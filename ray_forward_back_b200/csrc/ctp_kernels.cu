@@ -336,12 +336,13 @@ __device__ __forceinline__ void walk(bool active, const Walk& W, const int lo[3]
 
 // ------------------------------------------------------------------ forward --
 
-template <typename Off>
-__global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_FWD_MIN_BLOCKS) forward_kernel(FwdLaunch P, const ViewRec* __restrict__ views,
-                                                                     const double* __restrict__ trig,
-                                                                     const float* __restrict__ vol,
-                                                                     const float* __restrict__ volT,
-                                                                     float* __restrict__ sino) {
+// kB volumes per launch (a chunk of a batch sharing the geometry): each ray is
+// walked once and every segment gathers from all kB volumes, so the FP64
+// set-up and the walk control are shared; kB = 1 is the plain forward.
+template <typename Off, int kB>
+__global__ void __launch_bounds__(kFwdCols* kFwdRows, kB == 1 ? CTP_FWD_MIN_BLOCKS : 4)
+    forward_kernel(FwdLaunch P, const ViewRec* __restrict__ views, const double* __restrict__ trig,
+                   const float* __restrict__ vol, const float* __restrict__ volT, float* __restrict__ sino) {
   const int per_band = P.dims.n_views * P.n_col_tiles;
   const int band = blockIdx.x / per_band;
   const int rem = blockIdx.x - band * per_band;
@@ -367,10 +368,21 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_FWD_MIN_BLOCKS) forwar
   const Off sy = yfast ? (Off)1 : nx;
   const Off sz = nx * ny;
   const Off off = (Off)W.i[2] * sz + (Off)W.i[1] * sy + (Off)W.i[0] * sx;
-  float acc = 0.f;
+  const size_t n_vox = (size_t)P.vol.n[0] * (size_t)P.vol.n[1] * (size_t)P.vol.n[2];
+  float acc[kB];
+#pragma unroll
+  for (int j = 0; j < kB; ++j) acc[j] = 0.f;
   walk<true, false, Off>(hit, W, lo, hi, off, W.step[0] * sx, W.step[1] * sy, W.step[2] * sz,
-                         [&](Off o, float len, bool) { acc = fmaf(len, __ldg(base + o), acc); });
-  if (valid) sino[((size_t)v * P.dims.n_rows + r) * P.dims.n_cols + c] = acc;
+                         [&](Off o, float len, bool) {
+#pragma unroll
+                           for (int j = 0; j < kB; ++j) acc[j] = fmaf(len, __ldg(base + j * n_vox + o), acc[j]);
+                         });
+  if (valid) {
+    const size_t n_rays = (size_t)P.dims.n_views * P.dims.n_rows * P.dims.n_cols;
+    const size_t i = ((size_t)v * P.dims.n_rows + r) * P.dims.n_cols + c;
+#pragma unroll
+    for (int j = 0; j < kB; ++j) sino[j * n_rays + i] = acc[j];
+  }
 }
 
 // ------------------------------------------------------------------- count --
@@ -878,15 +890,27 @@ cudaError_t launch_transpose_xy(const float* vol, float* volT, const VolDesc& vd
 }
 
 cudaError_t launch_forward(const FwdLaunch& p, const ViewRec* views, const double* trig, const float* vol,
-                           const float* volT, float* sino, bool wide_index, cudaStream_t stream) {
+                           const float* volT, float* sino, int kb, bool wide_index, cudaStream_t stream) {
   const long long blocks = (long long)p.n_row_bands * p.dims.n_views * p.n_col_tiles;
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   dim3 block(kFwdCols, kFwdRows);
-  if (wide_index)
-    forward_kernel<long long><<<(unsigned)blocks, block, 0, stream>>>(p, views, trig, vol, volT, sino);
-  else
-    forward_kernel<int><<<(unsigned)blocks, block, 0, stream>>>(p, views, trig, vol, volT, sino);
+  const unsigned nb = (unsigned)blocks;
+#define CTP_FWD_LAUNCH(OFF, KB) forward_kernel<OFF, KB><<<nb, block, 0, stream>>>(p, views, trig, vol, volT, sino)
+  switch (kb) {
+    case 1:
+      if (wide_index) CTP_FWD_LAUNCH(long long, 1); else CTP_FWD_LAUNCH(int, 1);
+      break;
+    case 2:
+      if (wide_index) CTP_FWD_LAUNCH(long long, 2); else CTP_FWD_LAUNCH(int, 2);
+      break;
+    case 4:
+      if (wide_index) CTP_FWD_LAUNCH(long long, 4); else CTP_FWD_LAUNCH(int, 4);
+      break;
+    default:
+      return cudaErrorInvalidValue;
+  }
+#undef CTP_FWD_LAUNCH
   return cudaGetLastError();
 }
 

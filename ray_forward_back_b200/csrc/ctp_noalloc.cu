@@ -162,7 +162,7 @@ extern "C" ctp_status ctp_forward_noalloc(const ctp_geom_desc* desc, const float
     e = launch_transpose_xy(vol, d_copy, f.vol, s);
     if (e != cudaSuccess) return host_cuda_error(e, "transpose launch");
   }
-  e = launch_forward(f, d_views, d_trig, vol, d_copy, sino, wide, s);
+  e = launch_forward(f, d_views, d_trig, vol, d_copy, sino, 1, wide, s);
   if (e != cudaSuccess) return host_cuda_error(e, "forward launch");
   return CTP_OK;
 }

@@ -11,6 +11,7 @@ torch CUDA tensors and the current torch stream.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 from typing import Optional
 
@@ -35,7 +36,7 @@ CTP_ADJOINT_BRICK = 1
 CTP_ADJOINT_SORT = 2
 
 EXPORTED = ["ctp_geom_create", "ctp_geom_destroy", "ctp_geom_query", "ctp_forward", "ctp_back",
-            "ctp_back_power", "ctp_geometry_gradient", "ctp_count_updates", "ctp_forward_noalloc", "ctp_solve", "ctp_solver_workspace_bytes",
+            "ctp_forward_batch", "ctp_back_batch", "ctp_back_power", "ctp_geometry_gradient", "ctp_count_updates", "ctp_forward_noalloc", "ctp_solve", "ctp_solver_workspace_bytes",
             "ctp_status_string", "ctp_last_error_detail", "ctp_version"]
 CTP_SOLVER_CGLS = 1
 CTP_SOLVER_SIRT = 2
@@ -44,7 +45,7 @@ CTP_SOLVER_SIRT = 2
 class ctp_plan(ctypes.Structure):
     _fields_ = [("adjoint_variant", ctypes.c_int32), ("brick", ctypes.c_int32 * 3),
                 ("view_groups", ctypes.c_int32), ("forward_layout", ctypes.c_int32),
-                ("reserved", ctypes.c_int32 * 10)]
+                ("batch_chunk", ctypes.c_int32), ("reserved", ctypes.c_int32 * 9)]
 
 
 class ctp_geom_desc(ctypes.Structure):
@@ -62,7 +63,8 @@ class ctp_geom_info(ctypes.Structure):
     _fields_ = [("n_rays", ctypes.c_int64), ("n_vox", ctypes.c_int64), ("scratch_bytes", ctypes.c_int64),
                 ("adjoint_variant", ctypes.c_int32), ("brick", ctypes.c_int32 * 3),
                 ("view_groups", ctypes.c_int32), ("n_transposed_views", ctypes.c_int32),
-                ("collision_ratio", ctypes.c_double)]
+                ("collision_ratio", ctypes.c_double), ("batch_chunk", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
 
 
 class ctp_solver_options(ctypes.Structure):
@@ -106,6 +108,10 @@ def load(path: str = None):
         lib.ctp_forward.restype = ctypes.c_int
         lib.ctp_back.argtypes = [vp, vp, vp, vp]
         lib.ctp_back.restype = ctypes.c_int
+        lib.ctp_forward_batch.argtypes = [vp, vp, vp, i64, vp]
+        lib.ctp_forward_batch.restype = ctypes.c_int
+        lib.ctp_back_batch.argtypes = [vp, vp, vp, i64, vp]
+        lib.ctp_back_batch.restype = ctypes.c_int
         lib.ctp_back_power.argtypes = [vp, vp, vp, ctypes.c_int, vp]
         lib.ctp_back_power.restype = ctypes.c_int
         lib.ctp_geometry_gradient.argtypes = [vp, vp, vp, vp, vp]
@@ -183,6 +189,7 @@ class _Desc:
             p.brick[:] = [int(x) for x in plan.get("brick", (0, 0, 0))]
             p.view_groups = int(plan.get("view_groups", 0))
             p.forward_layout = int(plan.get("forward_layout", 0))
+            p.batch_chunk = int(plan.get("batch_chunk", 0))
             self.plan = p
             d.plan = ctypes.pointer(p)
         self.desc = d
@@ -207,7 +214,8 @@ def ctp_geom_query(handle: int) -> dict:
     _check(load().ctp_geom_query(handle, ctypes.byref(info)))
     return {"n_rays": info.n_rays, "n_vox": info.n_vox, "scratch_bytes": info.scratch_bytes,
             "adjoint_variant": info.adjoint_variant, "brick": tuple(info.brick), "view_groups": info.view_groups,
-            "n_transposed_views": info.n_transposed_views, "collision_ratio": info.collision_ratio}
+            "n_transposed_views": info.n_transposed_views, "collision_ratio": info.collision_ratio,
+            "batch_chunk": info.batch_chunk}
 
 
 def ctp_forward(handle: int, vol, sino, stream=None) -> None:
@@ -216,6 +224,14 @@ def ctp_forward(handle: int, vol, sino, stream=None) -> None:
 
 def ctp_back(handle: int, sino, vol, stream=None) -> None:
     _check(load().ctp_back(handle, _ptr(sino), _ptr(vol), _stream_handle(stream)))
+
+
+def ctp_forward_batch(handle: int, vol, sino, n_batch: int, stream=None) -> None:
+    _check(load().ctp_forward_batch(handle, _ptr(vol), _ptr(sino), int(n_batch), _stream_handle(stream)))
+
+
+def ctp_back_batch(handle: int, sino, vol, n_batch: int, stream=None) -> None:
+    _check(load().ctp_back_batch(handle, _ptr(sino), _ptr(vol), int(n_batch), _stream_handle(stream)))
 
 
 def ctp_back_power(handle: int, sino, vol, power: int, stream=None) -> None:
@@ -275,10 +291,10 @@ def ctp_version() -> str:
 class Projector:
     """Matched forward / back projector on one CUDA device.
 
-    ``forward(vol)`` takes a float32 CUDA tensor (nz, ny, nx) and returns the
-    sinogram (n_views, n_rows, n_cols); ``back(sino)`` the reverse.  Both run
-    on the current torch stream unless a stream is given, and never
-    synchronise.
+    ``forward(vol)`` takes a float32 CUDA tensor (..., nz, ny, nx) and returns
+    the sinogram (..., n_views, n_rows, n_cols); ``back(sino)`` the reverse.
+    Leading batch dimensions are preserved, empty ones included.  Both run on
+    the current torch stream unless a stream is given, and never synchronise.
     """
 
     def __init__(self, geom, device: int = 0, plan: Optional[dict] = None):
@@ -313,22 +329,39 @@ class Projector:
         if tuple(t.shape) != tuple(shape) or not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous with shape {tuple(shape)}")
 
+    def _lead(self, t, inner, name):
+        """Leading batch shape of t, whose trailing dimensions must be `inner`."""
+        import torch
+        if not isinstance(t, torch.Tensor) or t.dim() < len(inner):
+            raise TypeError(f"{name} must be a float32 CUDA tensor (..., {', '.join(map(str, inner))})")
+        lead = tuple(t.shape[: t.dim() - len(inner)])
+        self._check_tensor(t, lead + tuple(inner), name)
+        return lead
+
     def forward(self, vol, out=None, stream=None):
         import torch
-        self._check_tensor(vol, self.geom.vol_shape, "vol")
+        lead = self._lead(vol, self.geom.vol_shape, "vol")
+        shape = lead + tuple(self.geom.sino_shape)
         if out is None:
-            out = torch.empty(self.geom.sino_shape, dtype=torch.float32, device=vol.device)
-        self._check_tensor(out, self.geom.sino_shape, "out")
-        ctp_forward(self.handle, vol, out, stream)
+            out = torch.empty(shape, dtype=torch.float32, device=vol.device)
+        self._check_tensor(out, shape, "out")
+        if lead:
+            ctp_forward_batch(self.handle, vol, out, math.prod(lead), stream)
+        else:
+            ctp_forward(self.handle, vol, out, stream)
         return out
 
     def back(self, sino, out=None, stream=None):
         import torch
-        self._check_tensor(sino, self.geom.sino_shape, "sino")
+        lead = self._lead(sino, self.geom.sino_shape, "sino")
+        shape = lead + tuple(self.geom.vol_shape)
         if out is None:
-            out = torch.empty(self.geom.vol_shape, dtype=torch.float32, device=sino.device)
-        self._check_tensor(out, self.geom.vol_shape, "out")
-        ctp_back(self.handle, sino, out, stream)
+            out = torch.empty(shape, dtype=torch.float32, device=sino.device)
+        self._check_tensor(out, shape, "out")
+        if lead:
+            ctp_back_batch(self.handle, sino, out, math.prod(lead), stream)
+        else:
+            ctp_back(self.handle, sino, out, stream)
         return out
 
     def back_power(self, sino, power: int, out=None, stream=None):

@@ -116,6 +116,8 @@ def test_cylindrical_needs_cone_and_orthogonal_frame(lib):
 def test_bad_plan(lib):
     _expect(ctp.CTP_ERR_INVALID_ARGUMENT, _cone(), {"adjoint_variant": 7})
     _expect(ctp.CTP_ERR_INVALID_ARGUMENT, _cone(), {"brick": (0, -1, 0)})
+    for chunk in (-1, 3, 8):
+        _expect(ctp.CTP_ERR_INVALID_ARGUMENT, _cone(), {"batch_chunk": chunk})
 
 
 def test_valid_geometry_without_a_gpu_fails_with_cuda_status(lib):
@@ -130,4 +132,6 @@ def test_null_arguments(lib):
     assert lib.ctp_geom_create(None, ctypes.byref(h)) == ctp.CTP_ERR_INVALID_ARGUMENT
     assert lib.ctp_forward(None, None, None, None) == ctp.CTP_ERR_INVALID_ARGUMENT
     assert lib.ctp_back(None, None, None, None) == ctp.CTP_ERR_INVALID_ARGUMENT
+    assert lib.ctp_forward_batch(None, None, None, 0, None) == ctp.CTP_ERR_INVALID_ARGUMENT
+    assert lib.ctp_back_batch(None, None, None, 2, None) == ctp.CTP_ERR_INVALID_ARGUMENT
     lib.ctp_geom_destroy(None)
