@@ -106,3 +106,102 @@ def test_sharded_projection_equals_unsharded(world, n_views):
     slabs = sorted((out[r][4], out[r][5], out[r][6]) for r in range(world))
     x_slabs = np.concatenate([s for _, _, s in slabs], axis=0)
     np.testing.assert_allclose(x_slabs, x_ref, rtol=1e-6, atol=1e-6 * np.abs(x_ref).max())
+
+
+# ------------------------------------------------------------ slice sharding --
+
+def _slice_geometries():
+    from ray_forward_back_b200 import workloads as W
+    gs = {}
+    # one row per slice, rows and slices aligned
+    gs["aligned"] = W.make_parallel(9, 8, 7, 5, 7, 11, pitch_u=0.9, pitch_v=1.0, start=0.21)
+    # several rows per slice, rows beyond the volume on both sides
+    gs["dense_rows"] = W.make_parallel(9, 8, 5, 4, 13, 10, pitch_u=1.1, pitch_v=0.55, start=0.37,
+                                       spacing=(1.0, 1.0, 1.3))
+    # coarse rows: some slices hold no row; rows step downwards
+    g = W.make_parallel(8, 9, 9, 3, 4, 9, pitch_u=1.0, pitch_v=2.1, start=0.11)
+    g.det_v = -g.det_v
+    gs["coarse_descending"] = g
+    return gs
+
+
+@pytest.mark.parametrize("name", sorted(_slice_geometries()))
+def test_slice_partition_covers_the_rows_inside_the_volume_once(name):
+    from ray_forward_back_b200.sharded import slice_partition
+    g = _slice_geometries()[name]
+    rc = 0.5 * (g.n_rows - 1)
+    z = g.det_c[0, 2] + (np.arange(g.n_rows) - rc) * g.det_v[0, 2]
+    inside = (z >= g.origin[2]) & (z < g.origin[2] + g.nz * g.spacing[2])
+    for world in (1, 2, 3, g.nz + 2):
+        owned = np.zeros(g.n_rows, dtype=int)
+        for r in range(world):
+            z0, z1, r0, r1 = slice_partition(g, r, world)
+            owned[r0:r1] += 1
+            sl = np.floor((z[r0:r1] - g.origin[2]) / g.spacing[2])
+            assert np.all((sl >= z0) & (sl < z1))
+        np.testing.assert_array_equal(owned, inside.astype(int))
+
+
+@pytest.mark.parametrize("name", sorted(_slice_geometries()))
+def test_slice_sharded_projection_equals_unsharded(name):
+    """Ranks emulated in one process (they exchange nothing): the rows and
+    slabs they produce reassemble the unsharded oracle projections."""
+    import torch
+    import oracle
+    from ray_forward_back_b200.sharded import SliceShardedProjector
+    g = _slice_geometries()[name]
+    rng = np.random.default_rng(1)
+    vol = rng.random(g.vol_shape).astype(np.float32)
+    sino = rng.random(g.sino_shape).astype(np.float32)
+    y_ref = oracle.forward(g, vol)
+    x_ref = oracle.back(g, sino)
+    for world in (2, 3):
+        y = np.zeros(g.sino_shape)
+        x = np.zeros(g.vol_shape)
+        for rank in range(world):
+            S = SliceShardedProjector(g, make_projector=_OracleProjector, rank=rank, world=world)
+            y[:, S.r0:S.r1] = S.forward(torch.from_numpy(vol[S.z0:S.z1].copy())).numpy()
+            x[S.z0:S.z1] = S.back(torch.from_numpy(sino[:, S.r0:S.r1].copy())).numpy()
+        np.testing.assert_allclose(y, y_ref.astype(np.float32), rtol=1e-6, atol=1e-6 * np.abs(y_ref).max())
+        np.testing.assert_allclose(x, x_ref.astype(np.float32), rtol=1e-6, atol=1e-6 * np.abs(x_ref).max())
+
+
+def test_slice_sharding_rejects_coupled_slices():
+    from ray_forward_back_b200 import workloads as W
+    from ray_forward_back_b200.sharded import slice_partition
+    cone = W.make_cone(8, 8, 8, 3, 4, 5, sid=30.0, sdd=50.0)
+    with pytest.raises(ValueError):
+        slice_partition(cone, 0, 2)
+    tilted = W.make_parallel(8, 8, 8, 3, 4, 5)
+    src = tilted.src.copy()
+    src[:, 2] = 0.1
+    tilted.src = src
+    with pytest.raises(ValueError):
+        slice_partition(tilted, 0, 2)
+    helix_like = W.make_parallel(8, 8, 8, 3, 4, 5)
+    dc = helix_like.det_c.copy()
+    dc[1, 2] += 0.25
+    helix_like.det_c = dc
+    with pytest.raises(ValueError):
+        slice_partition(helix_like, 0, 2)
+
+
+def _slice_rank_main(rank, world, port, out):
+    import torch.distributed as dist
+    from ray_forward_back_b200.sharded import SliceShardedProjector
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        g = _slice_geometries()["aligned"]
+        S = SliceShardedProjector(g, make_projector=_OracleProjector)
+        out[rank] = (S.rank, S.world, S.z0, S.z1, S.r0, S.r1)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_slice_sharding_takes_rank_and_world_from_the_group():
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.spawn(_slice_rank_main, args=(2, _free_port(), out), nprocs=2, join=True)
+    assert out[0] == (0, 2, 0, 4, 0, 4) and out[1] == (1, 2, 4, 7, 4, 7)
