@@ -550,8 +550,16 @@ __device__ void brick_footprint(const ViewRec& V, const BackLaunch& P, const int
     rmin = (q_lo * V.R - V.axial0) / V.vlen;
     rmax = (q_hi * V.R - V.axial0) / V.vlen;
   }
-  const double cl = fmax(floor(cmin - 1e-7), -1.0), ch = fmin(ceil(cmax + 1e-7), (double)nc);
-  const double rl = fmax(floor(rmin - 1e-7), -1.0), rh = fmin(ceil(rmax + 1e-7), (double)nr);
+  // Parallel and flat cone beams: the box projects exactly onto the hull of
+  // its projected corners, so the pixels inside [min, max] (widened by 1e-7
+  // pixel against FP64 rounding, which is below 1e-12 pixel here) are the
+  // only ones whose rays can meet it.  The cylindrical bounds above are
+  // themselves relaxations; they keep one more pixel on each side.
+  const bool exact = P.dims.beam == CTP_BEAM_PARALLEL || P.dims.det == CTP_DET_FLAT;
+  const double cl = fmax(exact ? ceil(cmin - 1e-7) : floor(cmin - 1e-7), -1.0);
+  const double ch = fmin(exact ? floor(cmax + 1e-7) : ceil(cmax + 1e-7), (double)nc);
+  const double rl = fmax(exact ? ceil(rmin - 1e-7) : floor(rmin - 1e-7), -1.0);
+  const double rh = fmin(exact ? floor(rmax + 1e-7) : ceil(rmax + 1e-7), (double)nr);
   c0 = max((int)cl, 0);
   c1 = min((int)ch, nc - 1);
   r0 = max((int)rl, 0);
