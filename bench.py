@@ -347,7 +347,9 @@ def run_ours(args, rank, world, local_rank):
     total_ms = start.elapsed_time(end)
     fwd_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(args.steps)]
     back_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(args.steps)]
-    total_ms, fwd_avg, back_avg = aggregate_over_ranks([total_ms, np.mean(fwd_ms), np.mean(back_ms)], world, dev)
+    (total_ms, fwd_avg, back_avg, fwd_med, back_med, fwd_min, back_min) = aggregate_over_ranks(
+        [total_ms, np.mean(fwd_ms), np.mean(back_ms), np.median(fwd_ms), np.median(back_ms), np.min(fwd_ms),
+         np.min(back_ms)], world, dev)
     ms_per_step = total_ms / args.steps
     value = throughput(2 * U, world, ms_per_step)
 
@@ -385,11 +387,11 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None, "dtype": "f32 (fp64 ray setup)", "data": "synthetic",
         "config": workload_config(wl),
         "updates_per_direction": U,
-        "forward": {"ms": fwd_avg, "gupdates_s": U / (fwd_avg * 1e-3) / 1e9,
+        "forward": {"ms": fwd_avg, "ms_median": fwd_med, "ms_min": fwd_min, "gupdates_s": U / (fwd_avg * 1e-3) / 1e9,
                     "views_s": g.n_views / (fwd_avg * 1e-3),
                     "effective_gbs": B / (fwd_avg * 1e-3) / 1e9,
                     "frac_of_hbm": B / (fwd_avg * 1e-3) / 1e9 / peak},
-        "back": {"ms": back_avg, "gupdates_s": U / (back_avg * 1e-3) / 1e9,
+        "back": {"ms": back_avg, "ms_median": back_med, "ms_min": back_min, "gupdates_s": U / (back_avg * 1e-3) / 1e9,
                  "views_s": g.n_views / (back_avg * 1e-3),
                  "effective_gbs": B / (back_avg * 1e-3) / 1e9,
                  "frac_of_hbm": B / (back_avg * 1e-3) / 1e9 / peak,
