@@ -137,17 +137,18 @@ __device__ __forceinline__ float crossing_sums(bool active, const Walk& W, const
       kmax = span_plain;
     }
     if (!active) d = 1 << 30;  // s = k - d stays negative: never inside [0, Na]
+    float fs = -(float)d;      // s as a float, counted (exact for active lanes)
     const float L = W.L;
     const float fNb = (float)Nb, fNc = (float)Nc;
     float tb = Nb > 0 ? l0b : CUDART_INF_F, tc = Nc > 0 ? l0c : CUDART_INF_F;
     float fjb = 1.f, fjc = 1.f, cur = 0.f;
     if (!__any_sync(kFull, active && Nc > 0)) {
 #pragma unroll kGradUnroll2
-      for (int k = 0; k <= kmax; ++k) {
+      for (int k = 0; k <= kmax; ++k, fs += 1.f) {
         const int s = k - d;
         const bool on = (unsigned)s <= (unsigned)Na;
         const bool ona = (unsigned)s < (unsigned)Na;  // a major plane ends this slab
-        const float tx = ona ? fminf(fmaf((float)s, inca, l0a), L) : L;
+        const float tx = ona ? fminf(fmaf(fs, inca, l0a), L) : L;
         const bool cb = on && tb < tx;
         const float m1 = fmaxf(fminf(tb, tx), cur);
         const Off o2 = off + (cb ? sb : (Off)0);
@@ -173,11 +174,11 @@ __device__ __forceinline__ float crossing_sums(bool active, const Walk& W, const
       }
     } else {
 #pragma unroll kGradUnroll3
-      for (int k = 0; k <= kmax; ++k) {
+      for (int k = 0; k <= kmax; ++k, fs += 1.f) {
         const int s = k - d;
         const bool on = (unsigned)s <= (unsigned)Na;
         const bool ona = (unsigned)s < (unsigned)Na;
-        const float tx = ona ? fminf(fmaf((float)s, inca, l0a), L) : L;
+        const float tx = ona ? fminf(fmaf(fs, inca, l0a), L) : L;
         const bool cb = on && tb < tx, cc = on && tc < tx;
         const bool bfirst = tb <= tc;
         const float m1 = fmaxf(fminf(fminf(tb, tc), tx), cur);

@@ -63,6 +63,8 @@ constexpr int kBackThreads = 256;
 #define CTP_BACK_STAGE 64
 #endif
 constexpr int kBackStage = CTP_BACK_STAGE;  // views per fixed-point accumulation stage of the adjoint
+constexpr float kRoundBias = 12582912.0f;   // 1.5 * 2^23
+constexpr int kRoundBiasBits = 0x4B400000;  // its bit pattern
 
 // FP32 Siddon walk in major-axis slabs, one lane per ray (lanes run
 // independently).  Each slab between two successive planes of the major axis
@@ -92,9 +94,10 @@ __device__ __forceinline__ void walk_lane(const Walk& W, Off off, Off s0, Off s1
   float fjb = 1.f;
   float cur = 0.f;
   if (Nc == 0) {
+    float fs = 0.f;  // s as a float, counted rather than converted each slab
 #pragma unroll kLaneWalk2Unroll
-    for (int s = 0; s < Na; ++s) {
-      const float tx = fminf(fmaf((float)s, inca, l0a), L);
+    for (int s = 0; s < Na; ++s, fs += 1.f) {
+      const float tx = fminf(fmaf(fs, inca, l0a), L);
       const bool cb = tb < tx;
       const float m1 = fmaxf(fminf(tb, tx), cur);
       const Off o2 = off + (cb ? sb : (Off)0);
@@ -112,9 +115,10 @@ __device__ __forceinline__ void walk_lane(const Walk& W, Off off, Off s0, Off s1
   } else {
     float tc = l0c;
     float fjc = 1.f;
+    float fs = 0.f;
 #pragma unroll kWalk3Unroll
-    for (int s = 0; s <= Na; ++s) {
-      const float tx = s < Na ? fminf(fmaf((float)s, inca, l0a), L) : L;
+    for (int s = 0; s <= Na; ++s, fs += 1.f) {
+      const float tx = s < Na ? fminf(fmaf(fs, inca, l0a), L) : L;
       const bool cb = tb < tx, cc = tc < tx;
       const float m1 = fmaxf(fminf(fminf(tb, tc), tx), cur);
       const float m2 = fmaxf(fminf(fmaxf(tb, tc), tx), m1);
@@ -162,11 +166,12 @@ __device__ __forceinline__ void walk_warp_bf(bool active, const Walk& W, Off off
   if (kmax < 0) return;
   float tb = Nb > 0 ? l0b : CUDART_INF_F;
   float fjb = 1.f, cur = 0.f;
+  float fs = 0.f;  // s as a float, counted rather than converted each slab
   if (!__any_sync(kFull, active && Nc > 0)) {
 #pragma unroll kLaneWalk2Unroll
-    for (int s = 0; s <= kmax; ++s) {
+    for (int s = 0; s <= kmax; ++s, fs += 1.f) {
       const bool on = s <= Na;
-      const float tx = fminf(fmaf((float)s, inca, l0a), L);
+      const float tx = fminf(fmaf(fs, inca, l0a), L);
       const bool cb = tb < tx;
       const float m1 = fmaxf(fminf(tb, tx), cur);
       const Off o2 = off + (cb ? sb : (Off)0);
@@ -183,9 +188,9 @@ __device__ __forceinline__ void walk_warp_bf(bool active, const Walk& W, Off off
     float tc = Nc > 0 ? l0c : CUDART_INF_F;
     float fjc = 1.f;
 #pragma unroll kWalk3Unroll
-    for (int s = 0; s <= kmax; ++s) {
+    for (int s = 0; s <= kmax; ++s, fs += 1.f) {
       const bool on = s <= Na;
-      const float tx = fminf(fmaf((float)s, inca, l0a), L);
+      const float tx = fminf(fmaf(fs, inca, l0a), L);
       const bool cb = tb < tx, cc = tc < tx;
       const float m1 = fmaxf(fminf(fminf(tb, tc), tx), cur);
       const float m2 = fmaxf(fminf(fmaxf(tb, tc), tx), m1);
@@ -261,6 +266,9 @@ __device__ __forceinline__ void walk(bool active, const Walk& W, const int lo[3]
     else d = 0;
   }
   if (!active) d = 1 << 30;  // s = k - d stays negative: never inside [0, Na]
+  // s = k - d as a float, counted rather than converted each slab (exact for
+  // the active lanes, whose |s| stays far below 2^24)
+  float fs = -(float)d;
 
   const float L = W.L;
   const float fNb = (float)Nb, fNc = (float)Nc;
@@ -270,12 +278,12 @@ __device__ __forceinline__ void walk(bool active, const Walk& W, const int lo[3]
   if (!__any_sync(kFull, active && Nc > 0)) {
     // no lane crosses a second minor axis: at most two segments per slab
 #pragma unroll kWalk2Unroll
-    for (int k = 0; k <= kmax; ++k) {
+    for (int k = 0; k <= kmax; ++k, fs += 1.f) {
       const int s = k - d;
       const bool on = (unsigned)s <= (unsigned)Na;
       // the (Na+1)-th major crossing lies at or past the exit: clamping to L
       // ends the last slab there (to within rounding of the walk length)
-      const float tx = fminf(fmaf((float)s, inca, l0a), L);
+      const float tx = fminf(fmaf(fs, inca, l0a), L);
       const bool cb = on && tb < tx;
       const float m1 = fmaxf(fminf(tb, tx), cur);
       if (kUniform) {
@@ -299,10 +307,10 @@ __device__ __forceinline__ void walk(bool active, const Walk& W, const int lo[3]
     float tc = Nc > 0 ? l0c : CUDART_INF_F;
     float fjc = 1.f;
 #pragma unroll kWalk3Unroll
-    for (int k = 0; k <= kmax; ++k) {
+    for (int k = 0; k <= kmax; ++k, fs += 1.f) {
       const int s = k - d;
       const bool on = (unsigned)s <= (unsigned)Na;
-      const float tx = fminf(fmaf((float)s, inca, l0a), L);
+      const float tx = fminf(fmaf(fs, inca, l0a), L);
       const bool cb = on && tb < tx, cc = on && tc < tx;
       const float m1 = fmaxf(fminf(fminf(tb, tc), tx), cur);
       const float m2 = fmaxf(fminf(fmaxf(tb, tc), tx), m1);
@@ -589,6 +597,7 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
   __shared__ unsigned int s_ymax_bits;
   __shared__ long long s_nsum;
   __shared__ float s_scale;
+  __shared__ int s_fast_round;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int b = blockIdx.x;
@@ -690,17 +699,25 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
     if (tid == 0) {
       const unsigned int bits = s_ymax_bits;
       float sc = 0.f;
+      s_fast_round = 0;
       if (bits >= 0x7f800000u) {
         sc = CUDART_NAN_F;  // non-finite input: the brick is written as NaN
       } else {
         const double seg_max = kPower == 2 ? diag * diag : diag;
-        const double bound = (double)__uint_as_float(bits) * seg_max * (double)s_nsum;
-        if (bound > 0.0) sc = (float)((2147483647.0 - 4194304.0) / bound);
+        const double one = (double)__uint_as_float(bits) * seg_max;  // largest single contribution / S
+        const double bound = one * (double)s_nsum;
+        if (bound > 0.0) {
+          sc = (float)((2147483647.0 - 4194304.0) / bound);
+          // one contribution below 4.0e6 < 2^22: the FMA rounding's range
+          // (the margin covers segments a few FP32 ulps over the diagonal)
+          s_fast_round = (double)sc * one < 4.0e6 ? 1 : 0;
+        }
       }
       s_scale = sc;
     }
     __syncthreads();
     const float S = s_scale;
+    const bool fast_round = s_fast_round != 0;
     // pass 2: walk every ray of the stage through the brick.  Each warp takes
     // 32 consecutive footprint rays (parallel beams: in mirror order, rays
     // with similar chords through the brick), sets them up together and
@@ -740,15 +757,27 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
           off = ((W.i[2] - lo[2]) * P.brick[1] + (W.i[1] - lo[1])) * pitch + (W.i[0] - lo[0]);
         }
         const float yS = y * S;
-        auto visit = [&](int o, float len) { atomicAdd(acc + o, __float2int_rn(coef<kPower>(len) * yS)); };
+        // Round coef * yS to the nearest integer.  Where the stage's scale
+        // keeps every contribution below 4.0e6 (< 2^22), one FMA does it:
+        // adding 1.5 * 2^23 leaves the integer in the low mantissa bits.
+        // Elsewhere (few rays per voxel, a finer scale) a conversion does.
+        auto visit_fma = [&](int o, float len) {
+          atomicAdd(acc + o, __float_as_int(fmaf(coef<kPower>(len), yS, kRoundBias)) - kRoundBiasBits);
+        };
+        auto visit_cvt = [&](int o, float len) { atomicAdd(acc + o, __float2int_rn(coef<kPower>(len) * yS)); };
         // measured on B200: parallel rays (mirror-ordered, near-equal chords)
         // walk fastest with independent lane loops, cone rays with the
         // warp-uniform trip count
         if (P.dims.beam == CTP_BEAM_PARALLEL) {
-          if (act) walk_lane<int>(W, off, W.step[0], W.step[1] * pitch, W.step[2] * plane, visit);
+          if (act) {
+            if (fast_round) walk_lane<int>(W, off, W.step[0], W.step[1] * pitch, W.step[2] * plane, visit_fma);
+            else walk_lane<int>(W, off, W.step[0], W.step[1] * pitch, W.step[2] * plane, visit_cvt);
+          }
           __syncwarp();
+        } else if (fast_round) {
+          walk_warp_bf<int>(act, W, off, W.step[0], W.step[1] * pitch, W.step[2] * plane, visit_fma);
         } else {
-          walk_warp_bf<int>(act, W, off, W.step[0], W.step[1] * pitch, W.step[2] * plane, visit);
+          walk_warp_bf<int>(act, W, off, W.step[0], W.step[1] * pitch, W.step[2] * plane, visit_cvt);
         }
       }
     }
