@@ -754,30 +754,36 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
         int off = 0;
         if (act) {
           entry(R, t_in, t_out, lo, hi, W);
-          off = ((W.i[2] - lo[2]) * P.brick[1] + (W.i[1] - lo[1])) * pitch + (W.i[0] - lo[0]);
+          // byte offset into the accumulators: the shared atomics then
+          // address [offset + constant] with no scaling per segment
+          off = 4 * (((W.i[2] - lo[2]) * P.brick[1] + (W.i[1] - lo[1])) * pitch + (W.i[0] - lo[0]));
         }
         const float yS = y * S;
         // Round coef * yS to the nearest integer.  Where the stage's scale
         // keeps every contribution below 4.0e6 (< 2^22), one FMA does it:
         // adding 1.5 * 2^23 leaves the integer in the low mantissa bits.
         // Elsewhere (few rays per voxel, a finer scale) a conversion does.
+        char* const accb = reinterpret_cast<char*>(acc);
         auto visit_fma = [&](int o, float len) {
-          atomicAdd(acc + o, __float_as_int(fmaf(coef<kPower>(len), yS, kRoundBias)) - kRoundBiasBits);
+          atomicAdd(reinterpret_cast<int*>(accb + o),
+                    __float_as_int(fmaf(coef<kPower>(len), yS, kRoundBias)) - kRoundBiasBits);
         };
-        auto visit_cvt = [&](int o, float len) { atomicAdd(acc + o, __float2int_rn(coef<kPower>(len) * yS)); };
+        auto visit_cvt = [&](int o, float len) {
+          atomicAdd(reinterpret_cast<int*>(accb + o), __float2int_rn(coef<kPower>(len) * yS));
+        };
         // measured on B200: parallel rays (mirror-ordered, near-equal chords)
         // walk fastest with independent lane loops, cone rays with the
         // warp-uniform trip count
         if (P.dims.beam == CTP_BEAM_PARALLEL) {
           if (act) {
-            if (fast_round) walk_lane<int>(W, off, W.step[0], W.step[1] * pitch, W.step[2] * plane, visit_fma);
-            else walk_lane<int>(W, off, W.step[0], W.step[1] * pitch, W.step[2] * plane, visit_cvt);
+            if (fast_round) walk_lane<int>(W, off, 4 * W.step[0], 4 * W.step[1] * pitch, 4 * W.step[2] * plane, visit_fma);
+            else walk_lane<int>(W, off, 4 * W.step[0], 4 * W.step[1] * pitch, 4 * W.step[2] * plane, visit_cvt);
           }
           __syncwarp();
         } else if (fast_round) {
-          walk_warp_bf<int>(act, W, off, W.step[0], W.step[1] * pitch, W.step[2] * plane, visit_fma);
+          walk_warp_bf<int>(act, W, off, 4 * W.step[0], 4 * W.step[1] * pitch, 4 * W.step[2] * plane, visit_fma);
         } else {
-          walk_warp_bf<int>(act, W, off, W.step[0], W.step[1] * pitch, W.step[2] * plane, visit_cvt);
+          walk_warp_bf<int>(act, W, off, 4 * W.step[0], 4 * W.step[1] * pitch, 4 * W.step[2] * plane, visit_cvt);
         }
       }
     }
