@@ -211,7 +211,9 @@ ctp_status ctp_back_power(const ctp_geom *geom, const float *sino, float *vol, i
  * sino_grad: device pointer, float32 [n_views][n_rows][n_cols], read only.
  * grad:      device pointer, float64 [n_views][4][3], overwritten (zeroed,
  *            then accumulated; contents are undefined if the call fails).
- * Flat detectors only: a cylindrical detector gives CTP_ERR_UNSUPPORTED.
+ * Flat and cylindrical detectors (for the cylindrical one, the derivatives
+ * of its pixel formula with respect to all four vectors, whose orthogonality
+ * constraints are not imposed on the gradient).
  * Asynchronous on `stream`; summation order across blocks is not fixed, so
  * results can differ between calls in the last bits.
  */

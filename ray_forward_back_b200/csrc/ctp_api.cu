@@ -713,8 +713,6 @@ ctp_status ctp_geometry_gradient(const ctp_geom *g, const float *vol, const floa
                                  void *stream) {
   g_detail[0] = '\0';
   if (!g) return fail(CTP_ERR_INVALID_ARGUMENT, "geometry is NULL");
-  if (g->det != CTP_DET_FLAT)
-    return fail(CTP_ERR_UNSUPPORTED, "geometry gradients are available for flat detectors only");
   DeviceGuard dg(g->device);
   if (dg.err != cudaSuccess) return cuda_fail(dg.err, "cudaSetDevice");
   if (!is_device_pointer(vol, g->device) || !is_device_pointer(sino_grad, g->device) ||

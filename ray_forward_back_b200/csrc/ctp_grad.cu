@@ -32,7 +32,8 @@
 //
 // A flat detector's pixel (r, c) sits at det_c + (c - cc) det_u + (r - rc)
 // det_v with (rc, cc) the detector's centre, so the pixel gradient also
-// gives the det_c, det_u and det_v gradients.  Kinks (a ray through a voxel
+// gives the det_c, det_u and det_v gradients; a cylindrical detector's pixel
+// is a nonlinear function of the four vectors (cylinder_chain below).  Kinks (a ray through a voxel
 // edge, an endpoint on a plane) have no derivative; the formula then returns
 // one of the one-sided values.
 //
@@ -224,7 +225,55 @@ __device__ __forceinline__ float crossing_sums(bool active, const Walk& W, const
   return xe;
 }
 
-template <typename Off>
+// Cylindrical detector: the pixel gradient G (already weighted) carried to
+// the view's vectors.  With a = det_c - src, v^ = det_v / |det_v|,
+// alpha = a.v^, w = a - alpha v^, R = |w|, w^ = w / R, u^ = det_u / |det_u|,
+// gamma = (c - cc) |det_u| / R and rho = r - rc, the pixel is
+//   p = src + alpha v^ + R (cos gamma w^ + sin gamma u^) + rho det_v.
+// With t = -sin gamma w^ + cos gamma u^ (the unit tangent at the pixel),
+// h = (sin gamma u^ - gamma t).G and P = I - v^ v^T:
+//   dL/d det_c = (v^.G) v^ + cos gamma P G + h w^
+//   dL/d src   = (source endpoint gradient) + G - dL/d det_c
+//   dL/d det_u = (R gamma / |det_u|) (t.G) u^ + (R sin gamma / |det_u|) (G - (u^.G) u^)
+//   dL/d det_v = P X / |det_v| + rho G,
+//     X = (1 - cos gamma) ((v^.G) a + alpha G) - alpha h w^.
+// (Derivatives of the unconstrained formula above, the one the projector
+// evaluates; the view record holds u^, w^, v^, R, |det_u| / R and alpha.)
+__device__ __forceinline__ void cylinder_chain(const ViewRec& V, const double* __restrict__ trig, const Dims& dm,
+                                               int v, int c, double rho, const double gsrc[3], const double G[3],
+                                               double out[12]) {
+  const size_t ti = 2 * ((size_t)v * dm.n_cols + c);
+  const double cg = trig[ti], sg = trig[ti + 1];
+  const double gam = V.gam0 + (double)c * V.dgam;
+  const double alpha = V.axial0 + 0.5 * (double)(dm.n_rows - 1) * V.vlen;  // (det_c - src).v^
+  double t[3], a[3], vG = 0.0, uG = 0.0, tG = 0.0, hG = 0.0;
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    t[k] = cg * V.du[k] - sg * V.w[k];
+    a[k] = alpha * V.vhat[k] + V.R * V.w[k];
+    vG = fma(V.vhat[k], G[k], vG);
+    uG = fma(V.du[k], G[k], uG);
+    tG = fma(t[k], G[k], tG);
+  }
+  hG = sg * uG - gam * tG;
+  double X[3], vX = 0.0;
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    X[k] = (1.0 - cg) * (vG * a[k] + alpha * G[k]) - alpha * hG * V.w[k];
+    vX = fma(V.vhat[k], X[k], vX);
+  }
+  const double inv_dgam = 1.0 / V.dgam;  // R / |det_u|
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    const double ga = vG * V.vhat[k] + cg * (G[k] - vG * V.vhat[k]) + hG * V.w[k];
+    out[k] = gsrc[k] + G[k] - ga;
+    out[3 + k] = ga;
+    out[6 + k] = inv_dgam * (gam * tG * V.du[k] + sg * (G[k] - uG * V.du[k]));
+    out[9 + k] = (X[k] - vX * V.vhat[k]) / V.vlen + rho * G[k];
+  }
+}
+
+template <typename Off, bool kCyl>
 __global__ void __launch_bounds__(kGradThreads, CTP_GRAD_MIN_BLOCKS) geometry_gradient_kernel(FwdLaunch P,
                                                                          const ViewRec* __restrict__ views,
                                                                          const double* __restrict__ trig,
@@ -333,12 +382,16 @@ __global__ void __launch_bounds__(kGradThreads, CTP_GRAD_MIN_BLOCKS) geometry_gr
   const double cu = (double)c - 0.5 * (double)(P.dims.n_cols - 1);
   const double rv = (double)r - 0.5 * (double)(P.dims.n_rows - 1);
   double acc[12];
+  if (!kCyl) {
 #pragma unroll
-  for (int k = 0; k < 3; ++k) {
-    acc[k] = gs[k];
-    acc[3 + k] = gp[k];
-    acc[6 + k] = cu * gp[k];
-    acc[9 + k] = rv * gp[k];
+    for (int k = 0; k < 3; ++k) {
+      acc[k] = gs[k];
+      acc[3 + k] = gp[k];
+      acc[6 + k] = cu * gp[k];
+      acc[9 + k] = rv * gp[k];
+    }
+  } else {
+    cylinder_chain(V, trig, P.dims, v, valid ? c : 0, rv, gs, gp, acc);
   }
   // block reduction: warps by shuffles, then one warp over the 8 warp sums
   __shared__ double part[kGradThreads / 32][12];
@@ -369,10 +422,15 @@ cudaError_t launch_geometry_gradient(const FwdLaunch& p, const ViewRec* views, c
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   dim3 block(kGradCols, kGradRows);
-  if (wide_index)
-    geometry_gradient_kernel<long long><<<(unsigned)blocks, block, 0, stream>>>(p, views, trig, vol, volT, gsino, grad);
-  else
-    geometry_gradient_kernel<int><<<(unsigned)blocks, block, 0, stream>>>(p, views, trig, vol, volT, gsino, grad);
+  const unsigned nb = (unsigned)blocks;
+  const bool cyl = p.dims.det != CTP_DET_FLAT;
+  if (wide_index) {
+    if (cyl) geometry_gradient_kernel<long long, true><<<nb, block, 0, stream>>>(p, views, trig, vol, volT, gsino, grad);
+    else geometry_gradient_kernel<long long, false><<<nb, block, 0, stream>>>(p, views, trig, vol, volT, gsino, grad);
+  } else {
+    if (cyl) geometry_gradient_kernel<int, true><<<nb, block, 0, stream>>>(p, views, trig, vol, volT, gsino, grad);
+    else geometry_gradient_kernel<int, false><<<nb, block, 0, stream>>>(p, views, trig, vol, volT, gsino, grad);
+  }
   return cudaGetLastError();
 }
 
