@@ -8,7 +8,7 @@ resident in HBM.  value = (forward updates + back updates) / step time, in
 Gupdates/s (ray-voxel updates), summed over ranks; with N > 1 every rank runs
 its own copy of the workload (independent problems, weak scaling, no
 collective on the data path).  Rank 0 prints one JSON line.  The geometry
-gradient (flat detectors) is timed on its own after the step and reported
+gradient is timed on its own after the step and reported
 under "geometry_gradient"; it is not part of the step.
 
 --impl reference times the FP64 CPU oracle on a bounded sample of the same
@@ -357,9 +357,9 @@ def run_ours(args, rank, world, local_rank):
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, P, g, wl, vol_host, U, world, dev)
-    # geometry gradients (flat detectors): timed on their own after the step
+    # geometry gradients: timed on their own after the step
     grad = None
-    if not args.no_extras and g.detector == W.DET_FLAT:
+    if not args.no_extras:
         grad = time_geometry_gradient(args, P, g, vol, sino_in, stream, U, world, dev)
     if rank != 0:
         return 0
