@@ -63,6 +63,8 @@ constexpr int kBackThreads = 256;
 #define CTP_BACK_STAGE 64
 #endif
 constexpr int kBackStage = CTP_BACK_STAGE;  // views per fixed-point accumulation stage of the adjoint
+constexpr int kSortWin = 2048;     // parallel adjoint: rays per length-sorted window
+constexpr int kSortBuckets = 32;   // chord-length classes of the counting sort
 constexpr float kRoundBias = 12582912.0f;   // 1.5 * 2^23
 constexpr int kRoundBiasBits = 0x4B400000;  // its bit pattern
 
@@ -465,7 +467,7 @@ __device__ __forceinline__ int mirror_order(int t, int w) { return (t & 1) ? w -
 // Computed by one warp (lanes 0-7 project the eight corners); all lanes
 // return the result.
 __device__ void brick_footprint(const ViewRec& V, const BackLaunch& P, const int lo[3], const int hi[3], int lane,
-                                int& c0, int& c1, int& r0, int& r1, int& nvox) {
+                                int& c0, int& c1, int& r0, int& r1, int& nvox, float ucol[4]) {
   const int nc = P.dims.n_cols, nr = P.dims.n_rows;
   if (V.full_footprint) {
     c0 = 0, c1 = nc - 1, r0 = 0, r1 = nr - 1;
@@ -485,6 +487,25 @@ __device__ void brick_footprint(const ViewRec& V, const BackLaunch& P, const int
     const double d[3] = {X[0] - V.p00[0], X[1] - V.p00[1], X[2] - V.p00[2]};
     cmin = cmax = V.minv[0] * d[0] + V.minv[1] * d[1] + V.minv[2] * d[2];
     rmin = rmax = V.minv[3] * d[0] + V.minv[4] * d[1] + V.minv[5] * d[2];
+    // sort the eight corner columns across the lanes of each group of 8
+    // (bitonic); a brick whose chord depends on the column alone (rays and
+    // columns in z-planes) has the chord profile of a trapezoid with corners
+    // at sorted positions 0, 2, 5, 7 (each column appears twice)
+    float u = (float)cmin;
+#pragma unroll
+    for (int k = 2; k <= 8; k <<= 1) {
+#pragma unroll
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        const float o = __shfl_xor_sync(0xffffffffu, u, j);
+        const bool up = (q & k) == 0, low = (q & j) == 0;
+        u = (low == up) ? fminf(u, o) : fmaxf(u, o);
+      }
+    }
+    const int g0 = lane & ~7;
+    ucol[0] = __shfl_sync(0xffffffffu, u, g0);
+    ucol[1] = __shfl_sync(0xffffffffu, u, g0 + 2);
+    ucol[2] = __shfl_sync(0xffffffffu, u, g0 + 5);
+    ucol[3] = __shfl_sync(0xffffffffu, u, g0 + 7);
   } else if (P.dims.det == CTP_DET_FLAT) {
     const double d[3] = {X[0] - V.s[0], X[1] - V.s[1], X[2] - V.s[2]};
     const double lam = V.minv[0] * d[0] + V.minv[1] * d[1] + V.minv[2] * d[2];
@@ -586,7 +607,7 @@ __device__ void brick_footprint(const ViewRec& V, const BackLaunch& P, const int
 // summed per-view ray bounds.  Each stage is then flushed into the FP32
 // volume.  Integer sums are exact, so the result does not depend on the
 // order in which threads add.
-template <int kPower, typename Off>
+template <int kPower, typename Off, bool kParallel>
 __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
     back_brick_kernel(BackLaunch P, const ViewRec* __restrict__ views, const double* __restrict__ trig,
                       const float* __restrict__ sino, float* __restrict__ vol) {
@@ -594,6 +615,11 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
   // per staged view: first column, first row, width, footprint size, ray bound
   __shared__ int fc0[kBackStage], fr0[kBackStage], fw[kBackStage], cnt[kBackStage], nvb[kBackStage];
   __shared__ int pre[kBackStage + 1];
+  // parallel beams: per staged view, the chord trapezoid's outer columns and
+  // inverse ramp widths; the length-sorted order of one window of rays
+  __shared__ float fu0[kBackStage], fu3[kBackStage], firl[kBackStage], firr[kBackStage];
+  __shared__ unsigned short sched[kSortWin];
+  __shared__ int hist[kSortBuckets];
   __shared__ unsigned int s_ymax_bits;
   __shared__ long long s_nsum;
   __shared__ float s_scale;
@@ -629,8 +655,13 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
     __syncthreads();  // previous stage flushed (and accumulators zeroed)
     for (int s = warp; s < nvs; s += kBackThreads / 32) {
       int c0 = 0, c1 = -1, r0 = 0, r1 = -1, nv = 0;
-      brick_footprint(views[vb + s], P, lo, hi, lane, c0, c1, r0, r1, nv);
+      float uc[4] = {0.f, 0.f, 0.f, 0.f};
+      brick_footprint(views[vb + s], P, lo, hi, lane, c0, c1, r0, r1, nv, uc);
       if (lane == 0) {
+        fu0[s] = uc[0];
+        fu3[s] = uc[3];
+        firl[s] = uc[1] > uc[0] ? 1.f / (uc[1] - uc[0]) : 1e30f;
+        firr[s] = uc[3] > uc[2] ? 1.f / (uc[3] - uc[2]) : 1e30f;
         const int w = c1 >= c0 ? c1 - c0 + 1 : 0;
         const int h = r1 >= r0 ? r1 - r0 + 1 : 0;
         fc0[s] = c0;
@@ -718,72 +749,129 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
     __syncthreads();
     const float S = s_scale;
     const bool fast_round = s_fast_round != 0;
-    // pass 2: walk every ray of the stage through the brick.  Each warp takes
-    // 32 consecutive footprint rays (parallel beams: in mirror order, rays
-    // with similar chords through the brick), sets them up together and
-    // reconverges before the next 32.
-    if (S > 0.f) {
-      for (int q0 = warp * 32; q0 < total; q0 += kBackThreads) {
-        const int q = q0 + lane;
-        bool act = q < total;
-        int v = vb, r = 0, c = 0;
-        float y = 0.f;
+    // pass 2: walk every ray of the stage through the brick.  A warp takes
+    // 32 footprint rays, sets them up together and reconverges before the
+    // next 32.  Footprint ray q of the stage: view vb + sl, then row-major in
+    // its footprint rectangle; parallel beams take each row in mirror order
+    // (0, w-1, 1, w-2, ...).
+    auto locate = [&](int q, int& sl, int& r, int& c) {
+      int sh = nvs;
+      sl = 0;
+      while (sh - sl > 1) {
+        const int mid = (sl + sh) >> 1;
+        if (pre[mid] <= q) sl = mid;
+        else sh = mid;
+      }
+      const int qq = q - pre[sl];
+      const int w = fw[sl];
+      const int rr = qq / w;
+      r = fr0[sl] + rr;
+      c = fc0[sl] + (kParallel ? mirror_order(qq - rr * w, w) : qq - rr * w);
+    };
+    char* const accb = reinterpret_cast<char*>(acc);
+    // Set up and walk one ray per lane (all 32 lanes call this together;
+    // lanes without a ray pass valid = false).
+    auto process = [&](int q, bool valid) {
+      bool act = valid;
+      int v = vb, r = 0, c = 0;
+      float y = 0.f;
+      if (act) {
+        int sl;
+        locate(q, sl, r, c);
+        v = vb + sl;
+        y = __ldg(sino + ((size_t)v * nr + r) * nc + c);
+        act = y != 0.f;
+      }
+      Ray R;
+      double t_in = 0.0, t_out = 0.0;
+      if (act) {
+        make_ray(views[v], P.vol, trig, P.dims, v, r, c, R);
+        act = clip(R, lo, hi, t_in, t_out);
+      }
+      Walk W = {};
+      int off = 0;
+      if (act) {
+        entry(R, t_in, t_out, lo, hi, W);
+        // byte offset into the accumulators: the shared atomics then
+        // address [offset + constant] with no scaling per segment
+        off = 4 * (((W.i[2] - lo[2]) * P.brick[1] + (W.i[1] - lo[1])) * pitch + (W.i[0] - lo[0]));
+      }
+      const float yS = y * S;
+      // Round coef * yS to the nearest integer.  Where the stage's scale
+      // keeps every contribution below 4.0e6 (< 2^22), one FMA does it:
+      // adding 1.5 * 2^23 leaves the integer in the low mantissa bits.
+      // Elsewhere (few rays per voxel, a finer scale) a conversion does.
+      auto visit_fma = [&](int o, float len) {
+        atomicAdd(reinterpret_cast<int*>(accb + o),
+                  __float_as_int(fmaf(coef<kPower>(len), yS, kRoundBias)) - kRoundBiasBits);
+      };
+      auto visit_cvt = [&](int o, float len) {
+        atomicAdd(reinterpret_cast<int*>(accb + o), __float2int_rn(coef<kPower>(len) * yS));
+      };
+      // measured on B200: parallel rays (length-sorted, near-equal chords)
+      // walk fastest with independent lane loops, cone rays with the
+      // warp-uniform trip count
+      if (kParallel) {
         if (act) {
-          int sl = 0, sh = nvs;
-          while (sh - sl > 1) {
-            const int mid = (sl + sh) >> 1;
-            if (pre[mid] <= q) sl = mid;
-            else sh = mid;
+          if (fast_round) walk_lane<int>(W, off, 4 * W.step[0], 4 * W.step[1] * pitch, 4 * W.step[2] * plane, visit_fma);
+          else walk_lane<int>(W, off, 4 * W.step[0], 4 * W.step[1] * pitch, 4 * W.step[2] * plane, visit_cvt);
+        }
+        __syncwarp();
+      } else if (fast_round) {
+        walk_warp_bf<int>(act, W, off, 4 * W.step[0], 4 * W.step[1] * pitch, 4 * W.step[2] * plane, visit_fma);
+      } else {
+        walk_warp_bf<int>(act, W, off, 4 * W.step[0], 4 * W.step[1] * pitch, 4 * W.step[2] * plane, visit_cvt);
+      }
+    };
+    if (S > 0.f && !kParallel) {
+      for (int q0 = warp * 32; q0 < total; q0 += kBackThreads) process(q0 + lane, q0 + lane < total);
+    } else if (S > 0.f) {
+      // Parallel beams: windows of kSortWin rays, counting-sorted by the
+      // chord estimated from the view's trapezoid, so that the 32 lanes of
+      // a warp walk rays of near-equal length (chunks of consecutive rays
+      // of one view span a ramp of the trapezoid).
+      for (int w0 = 0; w0 < total; w0 += kSortWin) {
+        const int nwin = min(kSortWin, total - w0);
+        __syncthreads();  // the previous window's schedule is consumed
+        if (tid < kSortBuckets) hist[tid] = 0;
+        __syncthreads();
+        constexpr int kPer = kSortWin / kBackThreads;  // 8 rays per thread, buckets packed 4 to a word
+        static_assert(kPer == 8 && kSortBuckets <= 256, "bucket packing");
+        unsigned int bk[2] = {0u, 0u};
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+          const int i = tid + j * kBackThreads;
+          if (i < nwin) {
+            int sl, r, c;
+            locate(w0 + i, sl, r, c);
+            const float fc = (float)c;
+            const float e = fminf(fminf((fc - fu0[sl]) * firl[sl], (fu3[sl] - fc) * firr[sl]), 1.f);
+            const unsigned int b = (unsigned int)(fmaxf(e, 0.f) * (kSortBuckets - 0.5f));
+            bk[j >> 2] |= b << (8 * (j & 3));
+            atomicAdd(&hist[b], 1);
           }
-          const int qq = q - pre[sl];
-          const int w = fw[sl];
-          const int rr = qq / w;
-          r = fr0[sl] + rr;
-          c = fc0[sl] + (P.dims.beam == CTP_BEAM_PARALLEL ? mirror_order(qq - rr * w, w) : qq - rr * w);
-          v = vb + sl;
-          y = __ldg(sino + ((size_t)v * nr + r) * nc + c);
-          act = y != 0.f;
         }
-        Ray R;
-        double t_in = 0.0, t_out = 0.0;
-        if (act) {
-          make_ray(views[v], P.vol, trig, P.dims, v, r, c, R);
-          act = clip(R, lo, hi, t_in, t_out);
-        }
-        Walk W = {};
-        int off = 0;
-        if (act) {
-          entry(R, t_in, t_out, lo, hi, W);
-          // byte offset into the accumulators: the shared atomics then
-          // address [offset + constant] with no scaling per segment
-          off = 4 * (((W.i[2] - lo[2]) * P.brick[1] + (W.i[1] - lo[1])) * pitch + (W.i[0] - lo[0]));
-        }
-        const float yS = y * S;
-        // Round coef * yS to the nearest integer.  Where the stage's scale
-        // keeps every contribution below 4.0e6 (< 2^22), one FMA does it:
-        // adding 1.5 * 2^23 leaves the integer in the low mantissa bits.
-        // Elsewhere (few rays per voxel, a finer scale) a conversion does.
-        char* const accb = reinterpret_cast<char*>(acc);
-        auto visit_fma = [&](int o, float len) {
-          atomicAdd(reinterpret_cast<int*>(accb + o),
-                    __float_as_int(fmaf(coef<kPower>(len), yS, kRoundBias)) - kRoundBiasBits);
-        };
-        auto visit_cvt = [&](int o, float len) {
-          atomicAdd(reinterpret_cast<int*>(accb + o), __float2int_rn(coef<kPower>(len) * yS));
-        };
-        // measured on B200: parallel rays (mirror-ordered, near-equal chords)
-        // walk fastest with independent lane loops, cone rays with the
-        // warp-uniform trip count
-        if (P.dims.beam == CTP_BEAM_PARALLEL) {
-          if (act) {
-            if (fast_round) walk_lane<int>(W, off, 4 * W.step[0], 4 * W.step[1] * pitch, 4 * W.step[2] * plane, visit_fma);
-            else walk_lane<int>(W, off, 4 * W.step[0], 4 * W.step[1] * pitch, 4 * W.step[2] * plane, visit_cvt);
+        __syncthreads();
+        if (warp == 0) {  // exclusive scan of the bucket counts
+          const int n = hist[lane];
+          int incl = n;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
           }
-          __syncwarp();
-        } else if (fast_round) {
-          walk_warp_bf<int>(act, W, off, 4 * W.step[0], 4 * W.step[1] * pitch, 4 * W.step[2] * plane, visit_fma);
-        } else {
-          walk_warp_bf<int>(act, W, off, 4 * W.step[0], 4 * W.step[1] * pitch, 4 * W.step[2] * plane, visit_cvt);
+          hist[lane] = incl - n;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+          const int i = tid + j * kBackThreads;
+          if (i < nwin) sched[atomicAdd(&hist[(bk[j >> 2] >> (8 * (j & 3))) & 0xffu], 1)] = (unsigned short)i;
+        }
+        __syncthreads();
+        for (int j0 = warp * 32; j0 < nwin; j0 += kBackThreads) {
+          const bool ok = j0 + lane < nwin;
+          process(w0 + (ok ? (int)sched[j0 + lane] : 0), ok);
         }
       }
     }
@@ -1003,14 +1091,16 @@ size_t back_brick_smem_bytes(const int32_t brick[3]) {
 
 cudaError_t prepare_back_brick(size_t smem_bytes) {
   const int b = (int)smem_bytes;
-  cudaError_t e = cudaFuncSetAttribute(back_brick_kernel<1, int>, cudaFuncAttributeMaxDynamicSharedMemorySize, b);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(back_brick_kernel<1, long long>, cudaFuncAttributeMaxDynamicSharedMemorySize, b);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(back_brick_kernel<2, int>, cudaFuncAttributeMaxDynamicSharedMemorySize, b);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(back_brick_kernel<2, long long>, cudaFuncAttributeMaxDynamicSharedMemorySize, b);
-  return e;
+  const void* kernels[] = {
+      (const void*)back_brick_kernel<1, int, true>,  (const void*)back_brick_kernel<1, long long, true>,
+      (const void*)back_brick_kernel<2, int, true>,  (const void*)back_brick_kernel<2, long long, true>,
+      (const void*)back_brick_kernel<1, int, false>, (const void*)back_brick_kernel<1, long long, false>,
+      (const void*)back_brick_kernel<2, int, false>, (const void*)back_brick_kernel<2, long long, false>};
+  for (const void* k : kernels) {
+    const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, b);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t launch_back_brick(const BackLaunch& p, const ViewRec* views, const double* trig, const float* sino,
@@ -1022,13 +1112,23 @@ cudaError_t launch_back_brick(const BackLaunch& p, const ViewRec* views, const d
   cudaError_t e = prepare_back_brick(smem);
   if (e != cudaSuccess) return e;
   const unsigned nb = (unsigned)blocks;
+  const bool par = p.dims.beam == CTP_BEAM_PARALLEL;
+#define CTP_BACK_LAUNCH(KP, OFF, PAR) \
+  back_brick_kernel<KP, OFF, PAR><<<nb, kBackThreads, smem, stream>>>(p, views, trig, sino, vol)
   if (power == 2) {
-    if (wide_index) back_brick_kernel<2, long long><<<nb, kBackThreads, smem, stream>>>(p, views, trig, sino, vol);
-    else back_brick_kernel<2, int><<<nb, kBackThreads, smem, stream>>>(p, views, trig, sino, vol);
+    if (wide_index) {
+      if (par) CTP_BACK_LAUNCH(2, long long, true); else CTP_BACK_LAUNCH(2, long long, false);
+    } else {
+      if (par) CTP_BACK_LAUNCH(2, int, true); else CTP_BACK_LAUNCH(2, int, false);
+    }
   } else {
-    if (wide_index) back_brick_kernel<1, long long><<<nb, kBackThreads, smem, stream>>>(p, views, trig, sino, vol);
-    else back_brick_kernel<1, int><<<nb, kBackThreads, smem, stream>>>(p, views, trig, sino, vol);
+    if (wide_index) {
+      if (par) CTP_BACK_LAUNCH(1, long long, true); else CTP_BACK_LAUNCH(1, long long, false);
+    } else {
+      if (par) CTP_BACK_LAUNCH(1, int, true); else CTP_BACK_LAUNCH(1, int, false);
+    }
   }
+#undef CTP_BACK_LAUNCH
   return cudaGetLastError();
 }
 
