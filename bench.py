@@ -53,22 +53,33 @@ def workload_config(wl):
             "seed": wl.seed, "l2": "inputs larger than L2 (volume and sinogram each > 126 MB)"}
 
 
+def code_digest(paths):
+    """SHA-256 of the C++/CUDA code in `paths` with comments and whitespace
+    removed: edits to comments do not count as a change of the kernel."""
+    import hashlib
+    import re
+    h = hashlib.sha256()
+    for path in paths:
+        with open(os.path.join(ROOT, path)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(re.sub(r"\s+", "", text).encode())
+    return h.hexdigest()
+
+
 def measured_traffic(kernel, workload_index):
     """Per-launch DRAM bytes of `kernel` from the committed one-pass ncu
     capture, or None when the capture is for another workload or the kernel
-    source has changed since it was taken."""
-    import hashlib
+    code has changed since it was taken."""
     path = os.path.join(ROOT, "profiles", "dram_traffic_parallel512_900views.json")
     try:
         with open(path) as f:
             k = json.load(f)["kernels"][kernel]
-        h = hashlib.sha256()
-        for src in k["sources"]:
-            with open(os.path.join(ROOT, src), "rb") as f:
-                h.update(f.read())
+        digest = code_digest(k["sources"])
     except Exception:
         return None
-    if h.hexdigest() != k.get("sources_sha256") or workload_index != 4:
+    if digest != k.get("code_sha256") or workload_index != 4:
         return None
     return int(k["dram_bytes_per_launch"])
 

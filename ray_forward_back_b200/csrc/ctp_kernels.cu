@@ -22,13 +22,20 @@
 //                      lanes read neighbouring voxels, from an x-fastest or a
 //                      y-fastest copy of the volume, whichever the view's
 //                      column direction runs along; coalesced sinogram stores.
+//                      One walk can serve 1, 2 or 4 volumes of a batch.
 //   back_brick_kernel  one CTA owns a voxel brick in shared memory, visits every
-//                      ray of its view range that can cross the brick (detector
-//                      footprint of the brick per view), clips each ray to the
-//                      brick in FP64 (the per-tile entry of the pages), walks it
-//                      in FP32 with shared-memory atomics, and flushes the brick
-//                      once with coalesced stores (plain stores when the CTA
-//                      owns all views, red.global.add otherwise).
+//                      ray of its view range that can cross the brick (exact
+//                      detector footprint of the brick per view), clips each
+//                      ray to the brick in FP64 (the per-tile entry of the
+//                      pages), walks it in FP32 with int32 fixed-point
+//                      shared-memory atomics, and flushes the brick once per
+//                      stage with coalesced stores (plain stores when the CTA
+//                      owns all views, red.global.add otherwise).  Parallel
+//                      beams take each window of 2048 rays in order of
+//                      estimated chord length, so a warp's lanes finish
+//                      together; one instance per beam type.
+//   back_sort_kernel   the adjoint as a sorted segment reduction, for dense
+//                      ray-voxel collisions (and, counting, the collision ratio).
 //   count_kernel       the forward traversal counting positive-length segments.
 //   transpose_xy       x-fastest -> y-fastest copy of the volume.
 #include "ctp_ray.cuh"
@@ -453,10 +460,10 @@ __device__ __forceinline__ float coef(float len) {
 
 // Column of the t-th ray of a footprint row of width w taken from both ends
 // inwards (0, w-1, 1, w-2, ...).  With parallel rays a brick's chord profile
-// along a footprint row is a trapezoid symmetric about the row centre, so 32
-// consecutive rays in this order sit at two mirrored distances from the
-// centre and have nearly equal chords: the lanes of a warp finish their
-// walks together.  (Cone footprints are not symmetric; they keep plain order.)
+// along a footprint row is a trapezoid symmetric about the row centre, so
+// consecutive rays in this order come in pairs of equal chords.  (The length
+// sort of the parallel adjoint then groups rays across views; cone
+// footprints are not symmetric and keep plain order.)
 __device__ __forceinline__ int mirror_order(int t, int w) { return (t & 1) ? w - 1 - (t >> 1) : (t >> 1); }
 
 // Detector footprint of the brick [lo, hi) in view V: a rectangle of pixels
