@@ -12,7 +12,8 @@ gradient is timed on its own after the step and reported
 under "geometry_gradient"; it is not part of the step.
 
 --impl reference times the FP64 CPU oracle on a bounded sample of the same
-workload (the reference arm; slow by design).
+workload (the reference arm; slow by design).  --solver cgls|sirt prints the
+solvers' iteration time against one forward + back instead.
 """
 from __future__ import annotations
 
@@ -299,6 +300,64 @@ def time_geometry_gradient(args, P, g, vol, sino_grad, stream, U, world, dev):
             "launches_per_call": 1 + (1 if P.info()["n_transposed_views"] > 0 else 0)}
 
 
+def run_solver(args, rank, world, local_rank):
+    """Iteration time of the device solvers (ctp_solve) against one forward +
+    back projection of the same workload: every CGLS or SIRT iteration is one
+    forward and one adjoint plus a few vector kernels and one host read of
+    the step's norms.  Per-iteration time is the difference of two runs of
+    different lengths (so the set-up, e.g. SIRT's row and column sums, drops
+    out), CUDA events on the launching stream, max over ranks."""
+    import torch
+
+    from ray_forward_back_b200 import ctp
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = select_workload(args)
+    g = wl.geom
+    P = ctp.Projector(g, device=local_rank)
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        vol = torch.from_numpy(wl.phantom()).to(dev)
+        sino = P.forward(vol, stream=stream)   # consistent data: A x of the phantom
+        xo = torch.empty(g.vol_shape, dtype=torch.float32, device=dev)
+    stream.synchronize()
+    method = args.solver
+
+    def run(iters):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            P.solve(sino, method, iterations=iters, stream=stream)
+            e1.record(stream)
+        stream.synchronize()
+        return e0.elapsed_time(e1)
+
+    for _ in range(max(1, args.warmup)):
+        run(2)
+    short, long_ = run(2), run(2 + args.steps)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        P.forward(vol, out=sino, stream=stream)
+        P.back(sino, out=xo, stream=stream)
+    e1.record(stream)
+    stream.synchronize()
+    pair = e0.elapsed_time(e1) / args.steps
+    per_iter, short, pair = aggregate_over_ranks([(long_ - short) / args.steps, short, pair], world, dev)
+    if rank != 0:
+        return 0
+    line = {"metric": f"{method} iterations/s on one B200", "value": world * 1000.0 / per_iter,
+            "unit": "iterations/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_iteration": per_iter, "setup_ms": short - 2 * per_iter, "projector_pair_ms": pair,
+            "overhead_vs_pair": per_iter / pair - 1.0, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32 (fp64 ray setup, fp64 norms)", "data": "synthetic",
+            "config": workload_config(wl)}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -434,6 +493,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the geometry-gradient timing")
+    ap.add_argument("--solver", choices=["cgls", "sirt"], default=None,
+                    help="time solver iterations (against one forward + back) instead of the projector step")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -449,6 +510,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
+        if args.solver:
+            return run_solver(args, rank, world, local_rank)
         return run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
