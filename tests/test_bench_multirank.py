@@ -1,6 +1,7 @@
-"""The benchmark's multi-rank bookkeeping on two gloo ranks (CPU): every
-rank sees the slowest rank's timings and the whole-job throughput counts all
-ranks' work over that time."""
+"""The benchmark's bookkeeping on the CPU: on two gloo ranks every rank sees
+the slowest rank's timings and the whole-job throughput counts all ranks'
+work over that time; the digest that keys the committed DRAM-traffic
+capture ignores comments only."""
 import os
 import socket
 
@@ -46,3 +47,18 @@ def test_single_rank_is_identity():
     import bench
     assert bench.aggregate_over_ranks([1.5, 2.0], 1) == [1.5, 2.0]
     assert bench.throughput(1e9, 1, 1000.0) == pytest.approx(1.0)
+
+
+def test_code_digest_ignores_comments_and_whitespace_only(tmp_path, monkeypatch):
+    """The committed DRAM-traffic capture stays valid across comment edits of
+    the kernel sources and is voided by any change of code."""
+    import bench
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    a = tmp_path / "a.cu"
+    a.write_text("// header\\nint f(int x) {\\n  return x + 1;  /* add one */\\n}\\n")
+    d0 = bench.code_digest(["a.cu"])
+    a.write_text("// a longer header\\n/* block\\n comment */\\nint f(int x)   {\\n\\n  return x + 1;\\n}\\n")
+    assert bench.code_digest(["a.cu"]) == d0
+    a.write_text("int f(int x) {\\n  return x + 2;\\n}\\n")
+    assert bench.code_digest(["a.cu"]) != d0
+
