@@ -26,6 +26,7 @@ struct ctp_geom {
   ctp::Dims dims{};
   FwdLaunch fwd{};
   BackLaunch back{};
+  BackLaunch back2{};   // batched adjoint of member pairs: the brick halved along y (same shared memory)
   int adjoint_variant = CTP_ADJOINT_BRICK;
   int n_transposed = 0;
   double collision_ratio = 0.0;
@@ -324,6 +325,33 @@ ctp_status build_views(const ctp_geom_desc *d, std::vector<ViewRec> &views, std:
   return CTP_OK;
 }
 
+// Brick counts, shared-memory pitch and view groups of an adjoint launch
+// whose brick is already set (kb members share each CTA).
+void plan_back_groups(const ctp_geom *g, BackLaunch &p, const ctp_plan *plan, int sm_count, int kb) {
+  const int64_t n[3] = {g->nx, g->ny, g->nz};
+  int64_t nb = 1;
+  for (int k = 0; k < 3; ++k) {
+    p.nbrick[k] = (int)((n[k] + p.brick[k] - 1) / p.brick[k]);
+    nb *= p.nbrick[k];
+  }
+  p.pitch_x = p.brick[0] + 1;
+  // Resident CTAs per SM: shared memory (brick + staged footprints + the
+  // 1 KB the runtime reserves per CTA) and registers (three 256-thread CTAs).
+  const int64_t per_cta = (int64_t)ctp::back_brick_smem_bytes(p.brick, kb) + 6 * 1024;
+  const int64_t per_sm = std::max<int64_t>(1, std::min<int64_t>(3, (228 * 1024) / per_cta));
+  const int64_t slots = (int64_t)sm_count * per_sm;
+  // at least four waves of CTAs, so the last partial wave costs little:
+  // split the views over groups when there are too few bricks
+  int groups = 1;
+  if (nb < 4 * slots)
+    groups = (int)std::min<int64_t>((4 * slots + nb - 1) / nb, std::max<int64_t>(1, (g->n_views + 7) / 8));
+  if (plan && plan->view_groups > 0) groups = (int)std::min<int64_t>(plan->view_groups, g->n_views);
+  int vpg = (int)((g->n_views + groups - 1) / groups);
+  groups = (int)((g->n_views + vpg - 1) / vpg);
+  p.view_groups = groups;
+  p.views_per_group = vpg;
+}
+
 void plan_back(ctp_geom *g, const ctp_plan *plan, int sm_count) {
   int b[3];
   // measured on B200: flat, wide bricks amortise the per-ray FP64 entry best
@@ -340,28 +368,14 @@ void plan_back(ctp_geom *g, const ctp_plan *plan, int sm_count) {
   BackLaunch &p = g->back;
   p.dims = g->dims;
   p.vol = g->vol;
-  int64_t nb = 1;
-  for (int k = 0; k < 3; ++k) {
-    p.brick[k] = b[k];
-    p.nbrick[k] = (int)((n[k] + b[k] - 1) / b[k]);
-    nb *= p.nbrick[k];
-  }
-  p.pitch_x = b[0] + 1;
-  // Resident CTAs per SM: shared memory (brick + staged footprints + the
-  // 1 KB the runtime reserves per CTA) and registers (three 256-thread CTAs).
-  const int64_t per_cta = (int64_t)ctp::back_brick_smem_bytes(p.brick) + 6 * 1024;
-  const int64_t per_sm = std::max<int64_t>(1, std::min<int64_t>(3, (228 * 1024) / per_cta));
-  const int64_t slots = (int64_t)sm_count * per_sm;
-  // at least four waves of CTAs, so the last partial wave costs little:
-  // split the views over groups when there are too few bricks
-  int groups = 1;
-  if (nb < 4 * slots)
-    groups = (int)std::min<int64_t>((4 * slots + nb - 1) / nb, std::max<int64_t>(1, (g->n_views + 7) / 8));
-  if (plan && plan->view_groups > 0) groups = (int)std::min<int64_t>(plan->view_groups, g->n_views);
-  int vpg = (int)((g->n_views + groups - 1) / groups);
-  groups = (int)((g->n_views + vpg - 1) / vpg);
-  p.view_groups = groups;
-  p.views_per_group = vpg;
+  for (int k = 0; k < 3; ++k) p.brick[k] = b[k];
+  plan_back_groups(g, p, plan, sm_count, 1);
+  // member pairs: half the brick along y, so two accumulators fit the same
+  // shared memory as one
+  BackLaunch &p2 = g->back2;
+  p2 = p;
+  p2.brick[1] = (b[1] + 1) / 2;
+  plan_back_groups(g, p2, plan, sm_count, 2);
 }
 
 bool is_device_pointer(const void *ptr, int device) {
@@ -565,6 +579,8 @@ ctp_status ctp_geom_create(const ctp_geom_desc *desc, ctp_geom **out) {
     if (e == cudaSuccess && !trig.empty())
       e = cudaMemcpy(g->d_trig, trig.data(), sizeof(double) * trig.size(), cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = ctp::prepare_back_brick(ctp::back_brick_smem_bytes(g->back.brick));
+    if (e == cudaSuccess && g->batch_chunk >= 2)
+      e = ctp::prepare_back_brick(ctp::back_brick_smem_bytes(g->back2.brick, 2), 2);
     if (e != cudaSuccess) st = cuda_fail(e, "geometry upload");
   }
   if (st == CTP_OK) st = measure_collision_ratio(g, views, trig, &g->collision_ratio);
@@ -672,7 +688,28 @@ ctp_status ctp_back_batch(const ctp_geom *g, const float *sino, float *vol, int6
   if (!g) return fail(CTP_ERR_INVALID_ARGUMENT, "geometry is NULL");
   ctp_status st = check_batch(g, n_batch);
   if (st != CTP_OK || n_batch == 0) return st;
-  for (int64_t b = 0; b < n_batch; ++b) {
+  int64_t b = 0;
+  if (g->batch_chunk >= 2 && g->adjoint_variant == CTP_ADJOINT_BRICK && n_batch >= 2) {
+    // member pairs share each ray's set-up and walk (one launch per pair)
+    DeviceGuard dg(g->device);
+    if (dg.err != cudaSuccess) return cuda_fail(dg.err, "cudaSetDevice");
+    if (!is_device_pointer(sino, g->device))
+      return fail(CTP_ERR_INVALID_ARGUMENT, "sino is not device memory of device %d", g->device);
+    if (!is_device_pointer(vol, g->device))
+      return fail(CTP_ERR_INVALID_ARGUMENT, "vol is not device memory of device %d", g->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "pending error before ctp_back_batch");
+    for (; b + 2 <= n_batch; b += 2) {
+      float *v0 = vol + (size_t)b * (size_t)g->n_vox;
+      if (g->back2.view_groups > 1) e = cudaMemsetAsync(v0, 0, 2 * sizeof(float) * (size_t)g->n_vox, s);
+      if (e == cudaSuccess)
+        e = ctp::launch_back_brick(g->back2, g->d_views, g->d_trig, sino + (size_t)b * (size_t)g->n_rays, v0, 1, 2,
+                                   g->wide_index, s);
+      if (e != cudaSuccess) return cuda_fail(e, "batched adjoint launch");
+    }
+  }
+  for (; b < n_batch; ++b) {
     st = ctp_back_power(g, sino + (size_t)b * (size_t)g->n_rays, vol + (size_t)b * (size_t)g->n_vox, 1, stream);
     if (st != CTP_OK) return st;
   }
@@ -704,7 +741,7 @@ ctp_status ctp_back_power(const ctp_geom *g, const float *sino, float *vol, int 
   if (sorted)
     e = ctp::launch_back_sort(g->fwd, g->d_views, g->d_trig, sino, vol, power, g->wide_index, s);
   else
-    e = ctp::launch_back_brick(g->back, g->d_views, g->d_trig, sino, vol, power, g->wide_index, s);
+    e = ctp::launch_back_brick(g->back, g->d_views, g->d_trig, sino, vol, power, 1, g->wide_index, s);
   if (e != cudaSuccess) return cuda_fail(e, "adjoint launch");
   return CTP_OK;
 }

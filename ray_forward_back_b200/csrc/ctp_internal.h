@@ -74,15 +74,17 @@ cudaError_t launch_transpose_xy(const float* vol, float* volT, const VolDesc& vd
 // copies at volT, volT + n_vox, ...) into kb sinograms at sino, sino + n_rays, ...
 cudaError_t launch_forward(const FwdLaunch& p, const ViewRec* views, const double* trig, const float* vol,
                            const float* volT, float* sino, int kb, bool wide_index, cudaStream_t stream);
+// Brick adjoint of kb (1 or 2) batch members: sinograms at sino, sino + n_rays,
+// volumes at vol, vol + n_vox.
 cudaError_t launch_back_brick(const BackLaunch& p, const ViewRec* views, const double* trig, const float* sino,
-                              float* vol, int power, bool wide_index, cudaStream_t stream);
+                              float* vol, int power, int kb, bool wide_index, cudaStream_t stream);
 cudaError_t launch_count(const FwdLaunch& p, const ViewRec* views, const double* trig,
                          unsigned long long* counter, cudaStream_t stream);
 cudaError_t launch_back_sort(const FwdLaunch& p, const ViewRec* views, const double* trig, const float* sino,
                              float* vol, int power, bool wide_index, cudaStream_t stream);
 cudaError_t launch_collision_count(const FwdLaunch& p, const ViewRec* views, const double* trig,
                                    unsigned long long* counters, bool wide_index, cudaStream_t stream);
-size_t back_brick_smem_bytes(const int32_t brick[3]);
+size_t back_brick_smem_bytes(const int32_t brick[3], int kb = 1);
 cudaError_t launch_geometry_gradient(const FwdLaunch& p, const ViewRec* views, const double* trig, const float* vol,
                                      const float* volT, const float* gsino, double* grad, bool wide_index,
                                      cudaStream_t stream);
@@ -94,6 +96,6 @@ ctp_status host_error(ctp_status s, const char* msg);
 ctp_status host_cuda_error(cudaError_t e, const char* where);
 bool host_is_device_pointer(const void* ptr, int device);
 void host_clear_error();
-cudaError_t prepare_back_brick(size_t smem_bytes);
+cudaError_t prepare_back_brick(size_t smem_bytes, int kb = 1);
 
 }  // namespace ctp

@@ -614,7 +614,11 @@ __device__ void brick_footprint(const ViewRec& V, const BackLaunch& P, const int
 // summed per-view ray bounds.  Each stage is then flushed into the FP32
 // volume.  Integer sums are exact, so the result does not depend on the
 // order in which threads add.
-template <int kPower, typename Off, bool kParallel>
+// kB members of a batch (1 or 2) share each ray's set-up and walk: member m
+// reads sino + m * n_rays, accumulates in its own brick of fixed-point
+// counters (acc + m * n_acc) with its own per-stage scale, and writes
+// vol + m * n_vox.
+template <int kPower, typename Off, bool kParallel, int kB>
 __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
     back_brick_kernel(BackLaunch P, const ViewRec* __restrict__ views, const double* __restrict__ trig,
                       const float* __restrict__ sino, float* __restrict__ vol) {
@@ -627,9 +631,9 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
   __shared__ float fu0[kBackStage], fu3[kBackStage], firl[kBackStage], firr[kBackStage];
   __shared__ unsigned short sched[kSortWin];
   __shared__ int hist[kSortBuckets];
-  __shared__ unsigned int s_ymax_bits;
+  __shared__ unsigned int s_ymax_bits[kB];
   __shared__ long long s_nsum;
-  __shared__ float s_scale;
+  __shared__ float s_scale[kB];
   __shared__ int s_fast_round;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -646,7 +650,9 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
   const int pitch = P.pitch_x;
   const int plane = pitch * P.brick[1];
   const int n_acc = plane * P.brick[2];
-  for (int i = tid; i < n_acc; i += kBackThreads) acc[i] = 0;
+  for (int i = tid; i < kB * n_acc; i += kBackThreads) acc[i] = 0;
+  const size_t n_rays = (size_t)P.dims.n_views * P.dims.n_rows * P.dims.n_cols;
+  const size_t n_vox = (size_t)P.vol.n[0] * P.vol.n[1] * P.vol.n[2];
   const double diag = sqrt(P.vol.spacing[0] * P.vol.spacing[0] + P.vol.spacing[1] * P.vol.spacing[1] +
                            P.vol.spacing[2] * P.vol.spacing[2]);
   const int ex = hi[0] - lo[0], ey = hi[1] - lo[1], ez = hi[2] - lo[2];
@@ -678,7 +684,7 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
         nvb[s] = w * h > 0 ? nv : 0;
       }
     }
-    if (tid == 0) s_ymax_bits = 0u;
+    if (tid < kB) s_ymax_bits[tid] = 0u;
     __syncthreads();
     if (warp == 0) {
       // exclusive scan of cnt[0..nvs) and the sum of the ray bounds
@@ -716,7 +722,9 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
     // pass 1: largest |y| of the stage's footprint rays (NaN and inf sort
     // above every finite value as unsigned bit patterns)
     {
-      unsigned int mb = 0u;
+      unsigned int mb[kB];
+#pragma unroll
+      for (int m = 0; m < kB; ++m) mb[m] = 0u;
       for (int q = tid; q < total; q += kBackThreads) {
         int sl = 0, sh = nvs;
         while (sh - sl > 1) {
@@ -727,34 +735,49 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
         const int qq = q - pre[sl];
         const int rr = qq / fw[sl];
         const int r = fr0[sl] + rr, c = fc0[sl] + (qq - rr * fw[sl]);
-        mb = max(mb, __float_as_uint(fabsf(__ldg(sino + ((size_t)(vb + sl) * nr + r) * nc + c))));
+        const size_t i = ((size_t)(vb + sl) * nr + r) * nc + c;
+#pragma unroll
+        for (int m = 0; m < kB; ++m) mb[m] = max(mb[m], __float_as_uint(fabsf(__ldg(sino + m * n_rays + i))));
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
-      if (lane == 0 && mb) atomicMax(&s_ymax_bits, mb);
+      for (int m = 0; m < kB; ++m) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mb[m] = max(mb[m], __shfl_xor_sync(0xffffffffu, mb[m], o));
+        if (lane == 0 && mb[m]) atomicMax(&s_ymax_bits[m], mb[m]);
+      }
     }
     __syncthreads();
     if (tid == 0) {
-      const unsigned int bits = s_ymax_bits;
-      float sc = 0.f;
-      s_fast_round = 0;
-      if (bits >= 0x7f800000u) {
-        sc = CUDART_NAN_F;  // non-finite input: the brick is written as NaN
-      } else {
-        const double seg_max = kPower == 2 ? diag * diag : diag;
-        const double one = (double)__uint_as_float(bits) * seg_max;  // largest single contribution / S
-        const double bound = one * (double)s_nsum;
-        if (bound > 0.0) {
-          sc = (float)((2147483647.0 - 4194304.0) / bound);
-          // one contribution below 4.0e6 < 2^22: the FMA rounding's range
-          // (the margin covers segments a few FP32 ulps over the diagonal)
-          s_fast_round = (double)sc * one < 4.0e6 ? 1 : 0;
+      int fast = 1;
+#pragma unroll
+      for (int m = 0; m < kB; ++m) {
+        const unsigned int bits = s_ymax_bits[m];
+        float sc = 0.f;
+        if (bits >= 0x7f800000u) {
+          sc = CUDART_NAN_F;  // non-finite input: the brick is written as NaN
+        } else {
+          const double seg_max = kPower == 2 ? diag * diag : diag;
+          const double one = (double)__uint_as_float(bits) * seg_max;  // largest single contribution / S
+          const double bound = one * (double)s_nsum;
+          if (bound > 0.0) {
+            sc = (float)((2147483647.0 - 4194304.0) / bound);
+            // one contribution below 4.0e6 < 2^22: the FMA rounding's range
+            // (the margin covers segments a few FP32 ulps over the diagonal)
+            if (!((double)sc * one < 4.0e6)) fast = 0;
+          }
         }
+        s_scale[m] = sc;
       }
-      s_scale = sc;
+      s_fast_round = fast;
     }
     __syncthreads();
-    const float S = s_scale;
+    float S[kB];
+    bool any_walk = false;
+#pragma unroll
+    for (int m = 0; m < kB; ++m) {
+      S[m] = s_scale[m];
+      any_walk |= S[m] > 0.f;
+    }
     const bool fast_round = s_fast_round != 0;
     // pass 2: walk every ray of the stage through the brick.  A warp takes
     // 32 footprint rays, sets them up together and reconverges before the
@@ -781,13 +804,22 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
     auto process = [&](int q, bool valid) {
       bool act = valid;
       int v = vb, r = 0, c = 0;
-      float y = 0.f;
+      float y[kB];
+#pragma unroll
+      for (int m = 0; m < kB; ++m) y[m] = 0.f;
       if (act) {
         int sl;
         locate(q, sl, r, c);
         v = vb + sl;
-        y = __ldg(sino + ((size_t)v * nr + r) * nc + c);
-        act = y != 0.f;
+        const size_t i = ((size_t)v * nr + r) * nc + c;
+        act = false;
+#pragma unroll
+        for (int m = 0; m < kB; ++m) {
+          // a member whose stage scale is 0 or NaN adds nothing (its brick
+          // is all zero, or written as NaN, at the flush)
+          y[m] = S[m] > 0.f ? __ldg(sino + m * n_rays + i) : 0.f;
+          act |= y[m] != 0.f;
+        }
       }
       Ray R;
       double t_in = 0.0, t_out = 0.0;
@@ -803,17 +835,26 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
         // address [offset + constant] with no scaling per segment
         off = 4 * (((W.i[2] - lo[2]) * P.brick[1] + (W.i[1] - lo[1])) * pitch + (W.i[0] - lo[0]));
       }
-      const float yS = y * S;
+      float yS[kB];
+#pragma unroll
+      for (int m = 0; m < kB; ++m) yS[m] = y[m] * S[m];
       // Round coef * yS to the nearest integer.  Where the stage's scale
       // keeps every contribution below 4.0e6 (< 2^22), one FMA does it:
       // adding 1.5 * 2^23 leaves the integer in the low mantissa bits.
       // Elsewhere (few rays per voxel, a finer scale) a conversion does.
+      const int mbytes = 4 * n_acc;  // byte distance between the members' bricks
       auto visit_fma = [&](int o, float len) {
-        atomicAdd(reinterpret_cast<int*>(accb + o),
-                  __float_as_int(fmaf(coef<kPower>(len), yS, kRoundBias)) - kRoundBiasBits);
+        const float w = coef<kPower>(len);
+#pragma unroll
+        for (int m = 0; m < kB; ++m)
+          atomicAdd(reinterpret_cast<int*>(accb + m * mbytes + o),
+                    __float_as_int(fmaf(w, yS[m], kRoundBias)) - kRoundBiasBits);
       };
       auto visit_cvt = [&](int o, float len) {
-        atomicAdd(reinterpret_cast<int*>(accb + o), __float2int_rn(coef<kPower>(len) * yS));
+        const float w = coef<kPower>(len);
+#pragma unroll
+        for (int m = 0; m < kB; ++m)
+          atomicAdd(reinterpret_cast<int*>(accb + m * mbytes + o), __float2int_rn(w * yS[m]));
       };
       // measured on B200: parallel rays (length-sorted, near-equal chords)
       // walk fastest with independent lane loops, cone rays with the
@@ -830,9 +871,9 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
         walk_warp_bf<int>(act, W, off, 4 * W.step[0], 4 * W.step[1] * pitch, 4 * W.step[2] * plane, visit_cvt);
       }
     };
-    if (S > 0.f && !kParallel) {
+    if (any_walk && !kParallel) {
       for (int q0 = warp * 32; q0 < total; q0 += kBackThreads) process(q0 + lane, q0 + lane < total);
-    } else if (S > 0.f) {
+    } else if (any_walk) {
       // Parallel beams: windows of kSortWin rays, counting-sorted by the
       // chord estimated from the view's trapezoid, so that the 32 lanes of
       // a warp walk rays of near-equal length (chunks of consecutive rays
@@ -884,23 +925,29 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
     }
     __syncthreads();
     // flush the stage into the volume and clear the accumulators
-    const bool nan_stage = S != S;
-    const float inv = S > 0.f ? 1.f / S : 0.f;
+    float inv[kB];
+#pragma unroll
+    for (int m = 0; m < kB; ++m) inv[m] = S[m] > 0.f ? 1.f / S[m] : 0.f;
     for (int i = tid; i < n_out; i += kBackThreads) {
       const int x = i % ex;
       const int t = i / ex;
       const int yy = t % ey;
       const int z = t / ey;
       const int ai = (z * P.brick[1] + yy) * pitch + x;
-      const float val = nan_stage ? CUDART_NAN_F : (float)acc[ai] * inv;
-      acc[ai] = 0;
       const Off gi = ((Off)(lo[2] + z) * ny + (Off)(lo[1] + yy)) * nx + (Off)(lo[0] + x);
-      if (P.view_groups > 1) {
-        if (val != 0.f) atomicAdd(vol + gi, val);
-      } else if (first) {
-        vol[gi] = val;
-      } else {
-        vol[gi] += val;
+#pragma unroll
+      for (int m = 0; m < kB; ++m) {
+        const bool nan_stage = S[m] != S[m];
+        const float val = nan_stage ? CUDART_NAN_F : (float)acc[m * n_acc + ai] * inv[m];
+        acc[m * n_acc + ai] = 0;
+        float* const vm = vol + m * n_vox;
+        if (P.view_groups > 1) {
+          if (val != 0.f) atomicAdd(vm + gi, val);
+        } else if (first) {
+          vm[gi] = val;
+        } else {
+          vm[gi] += val;
+        }
       }
     }
     first = false;
@@ -1092,36 +1139,31 @@ cudaError_t launch_collision_count(const FwdLaunch& p, const ViewRec* views, con
   return cudaGetLastError();
 }
 
-size_t back_brick_smem_bytes(const int32_t brick[3]) {
-  return sizeof(int) * (size_t)(brick[0] + 1) * brick[1] * brick[2];
+size_t back_brick_smem_bytes(const int32_t brick[3], int kb) {
+  return sizeof(int) * (size_t)kb * (size_t)(brick[0] + 1) * brick[1] * brick[2];
 }
 
-cudaError_t prepare_back_brick(size_t smem_bytes) {
-  const int b = (int)smem_bytes;
+namespace {
+template <int kB>
+cudaError_t set_back_smem(int bytes) {
   const void* kernels[] = {
-      (const void*)back_brick_kernel<1, int, true>,  (const void*)back_brick_kernel<1, long long, true>,
-      (const void*)back_brick_kernel<2, int, true>,  (const void*)back_brick_kernel<2, long long, true>,
-      (const void*)back_brick_kernel<1, int, false>, (const void*)back_brick_kernel<1, long long, false>,
-      (const void*)back_brick_kernel<2, int, false>, (const void*)back_brick_kernel<2, long long, false>};
+      (const void*)back_brick_kernel<1, int, true, kB>,  (const void*)back_brick_kernel<1, long long, true, kB>,
+      (const void*)back_brick_kernel<2, int, true, kB>,  (const void*)back_brick_kernel<2, long long, true, kB>,
+      (const void*)back_brick_kernel<1, int, false, kB>, (const void*)back_brick_kernel<1, long long, false, kB>,
+      (const void*)back_brick_kernel<2, int, false, kB>, (const void*)back_brick_kernel<2, long long, false, kB>};
   for (const void* k : kernels) {
-    const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, b);
+    const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
 }
 
-cudaError_t launch_back_brick(const BackLaunch& p, const ViewRec* views, const double* trig, const float* sino,
-                              float* vol, int power, bool wide_index, cudaStream_t stream) {
-  const long long blocks = (long long)p.nbrick[0] * p.nbrick[1] * p.nbrick[2] * p.view_groups;
-  if (blocks <= 0) return cudaSuccess;
-  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  const size_t smem = back_brick_smem_bytes(p.brick);
-  cudaError_t e = prepare_back_brick(smem);
-  if (e != cudaSuccess) return e;
-  const unsigned nb = (unsigned)blocks;
+template <int kB>
+void launch_back_brick_kb(const BackLaunch& p, const ViewRec* views, const double* trig, const float* sino,
+                          float* vol, int power, bool wide_index, unsigned nb, size_t smem, cudaStream_t stream) {
   const bool par = p.dims.beam == CTP_BEAM_PARALLEL;
 #define CTP_BACK_LAUNCH(KP, OFF, PAR) \
-  back_brick_kernel<KP, OFF, PAR><<<nb, kBackThreads, smem, stream>>>(p, views, trig, sino, vol)
+  back_brick_kernel<KP, OFF, PAR, kB><<<nb, kBackThreads, smem, stream>>>(p, views, trig, sino, vol)
   if (power == 2) {
     if (wide_index) {
       if (par) CTP_BACK_LAUNCH(2, long long, true); else CTP_BACK_LAUNCH(2, long long, false);
@@ -1136,6 +1178,24 @@ cudaError_t launch_back_brick(const BackLaunch& p, const ViewRec* views, const d
     }
   }
 #undef CTP_BACK_LAUNCH
+}
+}  // namespace
+
+cudaError_t prepare_back_brick(size_t smem_bytes, int kb) {
+  return kb == 2 ? set_back_smem<2>((int)smem_bytes) : set_back_smem<1>((int)smem_bytes);
+}
+
+cudaError_t launch_back_brick(const BackLaunch& p, const ViewRec* views, const double* trig, const float* sino,
+                              float* vol, int power, int kb, bool wide_index, cudaStream_t stream) {
+  if (kb != 1 && kb != 2) return cudaErrorInvalidValue;
+  const long long blocks = (long long)p.nbrick[0] * p.nbrick[1] * p.nbrick[2] * p.view_groups;
+  if (blocks <= 0) return cudaSuccess;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  const size_t smem = back_brick_smem_bytes(p.brick, kb);
+  cudaError_t e = prepare_back_brick(smem, kb);
+  if (e != cudaSuccess) return e;
+  if (kb == 2) launch_back_brick_kb<2>(p, views, trig, sino, vol, power, wide_index, (unsigned)blocks, smem, stream);
+  else launch_back_brick_kb<1>(p, views, trig, sino, vol, power, wide_index, (unsigned)blocks, smem, stream);
   return cudaGetLastError();
 }
 

@@ -93,3 +93,45 @@ def test_scratch_grows_with_the_chunk_only_when_views_are_transposed():
     x_only = projector(g, plan={"batch_chunk": 4, "forward_layout": 1}).info()
     assert x_only["n_transposed_views"] == 0
     assert x_only["scratch_bytes"] < one["scratch_bytes"]
+
+
+@pytest.mark.parametrize("name", ["parallel_both_layouts", "cone_flat", "helical_cyl"])
+@pytest.mark.parametrize("chunk,n", [(2, 2), (2, 3), (4, 5)])
+def test_fused_batched_back_meets_the_oracle(name, chunk, n):
+    """plan.batch_chunk >= 2: member pairs share each ray's walk in one
+    launch (a brick half as deep in y, two fixed-point accumulators).  Each
+    member meets the oracle's tolerances and agrees with its single call to
+    FP32 accumulation (the two use different bricks, hence different
+    fixed-point scales); an odd last member runs alone."""
+    import torch
+    from tests.gpu_helpers import check_back
+    g = _geoms()[name]
+    P = projector(g, plan={"batch_chunk": chunk})
+    rng = np.random.default_rng(7)
+    sino = rng.random((n,) + tuple(g.sino_shape)).astype(np.float32)
+    x = P.back(torch.from_numpy(sino).cuda()).cpu().numpy()
+    local_len = float(np.linalg.norm(np.array(P.info()["brick"]) * np.array(g.spacing)))
+    for b in range(n):
+        ref = oracle.back(g, sino[b])
+        check_back(x[b], ref, oracle.back(g, sino[b], power=0), local_len, f"{name} member {b}")
+        single = P.back(torch.from_numpy(sino[b]).cuda()).cpu().numpy()
+        np.testing.assert_allclose(x[b], single, rtol=1e-5, atol=1e-6 * np.abs(single).max())
+
+
+def test_fused_batched_back_keeps_members_apart():
+    """A non-finite value in one member reaches only that member's voxels; an
+    all-zero member gives exactly zero."""
+    import torch
+    g = _geoms()["parallel_both_layouts"]
+    P = projector(g, plan={"batch_chunk": 2})
+    rng = np.random.default_rng(8)
+    sino = rng.random((2,) + tuple(g.sino_shape)).astype(np.float32)
+    sino[0, 3, 2, 10] = np.nan
+    x = P.back(torch.from_numpy(sino).cuda()).cpu().numpy()
+    assert np.isnan(x[0]).any()
+    single = P.back(torch.from_numpy(sino[1]).cuda()).cpu().numpy()
+    assert np.isfinite(x[1]).all()
+    np.testing.assert_allclose(x[1], single, rtol=1e-5, atol=1e-6 * np.abs(single).max())
+    sino[0] = 0.0
+    x = P.back(torch.from_numpy(sino).cuda()).cpu().numpy()
+    assert np.count_nonzero(x[0]) == 0 and np.isfinite(x[1]).all()
