@@ -84,7 +84,8 @@ typedef struct {
   int32_t view_groups;       /* adjoint: split the views over this many CTA groups; 0 = automatic */
   int32_t forward_layout;    /* 0 = automatic per view, 1 = always x-fastest volume, 2 = always y-fastest */
   int32_t batch_chunk;       /* ctp_forward_batch: volumes per fused launch, 1, 2 or 4; 0 = 1.  The
-                                y-fastest scratch copy (if any view uses it) grows by this factor. */
+                                y-fastest scratch copy (if any view uses it) grows by this factor.
+                                2 or 4 also lets ctp_back_batch take member pairs in one launch. */
   int32_t reserved[9];
 } ctp_plan;
 
@@ -170,13 +171,17 @@ ctp_status ctp_back(const ctp_geom *geom, const float *sino, float *vol, void *s
  * (sinograms) that share one geometry, laid out one after the other:
  *   vol:  device pointer, float32 [n_batch][nz][ny][nx]
  *   sino: device pointer, float32 [n_batch][n_views][n_rows][n_cols]
- * Member b's output is exactly what ctp_forward / ctp_back give for member b
+ * Member b's forward output is exactly what ctp_forward gives for member b
  * alone (leading batch dimensions are preserved, diffct "Execution", section
  * "Batch dimensions and axis spacing"; empty batches included: n_batch = 0
  * does nothing and returns CTP_OK without looking at the pointers).
  * The forward walks every ray once per chunk of plan.batch_chunk members and
  * gathers from all of them, so the per-ray set-up and walk control are shared
- * across the chunk; the adjoint runs member by member.  n_batch < 0, or a
+ * across the chunk; each member's sinogram is bit-identical to ctp_forward's.
+ * With plan.batch_chunk >= 2 the brick adjoint takes member pairs in one
+ * launch (its brick halved along y); their volumes then differ from
+ * ctp_back's by fixed-point rounding only.  Otherwise, and for the sort
+ * adjoint, it runs member by member.  n_batch < 0, or a
  * batch whose element count exceeds 2^62, gives CTP_ERR_INVALID_ARGUMENT.
  * Same pointer, stream and synchronisation rules as ctp_forward / ctp_back.
  */
