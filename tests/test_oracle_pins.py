@@ -347,10 +347,13 @@ def test_fd_geometry_gradient_matches_rectangle_chord_slope():
     a trapezoid in q; shifting det_c along the detector's column direction by
     e moves the ray by e, so dy/d(det_c . u_hat) is the trapezoid's slope,
     computed from the rectangle's edge lines (closed form), and shifting
-    det_c along the ray direction changes nothing."""
+    det_c along the ray direction changes nothing.  The levers of det_u and
+    det_v (the pixel's column and row offsets) and the turn of the ray about
+    its pixel under a tilt of the direction follow from the same closed form."""
     from oracle.geometry_grad import geometry_gradient_fd
     theta = 0.41
-    g = _box_geom(theta)
+    pitch = 3.9   # columns 0, 1, 7, 8 fall on the ramps of the 20 x 30 rectangle's chord profile
+    g = _box_geom(theta, pitch=pitch)
     vol = np.ones(g.vol_shape, np.float32)
     Wd, Hd = g.nx * g.spacing[0], g.ny * g.spacing[1]
     d = np.array([math.cos(theta), math.sin(theta)])
@@ -362,11 +365,32 @@ def test_fd_geometry_gradient_matches_rectangle_chord_slope():
         us = sorted([(-Hd / 2 - p[1]) / d[1], (Hd / 2 - p[1]) / d[1]])
         return max(0.0, min(ts[1], us[1]) - max(ts[0], us[0]))
 
-    for c in (0, 2, 6, 8):   # rays on the sloped part of the trapezoid
-        q = (c - (g.n_cols - 1) / 2) * 0.77
+    def chord_line(p, u):
+        """Chord of the line p + t u (u any length) through the rectangle."""
+        u = u / np.hypot(u[0], u[1])
+        ts = sorted([(-Wd / 2 - p[0]) / u[0], (Wd / 2 - p[0]) / u[0]])
+        us = sorted([(-Hd / 2 - p[1]) / u[1], (Hd / 2 - p[1]) / u[1]])
+        return max(0.0, min(ts[1], us[1]) - max(ts[0], us[0]))
+
+    n3 = np.array([n[0], n[1], 0.0])
+    for c in (0, 1, 7, 8):   # rays on the sloped part of the trapezoid
+        lever = c - (g.n_cols - 1) / 2
+        q = lever * pitch
         slope = (chord(q + 1e-4) - chord(q - 1e-4)) / 2e-4
+        assert abs(slope) > 0.5   # a ramp, so every check below has a nonzero target
         up = np.zeros(g.sino_shape)
         up[0, 1, c] = 1.0
         grad = geometry_gradient_fd(g, vol, up)
-        assert grad[0, 1] @ np.array([n[0], n[1], 0.0]) == pytest.approx(slope, rel=1e-6, abs=1e-7)
+        assert grad[0, 1] @ n3 == pytest.approx(slope, rel=1e-6, abs=1e-7)
         assert grad[0, 1] @ np.array([d[0], d[1], 0.0]) == pytest.approx(0.0, abs=1e-6)
+        # det_u moves column c by (c - cc) times the step; det_v moves row 1,
+        # the middle row, not at all
+        assert grad[0, 2] @ n3 == pytest.approx(lever * slope, rel=1e-6, abs=1e-6)
+        assert grad[0, 3] @ n3 == pytest.approx(0.0, abs=1e-6)
+        # tilting the direction turns the ray about its pixel
+        turn = (chord_line(q * n, d + 1e-5 * n) - chord_line(q * n, d - 1e-5 * n)) / 2e-5
+        assert grad[0, 0] @ n3 == pytest.approx(turn, rel=1e-5, abs=1e-6)
+        # the bottom row (r = 0) moves with det_v by -1 times the step
+        up = np.zeros(g.sino_shape)
+        up[0, 0, c] = 1.0
+        assert geometry_gradient_fd(g, vol, up)[0, 3] @ n3 == pytest.approx(-slope, rel=1e-6, abs=1e-6)
