@@ -102,3 +102,20 @@ def test_sirt_nonnegativity_and_relaxation():
     xa, _, _ = solvers.sirt(A, y, 1, relaxation=1.0, nonnegative=False)
     xb, _, _ = solvers.sirt(A, y, 1, relaxation=0.5, nonnegative=False)
     np.testing.assert_allclose(xb, 0.5 * xa, atol=1e-14)
+
+
+def test_sirt_clamp_is_the_projection_onto_nonnegative_values():
+    """The nonnegativity rule is the projection max(x, 0), not any other map to
+    x >= 0: from x = 0 on data y <= 0 every unclamped update is <= 0 (A, R, C
+    are nonnegative), so the clamped iterate stays exactly zero, and one
+    clamped step equals max(unclamped step, 0)."""
+    g, A = _system()
+    y = -np.random.default_rng(7).random(A.shape[0])
+    x, _, _ = solvers.sirt(A, y, 5, nonnegative=True)
+    assert np.count_nonzero(x) == 0
+    xu, _, _ = solvers.sirt(A, y, 1, nonnegative=False)
+    assert xu.max() <= 0.0 and xu.min() < 0.0
+    y2 = np.random.default_rng(8).standard_normal(A.shape[0])
+    one_free, _, _ = solvers.sirt(A, y2, 1, nonnegative=False)
+    one_clamped, _, _ = solvers.sirt(A, y2, 1, nonnegative=True)
+    np.testing.assert_array_equal(one_clamped, np.maximum(one_free, 0.0))
