@@ -30,6 +30,9 @@ MUTATIONS = {
         "back_ctx b = {vol, (double)sino[((v - v0) * g->n_cols + c) * g->n_rows + r], power};"),
     "clip ignores far face": ("if (tmax < t_out) t_out = tmax;", "(void)tmax;"),
     "last interior plane dropped": ("for (int64_t q = 0; q <= g->n[k]; ++q)", "for (int64_t q = 0; q <= g->n[k] - 2; ++q)"),
+    "cone segment taken as a line": ("double t_in = 0.0, t_out = 1.0;", "double t_in = -1e30, t_out = 1e30;"),
+    "power 2 ignored": ("b->power == 1 ? w : w * w", "b->power == 1 ? w : w"),
+    "cylinder columns reversed": ("R * (cos(gam) * what[k] + sin(gam) * uhat[k])", "R * (cos(gam) * what[k] - sin(gam) * uhat[k])"),
 }
 
 PIN_TESTS = [
@@ -41,6 +44,8 @@ PIN_TESTS = [
     lambda: pins.test_single_voxel_chord_matches_brute_force(),
     lambda: pins.test_random_volume_matches_brute_force("helical_cyl"),
     lambda: pins.test_dense_transpose_8cubed_every_geometry_kind(),
+    lambda: pins.test_cone_segment_ends_at_an_endpoint_inside_the_box(),
+    lambda: pins.test_back_coefficient_powers(),
 ]
 
 

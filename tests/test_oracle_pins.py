@@ -133,6 +133,26 @@ def test_cone_axis_aligned_chord_through_box():
     assert y[0, 0, 2] == 0.0 and y[0, 0, 0] == 0.0
 
 
+def test_cone_segment_ends_at_an_endpoint_inside_the_box():
+    """A cone ray is the segment from the source to the pixel, not a line: an
+    axis-aligned ray whose source lies inside the box integrates from the
+    source to the far face; one whose pixel lies inside integrates from the
+    near face to the pixel (box widths, closed form)."""
+    nx, ny, nz = 10, 8, 6
+    sp = (1.0, 1.0, 1.0)
+    o = W.centred_origin(nx, ny, nz, sp)   # box [-5, 5) x [-4, 4) x [-3, 3)
+    # view 0: source inside at x = 1.3, pixel far outside along +x
+    # view 1: source far outside at x = -40, pixel inside at x = 2.2
+    src = np.array([[1.3, -0.7, 0.4], [-40.0, 0.3, 0.2]])
+    dc = np.array([[40.0, -0.7, 0.4], [2.2, 0.3, 0.2]])
+    du = np.array([[0.0, 30.0, 0.0], [0.0, 30.0, 0.0]])   # the side columns miss the box
+    dv = np.array([[0.0, 0.0, 1.0], [0.0, 0.0, 1.0]])
+    g = W.Geometry(W.BEAM_CONE, W.DET_FLAT, 1, 3, src, dc, du, dv, nx, ny, nz, o, sp)
+    y = oracle.forward(g, np.ones(g.vol_shape, np.float32))
+    assert y[0, 0, 1] == pytest.approx(5.0 - 1.3, rel=1e-12)
+    assert y[1, 0, 1] == pytest.approx(2.2 + 5.0, rel=1e-12)
+
+
 def test_textbook_reduction_axis_aligned_views():
     """Parallel views along +x and +y through voxel centres reduce to a numpy
     sum along that axis times the pitch (exact in FP64 up to summation order)."""
