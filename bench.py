@@ -13,7 +13,8 @@ under "geometry_gradient"; it is not part of the step.
 
 --impl reference times the FP64 CPU oracle on a bounded sample of the same
 workload (the reference arm; slow by design).  --solver cgls|sirt prints the
-solvers' iteration time against one forward + back instead.
+solvers' iteration time against one forward + back instead; --batch B the
+per-member time of the batched calls against single calls.
 """
 from __future__ import annotations
 
@@ -358,6 +359,62 @@ def run_solver(args, rank, world, local_rank):
     return 0
 
 
+def run_batch(args, rank, world, local_rank):
+    """Per-member time of the batched calls (ctp_forward_batch, ctp_back_batch
+    with plan.batch_chunk = min(B, 4)) against the single-volume calls on the
+    same workload: B volumes and B sinograms resident in HBM, CUDA events on
+    the launching stream, K timed repetitions after W warm-ups, max over
+    ranks."""
+    import torch
+
+    from ray_forward_back_b200 import ctp
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = select_workload(args)
+    g = wl.geom
+    B = args.batch
+    chunk = 4 if B >= 4 else (2 if B >= 2 else 1)
+    P = ctp.Projector(g, device=local_rank, plan={"batch_chunk": chunk})
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        vols = torch.rand((B,) + tuple(g.vol_shape), device=dev)
+        sinos = torch.rand((B,) + tuple(g.sino_shape), device=dev)
+        yo = torch.empty_like(sinos)
+        xo = torch.empty_like(vols)
+    stream.synchronize()
+
+    def timed(fn):
+        for _ in range(max(1, args.warmup)):
+            fn()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        stream.synchronize()
+        return e0.elapsed_time(e1) / args.steps
+
+    fwd_b = timed(lambda: P.forward(vols, out=yo, stream=stream)) / B
+    back_b = timed(lambda: P.back(sinos, out=xo, stream=stream)) / B
+    fwd_1 = timed(lambda: P.forward(vols[0], out=yo[0], stream=stream))
+    back_1 = timed(lambda: P.back(sinos[0], out=xo[0], stream=stream))
+    fwd_b, back_b, fwd_1, back_1 = aggregate_over_ranks([fwd_b, back_b, fwd_1, back_1], world, dev)
+    if rank != 0:
+        return 0
+    U = P.count_updates(stream=stream)
+    line = {"metric": f"batched forward + back Gupdates/s, batch of {B}", "unit": "Gupdates/s",
+            "value": world * 2 * U / ((fwd_b + back_b) * 1e-3) / 1e9, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32 (fp64 ray setup)", "data": "synthetic", "config": workload_config(wl),
+            "batch": B, "batch_chunk": P.info()["batch_chunk"],
+            "forward_ms_per_member": fwd_b, "back_ms_per_member": back_b,
+            "forward_ms_single": fwd_1, "back_ms_single": back_1,
+            "forward_speedup": fwd_1 / fwd_b, "back_speedup": back_1 / back_b}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -493,6 +550,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the geometry-gradient timing")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="time the batched calls on this many members against single calls instead")
     ap.add_argument("--solver", choices=["cgls", "sirt"], default=None,
                     help="time solver iterations (against one forward + back) instead of the projector step")
     args = ap.parse_args()
@@ -512,6 +571,8 @@ def main():
     try:
         if args.solver:
             return run_solver(args, rank, world, local_rank)
+        if args.batch > 0:
+            return run_batch(args, rank, world, local_rank)
         return run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
