@@ -816,8 +816,9 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
 #pragma unroll
         for (int m = 0; m < kB; ++m) {
           // a member whose stage scale is 0 or NaN adds nothing (its brick
-          // is all zero, or written as NaN, at the flush)
-          y[m] = S[m] > 0.f ? __ldg(sino + m * n_rays + i) : 0.f;
+          // is all zero, or written as NaN, at the flush); a single member
+          // only gets here with a positive scale
+          y[m] = (kB == 1 || S[m] > 0.f) ? __ldg(sino + m * n_rays + i) : 0.f;
           act |= y[m] != 0.f;
         }
       }
@@ -926,8 +927,12 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
     __syncthreads();
     // flush the stage into the volume and clear the accumulators
     float inv[kB];
+    bool nan_stage[kB];
 #pragma unroll
-    for (int m = 0; m < kB; ++m) inv[m] = S[m] > 0.f ? 1.f / S[m] : 0.f;
+    for (int m = 0; m < kB; ++m) {
+      inv[m] = S[m] > 0.f ? 1.f / S[m] : 0.f;
+      nan_stage[m] = S[m] != S[m];
+    }
     for (int i = tid; i < n_out; i += kBackThreads) {
       const int x = i % ex;
       const int t = i / ex;
@@ -937,8 +942,7 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
       const Off gi = ((Off)(lo[2] + z) * ny + (Off)(lo[1] + yy)) * nx + (Off)(lo[0] + x);
 #pragma unroll
       for (int m = 0; m < kB; ++m) {
-        const bool nan_stage = S[m] != S[m];
-        const float val = nan_stage ? CUDART_NAN_F : (float)acc[m * n_acc + ai] * inv[m];
+        const float val = nan_stage[m] ? CUDART_NAN_F : (float)acc[m * n_acc + ai] * inv[m];
         acc[m * n_acc + ai] = 0;
         float* const vm = vol + m * n_vox;
         if (P.view_groups > 1) {
