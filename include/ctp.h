@@ -75,7 +75,7 @@ enum { CTP_BEAM_PARALLEL = 0, CTP_BEAM_CONE = 1 };
 enum { CTP_DET_FLAT = 0, CTP_DET_CYLINDRICAL = 1 };
 
 /* Adjoint variants.  AUTO picks by the collision ratio measured at create. */
-enum { CTP_ADJOINT_AUTO = 0, CTP_ADJOINT_BRICK = 1, CTP_ADJOINT_SORT = 2 };
+enum { CTP_ADJOINT_AUTO = 0, CTP_ADJOINT_BRICK = 1, CTP_ADJOINT_SORT = 2, CTP_ADJOINT_SCATTER = 3 };
 
 /* Optional plan overrides (all zero = library defaults). */
 typedef struct {

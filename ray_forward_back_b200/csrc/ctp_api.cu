@@ -152,7 +152,7 @@ ctp_status validate_desc(const ctp_geom_desc *d) {
     return fail(CTP_ERR_INVALID_ARGUMENT, "a per-view vector array is NULL");
   if (d->plan) {
     const ctp_plan *p = d->plan;
-    if (p->adjoint_variant < CTP_ADJOINT_AUTO || p->adjoint_variant > CTP_ADJOINT_SORT)
+    if (p->adjoint_variant < CTP_ADJOINT_AUTO || p->adjoint_variant > CTP_ADJOINT_SCATTER)
       return fail(CTP_ERR_INVALID_ARGUMENT, "plan.adjoint_variant %d", p->adjoint_variant);
     for (int k = 0; k < 3; ++k)
       if (p->brick[k] < 0 || p->brick[k] > 1024) return fail(CTP_ERR_INVALID_ARGUMENT, "plan.brick[%d]", k);
@@ -590,7 +590,7 @@ ctp_status ctp_geom_create(const ctp_geom_desc *desc, ctp_geom **out) {
   }
   // adjoint variant: forced by the plan, else by the measured collision ratio
   const int forced = plan ? plan->adjoint_variant : CTP_ADJOINT_AUTO;
-  if (forced == CTP_ADJOINT_BRICK || forced == CTP_ADJOINT_SORT)
+  if (forced == CTP_ADJOINT_BRICK || forced == CTP_ADJOINT_SORT || forced == CTP_ADJOINT_SCATTER)
     g->adjoint_variant = forced;
   else
     g->adjoint_variant = g->collision_ratio >= kSortMinCollisionRatio ? CTP_ADJOINT_SORT : CTP_ADJOINT_BRICK;
@@ -734,11 +734,16 @@ ctp_status ctp_back_power(const ctp_geom *g, const float *sino, float *vol, int 
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pending error before ctp_back");
   const bool sorted = g->adjoint_variant == CTP_ADJOINT_SORT;
-  if (sorted || g->back.view_groups > 1) {
+  const bool scatter = g->adjoint_variant == CTP_ADJOINT_SCATTER;
+  if (sorted || scatter || g->back.view_groups > 1) {
     e = cudaMemsetAsync(vol, 0, sizeof(float) * (size_t)g->n_vox, s);
+    if (e == cudaSuccess && scatter && g->fwd.any_transposed)
+      e = cudaMemsetAsync(g->d_volT, 0, sizeof(float) * (size_t)g->n_vox, s);
     if (e != cudaSuccess) return cuda_fail(e, "volume zero-fill");
   }
-  if (sorted)
+  if (scatter)
+    e = ctp::launch_back_scatter(g->fwd, g->d_views, g->d_trig, sino, vol, g->d_volT, power, g->wide_index, s);
+  else if (sorted)
     e = ctp::launch_back_sort(g->fwd, g->d_views, g->d_trig, sino, vol, power, g->wide_index, s);
   else
     e = ctp::launch_back_brick(g->back, g->d_views, g->d_trig, sino, vol, power, 1, g->wide_index, s);

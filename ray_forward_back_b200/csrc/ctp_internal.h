@@ -82,6 +82,10 @@ cudaError_t launch_count(const FwdLaunch& p, const ViewRec* views, const double*
                          unsigned long long* counter, cudaStream_t stream);
 cudaError_t launch_back_sort(const FwdLaunch& p, const ViewRec* views, const double* trig, const float* sino,
                              float* vol, int power, bool wide_index, cudaStream_t stream);
+// Ray-driven scatter adjoint into vol (x-fastest views) and volT (y-fastest
+// views), both zeroed by the caller; volT is then added into vol.
+cudaError_t launch_back_scatter(const FwdLaunch& p, const ViewRec* views, const double* trig, const float* sino,
+                                float* vol, float* volT, int power, bool wide_index, cudaStream_t stream);
 cudaError_t launch_collision_count(const FwdLaunch& p, const ViewRec* views, const double* trig,
                                    unsigned long long* counters, bool wide_index, cudaStream_t stream);
 size_t back_brick_smem_bytes(const int32_t brick[3], int kb = 1);

@@ -47,6 +47,9 @@ namespace {
 #ifndef CTP_FWD_MIN_BLOCKS
 #define CTP_FWD_MIN_BLOCKS 5
 #endif
+#ifndef CTP_SCATTER_MIN_BLOCKS
+#define CTP_SCATTER_MIN_BLOCKS 5
+#endif
 #ifndef CTP_BACK_MIN_BLOCKS
 #define CTP_BACK_MIN_BLOCKS 3
 #endif
@@ -237,14 +240,32 @@ __device__ __forceinline__ void walk_warp_bf(bool active, const Walk& W, Off off
 // leave the clipped box; a minor crossing that rounds past the exit is
 // dropped (its error is below one ulp of the walk length).
 //
+// Positions are measured from a local origin.  Without re-anchoring
+// (kAnchor = 0) that origin is the entry, and a crossing far along the ray
+// carries an FP32 error of about one ulp of its distance from the entry: a
+// few 1e-5 of a voxel after a few hundred voxels.  That is harmless where
+// segment errors telescope (a forward sum over one ray) but not where a
+// voxel sums a few short segments of different rays (the adjoint).  With
+// kAnchor = K, every K slabs each lane moves its origin to the start of its
+// current slab and recomputes its local FP32 parameters there in FP64, from
+// the entry's FP64 values at anc[q * kAncStride] (q = 0-2: l0 per axis,
+// 3-5: inc per axis, 6: length), so positions never grow beyond K slabs.
+//
 // All 32 lanes must call this together; lanes without a ray pass active = false.
 // With kUniform, every lane calls visit(offset, length, flag) at every segment
 // slot, flag telling whether the segment exists for that lane (so the visitor
 // may use warp collectives); a slot that no lane of the warp has is skipped.
 // Without it, visit(offset, length, true) is called for existing segments only.
-template <bool kAlign, bool kUniform, typename Off, typename Visit>
+constexpr int kAncStride = kFwdCols * kFwdRows;  // one FP64 record per thread of the block, field-major
+#ifndef CTP_WALK_ANCHOR
+#define CTP_WALK_ANCHOR 64
+#endif
+constexpr int kWalkAnchor = CTP_WALK_ANCHOR;  // slabs between re-anchorings of the whole-volume adjoint walks
+
+template <bool kAlign, bool kUniform, int kAnchor, typename Off, typename Visit>
 __device__ __forceinline__ void walk(bool active, const Walk& W, const int lo[3], const int hi[3], Off off, Off s0,
-                                     Off s1, Off s2, Visit&& visit) {
+                                     Off s1, Off s2, const double* __restrict__ anc, Visit&& visit) {
+  static_assert(kAnchor == 0 || (kAnchor & (kAnchor - 1)) == 0, "re-anchoring period is a power of two");
   constexpr unsigned kFull = 0xffffffffu;
   const float i0 = W.inc[0], i1 = W.inc[1], i2 = W.inc[2];
   int a, b, c;
@@ -254,9 +275,10 @@ __device__ __forceinline__ void walk(bool active, const Walk& W, const int lo[3]
   const int Na = active ? pick3(a, W.N[0], W.N[1], W.N[2]) : 0;
   const int Nb = pick3(b, W.N[0], W.N[1], W.N[2]);
   const int Nc = pick3(c, W.N[0], W.N[1], W.N[2]);
-  const float l0a = pick3(a, W.l0[0], W.l0[1], W.l0[2]), inca = pick3(a, i0, i1, i2);
-  const float l0b = pick3(b, W.l0[0], W.l0[1], W.l0[2]), incb = pick3(b, i0, i1, i2);
-  const float l0c = pick3(c, W.l0[0], W.l0[1], W.l0[2]), incc = pick3(c, i0, i1, i2);
+  float l0a = pick3(a, W.l0[0], W.l0[1], W.l0[2]);
+  float l0b = pick3(b, W.l0[0], W.l0[1], W.l0[2]);
+  float l0c = pick3(c, W.l0[0], W.l0[1], W.l0[2]);
+  const float inca = pick3(a, i0, i1, i2), incb = pick3(b, i0, i1, i2), incc = pick3(c, i0, i1, i2);
   const Off sa = pick3(a, s0, s1, s2), sb = pick3(b, s0, s1, s2), sc = pick3(c, s0, s1, s2);
 
   // slab alignment: entry position along the major axis in travel direction
@@ -279,29 +301,76 @@ __device__ __forceinline__ void walk(bool active, const Walk& W, const int lo[3]
   // the active lanes, whose |s| stays far below 2^24)
   float fs = -(float)d;
 
-  const float L = W.L;
-  const float fNb = (float)Nb, fNc = (float)Nc;
+  float L = W.L;
+  float fNb = (float)Nb, fNc = (float)Nc;
   float tb = Nb > 0 ? l0b : CUDART_INF_F;
-  float fjb = 1.f;
+  float tc = Nc > 0 ? l0c : CUDART_INF_F;
+  float fjb = 1.f, fjc = 1.f;
+  float jb0 = 0.f, jc0 = 0.f;  // entry-frame index of crossing 0 of the current frame (b, c)
   float cur = 0.f;
-  if (!__any_sync(kFull, active && Nc > 0)) {
-    // no lane crosses a second minor axis: at most two segments per slab
-#pragma unroll kWalk2Unroll
-    for (int k = 0; k <= kmax; ++k, fs += 1.f) {
-      const int s = k - d;
-      const bool on = (unsigned)s <= (unsigned)Na;
-      // the (Na+1)-th major crossing lies at or past the exit: clamping to L
-      // ends the last slab there (to within rounding of the walk length)
-      const float tx = fminf(fmaf(fs, inca, l0a), L);
-      const bool cb = on && tb < tx;
+  // Move the local origin to the start of slab s >= 1 (major crossing s - 1).
+  auto reanchor = [&](int s) {
+    const double la = anc[a * kAncStride], ja = anc[(3 + a) * kAncStride];
+    const double O = fma((double)(s - 1), ja, la);
+    l0a = (float)(fma((double)s, ja, la) - O);
+    L = (float)(anc[6 * kAncStride] - O);
+    cur = 0.f;
+    fs = 0.f;
+    if (tb < CUDART_INF_F) {  // the pending b crossing has entry-frame index jb0 + fjb - 1
+      const float db = fjb - 1.f;
+      jb0 += db;
+      fNb -= db;
+      fjb = 1.f;
+      l0b = (float)(fma((double)jb0, anc[(3 + b) * kAncStride], anc[b * kAncStride]) - O);
+      tb = l0b;
+    }
+    if (tc < CUDART_INF_F) {
+      const float dc = fjc - 1.f;
+      jc0 += dc;
+      fNc -= dc;
+      fjc = 1.f;
+      l0c = (float)(fma((double)jc0, anc[(3 + c) * kAncStride], anc[c * kAncStride]) - O);
+      tc = l0c;
+    }
+  };
+  // One slab of the two-segment walk (no lane crosses axis c).
+  auto slab2 = [&](int k) {
+    const int s = k - d;
+    const bool on = (unsigned)s <= (unsigned)Na;
+    // the (Na+1)-th major crossing lies at or past the exit: clamping to L
+    // ends the last slab there (to within rounding of the walk length)
+    const float tx = fminf(fmaf(fs, inca, l0a), L);
+    const bool cb = on && tb < tx;
+    const float m1 = fmaxf(fminf(tb, tx), cur);
+    if (kUniform) {
+      visit(off, m1 - cur, on);
+      if (__any_sync(kFull, cb)) visit(off + sb, tx - m1, cb);
+    } else {
+      if (on) visit(off, m1 - cur, true);
+      if (cb) visit(off + sb, tx - m1, true);
+    }
+    if (on) {
+      off += (cb ? sb : (Off)0) + sa;
+      cur = tx;
+    }
+    if (cb) {
+      tb = fjb < fNb ? fmaf(fjb, incb, l0b) : CUDART_INF_F;
+      fjb += 1.f;
+    }
+  };
+  // One slab of the three-segment walk.
+  auto slab3 = [&](int k) {
+    const int s = k - d;
+    const bool on = (unsigned)s <= (unsigned)Na;
+    const float tx = fminf(fmaf(fs, inca, l0a), L);
+    const bool cb = on && tb < tx, cc = on && tc < tx;
+    if (!kUniform && !__any_sync(kFull, cc)) {
+      // No lane crosses axis c in this slab (the common case: c is the axis
+      // crossed least often, and the aligned lanes of a warp cross it at
+      // nearly the same slab): the slab is one or two segments.
       const float m1 = fmaxf(fminf(tb, tx), cur);
-      if (kUniform) {
-        visit(off, m1 - cur, on);
-        if (__any_sync(kFull, cb)) visit(off + sb, tx - m1, cb);
-      } else {
-        if (on) visit(off, m1 - cur, true);
-        if (cb) visit(off + sb, tx - m1, true);
-      }
+      if (on) visit(off, m1 - cur, true);
+      if (cb) visit(off + sb, tx - m1, true);
       if (on) {
         off += (cb ? sb : (Off)0) + sa;
         cur = tx;
@@ -310,42 +379,59 @@ __device__ __forceinline__ void walk(bool active, const Walk& W, const int lo[3]
         tb = fjb < fNb ? fmaf(fjb, incb, l0b) : CUDART_INF_F;
         fjb += 1.f;
       }
+      return;
+    }
+    const float m1 = fmaxf(fminf(fminf(tb, tc), tx), cur);
+    const float m2 = fmaxf(fminf(fmaxf(tb, tc), tx), m1);
+    const Off db = cb ? sb : (Off)0, dc = cc ? sc : (Off)0;
+    const Off o2 = off + (tb <= tc ? db : dc);
+    const Off o3 = off + db + dc;
+    if (kUniform) {
+      visit(off, m1 - cur, on);
+      if (__any_sync(kFull, cb || cc)) visit(o2, m2 - m1, cb || cc);
+      if (__any_sync(kFull, cb && cc)) visit(o3, tx - m2, cb && cc);
+    } else {
+      if (on) visit(off, m1 - cur, true);
+      if (cb || cc) visit(o2, m2 - m1, true);
+      if (cb && cc) visit(o3, tx - m2, true);
+    }
+    if (on) {
+      off = o3 + sa;
+      cur = tx;
+    }
+    if (cb) {
+      tb = fjb < fNb ? fmaf(fjb, incb, l0b) : CUDART_INF_F;
+      fjb += 1.f;
+    }
+    if (cc) {
+      tc = fjc < fNc ? fmaf(fjc, incc, l0c) : CUDART_INF_F;
+      fjc += 1.f;
+    }
+  };
+  const bool three = __any_sync(kFull, active && Nc > 0);
+  if (kAnchor == 0) {
+    if (!three) {
+#pragma unroll kWalk2Unroll
+      for (int k = 0; k <= kmax; ++k, fs += 1.f) slab2(k);
+    } else {
+#pragma unroll kWalk3Unroll
+      for (int k = 0; k <= kmax; ++k, fs += 1.f) slab3(k);
     }
   } else {
-    // up to three segments per slab
-    float tc = Nc > 0 ? l0c : CUDART_INF_F;
-    float fjc = 1.f;
-#pragma unroll kWalk3Unroll
-    for (int k = 0; k <= kmax; ++k, fs += 1.f) {
-      const int s = k - d;
-      const bool on = (unsigned)s <= (unsigned)Na;
-      const float tx = fminf(fmaf(fs, inca, l0a), L);
-      const bool cb = on && tb < tx, cc = on && tc < tx;
-      const float m1 = fmaxf(fminf(fminf(tb, tc), tx), cur);
-      const float m2 = fmaxf(fminf(fmaxf(tb, tc), tx), m1);
-      const Off db = cb ? sb : (Off)0, dc = cc ? sc : (Off)0;
-      const Off o2 = off + (tb <= tc ? db : dc);
-      const Off o3 = off + db + dc;
-      if (kUniform) {
-        visit(off, m1 - cur, on);
-        if (__any_sync(kFull, cb || cc)) visit(o2, m2 - m1, cb || cc);
-        if (__any_sync(kFull, cb && cc)) visit(o3, tx - m2, cb && cc);
+    // blocks of kAnchor slabs; every lane already inside its walk re-anchors
+    // at the start of each block after the first
+    for (int k0 = 0; k0 <= kmax; k0 += kAnchor) {
+      if (k0 > 0) {
+        const int s = k0 - d;
+        if ((unsigned)s <= (unsigned)Na && s > 0) reanchor(s);
+      }
+      const int kend = min(k0 + kAnchor, kmax + 1);
+      if (!three) {
+#pragma unroll kWalk2Unroll
+        for (int k = k0; k < kend; ++k, fs += 1.f) slab2(k);
       } else {
-        if (on) visit(off, m1 - cur, true);
-        if (cb || cc) visit(o2, m2 - m1, true);
-        if (cb && cc) visit(o3, tx - m2, true);
-      }
-      if (on) {
-        off = o3 + sa;
-        cur = tx;
-      }
-      if (cb) {
-        tb = fjb < fNb ? fmaf(fjb, incb, l0b) : CUDART_INF_F;
-        fjb += 1.f;
-      }
-      if (cc) {
-        tc = fjc < fNc ? fmaf(fjc, incc, l0c) : CUDART_INF_F;
-        fjc += 1.f;
+#pragma unroll kWalk3Unroll
+        for (int k = k0; k < kend; ++k, fs += 1.f) slab3(k);
       }
     }
   }
@@ -389,7 +475,7 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows, kB == 1 ? CTP_FWD_MIN_BLOC
   float acc[kB];
 #pragma unroll
   for (int j = 0; j < kB; ++j) acc[j] = 0.f;
-  walk<true, false, Off>(hit, W, lo, hi, off, W.step[0] * sx, W.step[1] * sy, W.step[2] * sz,
+  walk<true, false, 0, Off>(hit, W, lo, hi, off, W.step[0] * sx, W.step[1] * sy, W.step[2] * sz, nullptr,
                          [&](Off o, float len, bool) {
 #pragma unroll
                            for (int j = 0; j < kB; ++j) acc[j] = fmaf(len, __ldg(base + j * n_vox + o), acc[j]);
@@ -424,7 +510,7 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows) count_kernel(FwdLaunch P, 
   const bool hit = valid && clip(R, lo, hi, t_in, t_out);
   Walk W = {};
   if (hit) entry(R, t_in, t_out, lo, hi, W);
-  walk<false, false, int>(hit, W, lo, hi, 0, 0, 0, 0, [&](int, float len, bool) { n += len > 0.f ? 1ull : 0ull; });
+  walk<false, false, 0, int>(hit, W, lo, hi, 0, 0, 0, 0, nullptr, [&](int, float len, bool) { n += len > 0.f ? 1ull : 0ull; });
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
   if ((threadIdx.x & 31) == 0 && n) atomicAdd(counter, n);
@@ -1054,11 +1140,15 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_FWD_MIN_BLOCKS)
   double t_in = 0.0, t_out = 0.0;
   const bool hit = valid && y != 0.f && clip(R, lo, hi, t_in, t_out);
   Walk W = {};
-  if (hit) entry(R, t_in, t_out, lo, hi, W);
+  // the counting form only counts segments: no re-anchoring needed
+  constexpr int kAnchor = kCount ? 0 : kWalkAnchor;
+  __shared__ double s_anc[kAnchor ? 7 * kAncStride : 1];
+  double* const anc = s_anc + (kAnchor ? threadIdx.y * kFwdCols + threadIdx.x : 0);
+  if (hit) entry(R, t_in, t_out, lo, hi, W, kAnchor ? anc : nullptr, kAncStride);
   const Off nx = P.vol.n[0], sz = (Off)P.vol.n[0] * P.vol.n[1];
   const Off off = (Off)W.i[2] * sz + (Off)W.i[1] * nx + (Off)W.i[0];
   unsigned long long n_upd = 0, n_runs = 0;
-  walk<true, true, Off>(hit, W, lo, hi, off, (Off)W.step[0], W.step[1] * nx, W.step[2] * sz,
+  walk<true, true, kAnchor, Off>(hit, W, lo, hi, off, (Off)W.step[0], W.step[1] * nx, W.step[2] * sz, anc,
                         [&](Off o, float len, bool f) {
                           warp_segment_reduce<kCount, Off>(o, coef<kPower>(len) * y, f, vol, n_upd, n_runs);
                         });
@@ -1068,9 +1158,94 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_FWD_MIN_BLOCKS)
   }
 }
 
+// ------------------------------------------------------- back: ray scatter --
+
+// Ray-driven scatter adjoint: the forward kernel's grid, set-up and aligned
+// slab walk, with every positive-length segment added into the volume by one
+// red.global.add.f32.  The warp's 32 lanes hold neighbouring rays of one view
+// and, aligned on absolute slab positions, add into neighbouring voxels of one
+// slab; views whose columns run along y accumulate into a y-fastest copy (as
+// the forward gathers from it), so a warp's adds stay within a few sectors.
+// Both accumulators must be zero on entry; transpose_add_kernel folds the copy
+// into the volume afterwards.
+template <int kPower, typename Off>
+__global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_SCATTER_MIN_BLOCKS)
+    back_scatter_kernel(FwdLaunch P, const ViewRec* __restrict__ views, const double* __restrict__ trig,
+                        const float* __restrict__ sino, float* __restrict__ vol, float* __restrict__ volT) {
+  const int per_band = P.dims.n_views * P.n_col_tiles;
+  const int band = blockIdx.x / per_band;
+  const int rem = blockIdx.x - band * per_band;
+  const int v = rem / P.n_col_tiles;
+  const int ct = rem - v * P.n_col_tiles;
+  const int c = ct * kFwdCols + threadIdx.x;
+  const int r = band * kFwdRows + threadIdx.y;
+  const bool valid = c < P.dims.n_cols && r < P.dims.n_rows;
+  const float y = valid ? __ldg(sino + ((size_t)v * P.dims.n_rows + r) * P.dims.n_cols + c) : 0.f;
+  const ViewRec& V = views[v];
+  Ray R;
+  make_ray(V, P.vol, trig, P.dims, v, valid ? r : 0, valid ? c : 0, R);
+  const int lo[3] = {0, 0, 0};
+  const int hi[3] = {P.vol.n[0], P.vol.n[1], P.vol.n[2]};
+  double t_in = 0.0, t_out = 0.0;
+  const bool hit = valid && y != 0.f && clip(R, lo, hi, t_in, t_out);
+  Walk W = {};
+  __shared__ double s_anc[7 * kAncStride];
+  double* const anc = s_anc + threadIdx.y * kFwdCols + threadIdx.x;
+  if (hit) entry(R, t_in, t_out, lo, hi, W, anc, kAncStride);
+  const Off nx = P.vol.n[0], ny = P.vol.n[1];
+  const bool yfast = V.layout != 0;
+  float* const base = yfast ? volT : vol;
+  const Off sx = yfast ? ny : (Off)1;
+  const Off sy = yfast ? (Off)1 : nx;
+  const Off sz = nx * ny;
+  const Off off = (Off)W.i[2] * sz + (Off)W.i[1] * sy + (Off)W.i[0] * sx;
+  walk<true, false, kWalkAnchor, Off>(hit, W, lo, hi, off, W.step[0] * sx, W.step[1] * sy, W.step[2] * sz, anc,
+                                      [&](Off o, float len, bool) {
+                           if (len > 0.f) atomicAdd(base + o, coef<kPower>(len) * y);
+                         });
+}
+
+// vol[z][y][x] += volT[z][x][y] (the scatter adjoint's y-fastest accumulator).
+__global__ void __launch_bounds__(256) transpose_add_kernel(const float* __restrict__ in, float* __restrict__ out,
+                                                            int nx, int ny) {
+  __shared__ float tile[32][33];
+  const size_t slice = (size_t)blockIdx.z * nx * ny;
+  const int x0 = blockIdx.x * 32, y0 = blockIdx.y * 32;
+  for (int j = threadIdx.y; j < 32; j += 8) {
+    const int y = y0 + threadIdx.x, x = x0 + j;
+    if (x < nx && y < ny) tile[j][threadIdx.x] = in[slice + (size_t)x * ny + y];
+  }
+  __syncthreads();
+  for (int j = threadIdx.y; j < 32; j += 8) {
+    const int x = x0 + threadIdx.x, y = y0 + j;
+    if (x < nx && y < ny) out[slice + (size_t)y * nx + x] += tile[threadIdx.x][j];
+  }
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------- launchers --
+
+cudaError_t launch_back_scatter(const FwdLaunch& p, const ViewRec* views, const double* trig, const float* sino,
+                                float* vol, float* volT, int power, bool wide_index, cudaStream_t stream) {
+  const long long blocks = (long long)p.n_row_bands * p.dims.n_views * p.n_col_tiles;
+  if (blocks <= 0) return cudaSuccess;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  dim3 block(kFwdCols, kFwdRows);
+  const unsigned nb = (unsigned)blocks;
+  if (power == 2) {
+    if (wide_index) back_scatter_kernel<2, long long><<<nb, block, 0, stream>>>(p, views, trig, sino, vol, volT);
+    else back_scatter_kernel<2, int><<<nb, block, 0, stream>>>(p, views, trig, sino, vol, volT);
+  } else {
+    if (wide_index) back_scatter_kernel<1, long long><<<nb, block, 0, stream>>>(p, views, trig, sino, vol, volT);
+    else back_scatter_kernel<1, int><<<nb, block, 0, stream>>>(p, views, trig, sino, vol, volT);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || !p.any_transposed) return e;
+  dim3 grid((p.vol.n[0] + 31) / 32, (p.vol.n[1] + 31) / 32, p.vol.n[2]);
+  transpose_add_kernel<<<grid, dim3(32, 8), 0, stream>>>(volT, vol, p.vol.n[0], p.vol.n[1]);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_transpose_xy(const float* vol, float* volT, const VolDesc& vd, cudaStream_t stream) {
   dim3 grid((vd.n[0] + 31) / 32, (vd.n[1] + 31) / 32, vd.n[2]);

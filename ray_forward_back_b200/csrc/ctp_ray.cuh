@@ -110,8 +110,11 @@ __device__ __forceinline__ int clampi(int x, int lo, int hi) { return x < lo ? l
 
 // Entry voxel, crossing counts and local FP32 crossing parameters of the
 // clipped segment [t_in, t_out] inside the box [lo, hi).
+// With w64 (a per-lane record of 7 doubles at stride `stride`: l0[3],
+// inc[3], L) the FP64 values behind W's FP32 l0, inc and L are kept too, for
+// walks that re-anchor their local FP32 parameters along the ray.
 __device__ __forceinline__ void entry(const Ray& R, double t_in, double t_out, const int lo[3], const int hi[3],
-                                      Walk& W) {
+                                      Walk& W, double* w64 = nullptr, int stride = 1) {
 #pragma unroll
   for (int k = 0; k < 3; ++k) {
     const double e = fma(t_in, R.D[k], R.A[k]);
@@ -125,8 +128,13 @@ __device__ __forceinline__ void entry(const Ray& R, double t_in, double t_out, c
       W.N[k] = max(i1 - i0, 0);
       W.step[k] = 1;
       const double tc = ((double)(i0 + 1) - R.A[k]) * R.rcp[k];
-      W.l0[k] = (float)((tc - t_in) * R.len);
-      W.inc[k] = (float)(R.rcp[k] * R.len);
+      const double l0d = (tc - t_in) * R.len, incd = R.rcp[k] * R.len;
+      W.l0[k] = (float)l0d;
+      W.inc[k] = (float)incd;
+      if (w64) {
+        w64[k * stride] = l0d;
+        w64[(3 + k) * stride] = incd;
+      }
     } else if (R.D[k] < 0.0) {
       const int i0 = clampi((int)ceil(el) - 1, lo[k], hi[k] - 1);
       const int i1 = clampi((int)floor(xl), lo[k], hi[k] - 1);
@@ -134,17 +142,28 @@ __device__ __forceinline__ void entry(const Ray& R, double t_in, double t_out, c
       W.N[k] = max(i0 - i1, 0);
       W.step[k] = -1;
       const double tc = ((double)i0 - R.A[k]) * R.rcp[k];
-      W.l0[k] = (float)((tc - t_in) * R.len);
-      W.inc[k] = (float)(-R.rcp[k] * R.len);
+      const double l0d = (tc - t_in) * R.len, incd = -R.rcp[k] * R.len;
+      W.l0[k] = (float)l0d;
+      W.inc[k] = (float)incd;
+      if (w64) {
+        w64[k * stride] = l0d;
+        w64[(3 + k) * stride] = incd;
+      }
     } else {
       W.i[k] = clampi((int)floor(el), lo[k], hi[k] - 1);
       W.N[k] = 0;
       W.step[k] = 1;
       W.l0[k] = CUDART_INF_F;
       W.inc[k] = CUDART_INF_F;
+      if (w64) {
+        w64[k * stride] = CUDART_INF;
+        w64[(3 + k) * stride] = CUDART_INF;
+      }
     }
   }
-  W.L = (float)((t_out - t_in) * R.len);
+  const double Ld = (t_out - t_in) * R.len;
+  W.L = (float)Ld;
+  if (w64) w64[6 * stride] = Ld;
 }
 
 template <typename T>

@@ -103,3 +103,34 @@ def adjoint_mismatch(P, geom, seed=0):
 def oracle_chords(geom):
     """Physical chord of every ray through the volume box (forward of ones)."""
     return oracle.forward(geom, np.ones(geom.vol_shape, np.float32))
+
+
+def forward_errors(y_gpu, y_ref, chord, min_spacing):
+    """Achieved errors of a forward projection under the forward tolerances:
+    relative L2; the worst relative error on rays crossing the volume (chord
+    >= one pitch and |y| >= 1e-3 max|y|); the worst |error| / max|y| on the
+    other rays."""
+    y_gpu = np.asarray(y_gpu, dtype=np.float64)
+    y_ref = np.asarray(y_ref, dtype=np.float64)
+    ymax = float(np.abs(y_ref).max())
+    err = np.abs(y_gpu - y_ref)
+    crossing = (chord >= min_spacing) & (np.abs(y_ref) >= 1e-3 * ymax)
+    return {"rel_l2": rel_l2(y_gpu, y_ref),
+            "crossing_rays": int(crossing.sum()),
+            "worst_rel_crossing": float((err[crossing] / np.abs(y_ref[crossing])).max()) if crossing.any() else 0.0,
+            "worst_abs_other_over_max": float(err[~crossing].max() / ymax) if (~crossing).any() else 0.0}
+
+
+def back_errors(x_gpu, x_ref):
+    """Achieved errors of a back projection under the adjoint tolerances:
+    relative L2; the worst relative error on voxels with |x| >= 1e-3 max|x|;
+    the worst |error| / max|x| on the other voxels."""
+    x_gpu = np.asarray(x_gpu, dtype=np.float64)
+    x_ref = np.asarray(x_ref, dtype=np.float64)
+    xmax = float(np.abs(x_ref).max())
+    err = np.abs(x_gpu - x_ref)
+    big = np.abs(x_ref) >= 1e-3 * xmax
+    return {"rel_l2": rel_l2(x_gpu, x_ref),
+            "checked_voxels": int(big.sum()),
+            "worst_rel": float((err[big] / np.abs(x_ref[big])).max()) if big.any() else 0.0,
+            "worst_abs_other_over_max": float(err[~big].max() / xmax) if (~big).any() else 0.0}

@@ -43,8 +43,15 @@ def ragged_geometries():
 
 
 def _local_len(P, geom):
-    b = np.array(P.info()["brick"], dtype=np.float64) * np.array(geom.spacing)
-    return float(np.linalg.norm(b))
+    """Longest distance over which an adjoint variant measures FP32 crossing
+    positions: the brick diagonal for the brick adjoint; for the ray-driven
+    variants (sort, scatter), whose walks re-anchor every 64 slabs, 65 voxel
+    diagonals, or the volume diagonal if that is shorter."""
+    if P.info()["adjoint_variant"] == 1:
+        b = np.array(P.info()["brick"], dtype=np.float64) * np.array(geom.spacing)
+        return float(np.linalg.norm(b))
+    vol_diag = float(np.linalg.norm(np.array([geom.nx, geom.ny, geom.nz]) * np.array(geom.spacing)))
+    return min(vol_diag, 65.0 * float(np.linalg.norm(geom.spacing)))
 
 
 def _seeded_volume(geom, seed):
@@ -173,7 +180,7 @@ def test_workload_full_size_sparse_back(index):
     ref = np.array([expect[i] for i in keys])
     cnt = np.array([count[i] for i in keys])
     got = x[torch.from_numpy(keys).cuda()].double().cpu().numpy()
-    tau = 8 * EPS32 * float(np.linalg.norm(np.array(P.info()["brick"]) * np.array(g.spacing)))
+    tau = 8 * EPS32 * _local_len(P, g)
     assert np.all(np.abs(got - ref) <= 1e-4 * np.abs(ref) + tau * cnt)
     # nothing outside the rays' support beyond FP32 crumbs
     mask = torch.ones(g.n_vox, dtype=torch.bool, device="cuda")
@@ -275,29 +282,30 @@ def test_host_pointer_is_rejected():
 
 # ------------------------------------------ sort / segment-reduce adjoint ---
 
+@pytest.mark.parametrize("variant", [1, 2, 3])
 @pytest.mark.parametrize("name", sorted(ragged_geometries()))
-def test_back_sort_variant_matches_oracle_small(name):
-    """The sort / segment-reduce adjoint meets the same tolerances."""
+def test_back_variant_matches_oracle_small(name, variant):
+    """Every adjoint variant (brick, sort / segment-reduce, ray scatter) meets
+    the same tolerances, forced through the plan."""
     g = ragged_geometries()[name]
     rng = np.random.default_rng(12)
     sino = rng.random(g.sino_shape).astype(np.float32)
-    P = projector(g, {"adjoint_variant": 2})
-    assert P.info()["adjoint_variant"] == 2
+    P = projector(g, {"adjoint_variant": variant})
+    assert P.info()["adjoint_variant"] == variant
     x = gpu_back(P, sino)
-    check_back(x, oracle.back(g, sino), oracle.back(g, np.abs(sino), power=0), float(np.linalg.norm(
-        np.array([g.nx, g.ny, g.nz]) * np.array(g.spacing))), name)
+    check_back(x, oracle.back(g, sino), oracle.back(g, np.abs(sino), power=0), _local_len(P, g), name)
     assert adjoint_mismatch(P, g) <= 1e-5
 
 
+@pytest.mark.parametrize("variant", [1, 2, 3])
 @pytest.mark.parametrize("index", [0, 1])
-def test_back_sort_variant_workloads(index):
+def test_back_variant_workloads(index, variant):
     wl = W.workload(index)
     g = wl.geom
     sino = wl.sinogram()
-    P = projector(g, {"adjoint_variant": 2})
+    P = projector(g, {"adjoint_variant": variant})
     x = gpu_back(P, sino)
-    check_back(x, oracle.back(g, sino), oracle.back(g, sino, power=0),
-               float(np.linalg.norm(np.array([g.nx, g.ny, g.nz]) * np.array(g.spacing))), wl.name)
+    check_back(x, oracle.back(g, sino), oracle.back(g, sino, power=0), _local_len(P, g), wl.name)
 
 
 def high_magnification_cone():
@@ -349,7 +357,7 @@ def test_device_update_count_matches_oracle_fixture(index):
 
 # ------------------------------------------------ coefficient powers (NEXT) ---
 
-@pytest.mark.parametrize("variant", [1, 2])
+@pytest.mark.parametrize("variant", [1, 2, 3])
 @pytest.mark.parametrize("name", ["parallel_ragged", "cone_ragged", "helical_ragged", "parallel_tilted"])
 def test_back_squared_coefficients(name, variant):
     """Back projection with squared weights (the normal operator's diagonal)
@@ -364,7 +372,7 @@ def test_back_squared_coefficients(name, variant):
     x = P.back_power(torch.from_numpy(sino).cuda(), 2)
     torch.cuda.synchronize()
     diag = float(np.linalg.norm(g.spacing))
-    local = _local_len(P, g) if variant == 1 else float(np.linalg.norm(np.array([g.nx, g.ny, g.nz]) * np.array(g.spacing)))
+    local = _local_len(P, g)
     check_back(x.cpu().numpy(), oracle.back(g, sino, power=2), oracle.back(g, np.abs(sino), power=0),
                2.0 * diag * local, f"{name} power 2")
 
