@@ -70,20 +70,77 @@ def code_digest(paths):
     return h.hexdigest()
 
 
-def measured_traffic(kernel, workload_index):
-    """Per-launch DRAM bytes of `kernel` from the committed one-pass ncu
-    capture, or None when the capture is for another workload or the kernel
-    code has changed since it was taken."""
-    path = os.path.join(ROOT, "profiles", "dram_traffic_parallel512_900views.json")
+def kernel_counters(kernel, workload_index):
+    """Committed ncu counters of `kernel` (profiles/kernel_counters.json),
+    captured on a view subset of the workload: DRAM bytes and warp
+    instructions per launch there, and the ray-voxel updates of that subset.
+    None when the capture is for another workload or the kernel's code has
+    changed since it was taken (a digest of its sources without comments or
+    whitespace)."""
+    path = os.path.join(ROOT, "profiles", "kernel_counters.json")
     try:
         with open(path) as f:
             k = json.load(f)["kernels"][kernel]
         digest = code_digest(k["sources"])
     except Exception:
         return None
-    if digest != k.get("code_sha256") or workload_index != 4:
+    if digest != k.get("code_sha256") or workload_index != k.get("workload"):
         return None
-    return int(k["dram_bytes_per_launch"])
+    return k
+
+
+def measured_traffic(kernel, workload_index, n_views):
+    """DRAM bytes of one full launch: the small capture's bytes scaled by the
+    view count (each view's rays are an equal share of the work)."""
+    k = kernel_counters(kernel, workload_index)
+    if k is None:
+        return None
+    return int(round(k["dram_bytes"] * n_views / k["views"]))
+
+
+def issue_fraction(kernel, workload_index, updates_per_s, sm_mhz, n_sm):
+    """Achieved updates/s over the instruction-issue ceiling: every SM issues
+    at most one warp instruction per clock on each of its four schedulers, so
+    the ceiling is (SMs x 4 x clock) / (warp instructions per update), the
+    latter from the committed capture."""
+    k = kernel_counters(kernel, workload_index)
+    if k is None or not sm_mhz:
+        return None
+    ipu = k["warp_instructions"] / k["updates"]
+    ceiling = n_sm * 4 * sm_mhz * 1e6 / ipu
+    return {"frac": updates_per_s / ceiling, "warp_instructions_per_update": ipu,
+            "ceiling_gupdates_s": ceiling / 1e9, "sm_mhz": sm_mhz, "sms": n_sm}
+
+
+def kernel_names(info):
+    """Names of the step's forward and adjoint kernels for this plan."""
+    rows = info.get("slice_rows", 1) > 1
+    fwd = "forward_rows_kernel" if rows else "forward_kernel"
+    back = {1: "back_brick_kernel", 2: "back_sort_kernel",
+            3: "back_scatter_rows_kernel" if rows else "back_scatter_kernel"}[info["adjoint_variant"]]
+    return fwd, back
+
+
+def launches_per_step(info):
+    """Kernels of the library launched by one forward + one back projection
+    (memsets are not kernels of the library)."""
+    t = 1 if info["n_transposed_views"] > 0 else 0
+    fwd = 1 + t                       # transpose_xy + forward
+    back = 1 + (t if info["adjoint_variant"] == 3 else 0)   # + transpose_add for the scatter adjoint
+    return fwd + back
+
+
+def host_facts():
+    """The host the CPU baseline ran on: core count and CPU model."""
+    model = ""
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model}
 
 
 def algorithmic_bytes(U, n_vox, n_rays):
@@ -157,6 +214,26 @@ def throughput(updates_per_rank_step, world, ms_per_step):
     return world * updates_per_rank_step / (ms_per_step * 1e-3) / 1e9
 
 
+def cpu_oracle_parallel_sample(wl, n_views_sample):
+    """The FP64 oracle forward + back over an evenly spaced view subset, the
+    views split over one thread per host core (oracle/pool.py).
+    Returns (updates/s, wall seconds, updates, threads)."""
+    import oracle
+    from oracle import pool as oracle_pool
+    g = wl.geom
+    views = np.linspace(0, g.n_views - 1, n_views_sample).round().astype(np.int64)
+    gs = g.subset_views(views)
+    vol = np.random.default_rng(wl.seed).random(g.vol_shape, dtype=np.float32)
+    sino = np.random.default_rng(wl.seed + 1).random(gs.sino_shape, dtype=np.float32)
+    U = oracle.count_updates(gs)
+    threads = oracle_pool.host_threads()
+    t0 = time.perf_counter()
+    oracle_pool.forward(gs, vol, threads=threads)
+    oracle_pool.back(gs, sino, threads=threads)
+    dt = time.perf_counter() - t0
+    return 2 * U / dt, dt, 2 * U, threads
+
+
 def cpu_oracle_sample(wl, n_views_sample=1):
     """FP64 oracle forward + back over an evenly spaced subset of views, on one
     host core.  Returns (updates/s, seconds, updates, description)."""
@@ -205,7 +282,8 @@ def run_reference(args, rank, world):
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(wl),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
+                             "host": host_facts()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -491,47 +569,64 @@ def run_ours(args, rank, world, local_rank):
     if rank != 0:
         return 0
     peak, peak_kind = measured_hbm_peak()
+    wl_key = wl.index if not args.views else None
     if grad is not None:
         gb = algorithmic_bytes(U, g.n_vox, g.n_rays) / (grad["ms"] * 1e-3) / 1e9
         grad.update({"effective_gbs": gb, "frac_of_hbm": gb / peak,
-                     "traffic": measured_traffic("geometry_gradient_kernel", wl.index) if not args.views else None})
+                     "traffic": measured_traffic("geometry_gradient_kernel", wl_key, g.n_views)})
     B = algorithmic_bytes(U, g.n_vox, g.n_rays)
+    fwd_kernel, back_kernel = kernel_names(info)
     dominant = "back" if back_avg >= fwd_avg else "forward"
-    if dominant == "back":
-        dom_kernel = "back_sort_kernel" if info["adjoint_variant"] == 2 else "back_brick_kernel"
-    else:
-        dom_kernel = "forward_kernel"
+    dom_kernel = back_kernel if dominant == "back" else fwd_kernel
     dom_ms = max(back_avg, fwd_avg)
     achieved = B / (dom_ms * 1e-3) / 1e9
+    sm_mhz = (clk or {}).get("sm_mhz") or 1965.0
+    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+    issue_fwd = issue_fraction(fwd_kernel, wl_key, U / (fwd_avg * 1e-3), sm_mhz, n_sm)
+    issue_back = issue_fraction(back_kernel, wl_key, U / (back_avg * 1e-3), sm_mhz, n_sm)
+    dom_issue = issue_back if dominant == "back" else issue_fwd
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         v, dt, Ucpu, desc = cpu_oracle_sample(wl, 1)
         cpu = {"value": v / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
-               "seconds": round(dt, 2)}
+               "seconds": round(dt, 2), "host": host_facts()}
+        n_par = max(1, min(g.n_views, 2 * host_facts()["nproc"]))
+        vp, dtp, Up, threads = cpu_oracle_parallel_sample(wl, n_par)
+        cpu["all_cores"] = {"value": vp / 1e9, "unit": UNIT, "threads": threads, "seconds": round(dtp, 2),
+                            "sample": f"FP64 oracle forward + back of {n_par} of {g.n_views} views (evenly "
+                                      f"spaced), views split over {threads} host threads, {Up} updates",
+                            "whole_workload_seconds_estimate": round(2 * U / vp, 1)}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32 (fp64 ray setup)", "data": "synthetic",
         "config": workload_config(wl),
         "updates_per_direction": U,
-        "forward": {"ms": fwd_avg, "ms_median": fwd_med, "ms_min": fwd_min, "gupdates_s": U / (fwd_avg * 1e-3) / 1e9,
+        "forward": {"kernel": fwd_kernel, "ms": fwd_avg, "ms_median": fwd_med, "ms_min": fwd_min,
+                    "gupdates_s": U / (fwd_avg * 1e-3) / 1e9,
                     "views_s": g.n_views / (fwd_avg * 1e-3),
                     "effective_gbs": B / (fwd_avg * 1e-3) / 1e9,
-                    "frac_of_hbm": B / (fwd_avg * 1e-3) / 1e9 / peak},
-        "back": {"ms": back_avg, "ms_median": back_med, "ms_min": back_min, "gupdates_s": U / (back_avg * 1e-3) / 1e9,
+                    "frac_of_hbm": B / (fwd_avg * 1e-3) / 1e9 / peak,
+                    "issue": issue_fwd, "traffic": measured_traffic(fwd_kernel, wl_key, g.n_views),
+                    "slice_rows": info.get("slice_rows", 1)},
+        "back": {"kernel": back_kernel, "ms": back_avg, "ms_median": back_med, "ms_min": back_min,
+                 "gupdates_s": U / (back_avg * 1e-3) / 1e9,
                  "views_s": g.n_views / (back_avg * 1e-3),
                  "effective_gbs": B / (back_avg * 1e-3) / 1e9,
                  "frac_of_hbm": B / (back_avg * 1e-3) / 1e9 / peak,
-                 "variant": info["adjoint_variant"], "brick": info["brick"], "view_groups": info["view_groups"]},
+                 "issue": issue_back, "traffic": measured_traffic(back_kernel, wl_key, g.n_views),
+                 "variant": {1: "brick", 2: "sort", 3: "scatter"}[info["adjoint_variant"]],
+                 "collision_ratio": info["collision_ratio"], "slice_rows": info.get("slice_rows", 1)},
         "roofline": {"kernel": dom_kernel,
                      "bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs",
                      "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": measured_traffic(dom_kernel, wl.index) if not args.views else None,
-                     "algorithmic_bytes_per_launch": B},
+                     "traffic": measured_traffic(dom_kernel, wl_key, g.n_views),
+                     "algorithmic_bytes_per_launch": B,
+                     "issue_frac": dom_issue["frac"] if dom_issue else None},
         "geometry_gradient": grad,
         "clocks": clk,
         "e2e": e2e,
-        "gpu_launches": args.steps * (2 + (1 if info["n_transposed_views"] > 0 else 0)),
+        "gpu_launches": args.steps * launches_per_step(info),
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)

@@ -86,7 +86,10 @@ typedef struct {
   int32_t batch_chunk;       /* ctp_forward_batch: volumes per fused launch, 1, 2 or 4; 0 = 1.  The
                                 y-fastest scratch copy (if any view uses it) grows by this factor.
                                 2 or 4 also lets ctp_back_batch take member pairs in one launch. */
-  int32_t reserved[9];
+  int32_t slice_rows;        /* parallel beams whose rays lie in z-planes and whose rows step along z:
+                                detector rows that share one (x, y) path per thread, 2 or 4 (one walk
+                                serves that many slices); 1 = one walk per ray; 0 = automatic */
+  int32_t reserved[8];
 } ctp_plan;
 
 /* Acquisition and volume description.  All pointers are HOST pointers; the
@@ -117,7 +120,7 @@ typedef struct {
   int32_t n_transposed_views;   /* views whose forward gathers from the y-fastest copy */
   double collision_ratio;       /* updates / distinct voxels per sort batch, measured at create */
   int32_t batch_chunk;          /* volumes per fused ctp_forward_batch launch */
-  int32_t reserved;
+  int32_t slice_rows;           /* detector rows per shared (x, y) walk (1 = one walk per ray) */
 } ctp_geom_info;
 
 /*

@@ -1,8 +1,9 @@
 """The FP64 oracle over several host threads, for parity at full size.
 
-TEST INFRASTRUCTURE ONLY.  Each thread runs the unchanged single-threaded
-oracle (``oracle.forward`` / ``oracle.back``) on its own contiguous range of
-views; the C oracle keeps no global state and ctypes releases the GIL for the
+TEST INFRASTRUCTURE ONLY, like the rest of this package: the tests and the
+benchmark's CPU-baseline leg call it, the product library never does.  Each
+thread runs the unchanged single-threaded oracle (``forward`` / ``back`` of
+this package) on its own contiguous range of views; the C oracle keeps no global state and ctypes releases the GIL for the
 duration of each call, so the ranges run in parallel.  The forward
 concatenates the ranges' sinograms in view order; the back projection sums
 the ranges' FP64 partial volumes in range order, so the result does not
@@ -16,7 +17,7 @@ from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 
-import oracle
+from oracle import back as _back, forward as _forward
 
 
 def host_threads() -> int:
@@ -39,7 +40,7 @@ def forward(geom, vol, threads: int = 0) -> np.ndarray:
     vol = np.ascontiguousarray(vol, dtype=np.float32)
     ranges = _ranges(geom.n_views, 4 * threads)
     with ThreadPoolExecutor(threads) as ex:
-        parts = list(ex.map(lambda r: oracle.forward(geom, vol, views=r), ranges))
+        parts = list(ex.map(lambda r: _forward(geom, vol, views=r), ranges))
     return np.concatenate(parts, axis=0)
 
 
@@ -59,7 +60,7 @@ def back(geom, sino, power: int = 1, threads: int = 0, max_host_bytes: float = 0
     sino = np.ascontiguousarray(sino, dtype=np.float32)
     ranges = _ranges(geom.n_views, threads)
     with ThreadPoolExecutor(len(ranges)) as ex:
-        parts = list(ex.map(lambda r: oracle.back(geom, sino[r[0]:r[1]], views=r, power=power), ranges))
+        parts = list(ex.map(lambda r: _back(geom, sino[r[0]:r[1]], views=r, power=power), ranges))
     total = parts[0]
     for p in parts[1:]:
         total += p

@@ -83,14 +83,18 @@ bool invert_columns(const double *c0, const double *c1, const double *c2, double
   return true;
 }
 
-// The sort / segment-reduce adjoint replaces the brick adjoint when each
-// distinct voxel of a warp batch receives at least this many contributions
-// on average.  Measured on B200 (256^3 cone, 90 views, 384x384 detector,
-// magnification 2 / 4 / 8 / 16: ratios 1.5 / 2.6 / 4.4 / 5.3): the brick
-// adjoint is 3.4x / 2.3x faster at the first two, the sort adjoint 2.0x /
-// 5.0x faster at the last two.  Dense rays are also where the brick
-// adjoint's fixed-point step is coarsest (it grows with the rays per voxel).
-constexpr double kSortMinCollisionRatio = 3.4;
+// Adjoint variant dispatch (automatic plans): the ray-scatter adjoint unless
+// each distinct voxel of a warp batch receives at least this many
+// contributions on average, where the sort / segment-reduce adjoint takes
+// over.  Measured on B200 (256^3 cone, 90 views, 384x384 detector, source at
+// 500 voxels, magnification 2 / 4 / 8 / 16 / 32 / 64, collision ratios 1.5 /
+// 2.6 / 4.7 / 8.1 / 12.8 / 18.4): the scatter adjoint is 8.0x / 5.7x / 3.5x /
+// 2.0x / 1.10x faster than the sort adjoint at the first five and 1.78x
+// slower at the last; the crossover, interpolated log-linearly, sits at 13.5.
+// The brick adjoint was slower than the scatter adjoint at every one of these
+// points and on workloads 1-4 (and equal within 2 % on workload 0); it stays
+// available through the plan, for bitwise-reproducible results.
+constexpr double kSortMinCollisionRatio = 13.5;
 
 constexpr double kNearLimit = 1e6;  // one endpoint within this many voxels of the centre
 constexpr double kFarLimit = 1e15;  // both endpoints within this many voxels
@@ -160,6 +164,8 @@ ctp_status validate_desc(const ctp_geom_desc *d) {
     if (p->forward_layout < 0 || p->forward_layout > 2) return fail(CTP_ERR_INVALID_ARGUMENT, "plan.forward_layout");
     if (p->batch_chunk != 0 && p->batch_chunk != 1 && p->batch_chunk != 2 && p->batch_chunk != 4)
       return fail(CTP_ERR_INVALID_ARGUMENT, "plan.batch_chunk %d is not 0, 1, 2 or 4", p->batch_chunk);
+    if (p->slice_rows != 0 && p->slice_rows != 1 && p->slice_rows != 2 && p->slice_rows != 4)
+      return fail(CTP_ERR_INVALID_ARGUMENT, "plan.slice_rows %d is not 0, 1, 2 or 4", p->slice_rows);
   }
   return CTP_OK;
 }
@@ -539,6 +545,12 @@ ctp_status ctp_geom_create(const ctp_geom_desc *desc, ctp_geom **out) {
   f.n_row_bands = (int32_t)((g->n_rows + 7) / 8);
   f.any_transposed = g->n_transposed > 0;
   const ctp_plan *plan = desc->plan;
+  // Rays in z-planes whose rows step along z share one (x, y) walk per column.
+  bool slices = g->beam == CTP_BEAM_PARALLEL && g->det == CTP_DET_FLAT;
+  for (const ViewRec &V : views)
+    slices = slices && V.s[2] == 0.0 && V.dv[0] == 0.0 && V.dv[1] == 0.0;
+  f.row_group = 1;
+  f.row_group_bands = f.n_row_bands;
   g->adjoint_variant = CTP_ADJOINT_BRICK;
   g->batch_chunk = plan && plan->batch_chunk > 0 ? plan->batch_chunk : 1;
 
@@ -552,6 +564,25 @@ ctp_status ctp_geom_create(const ctp_geom_desc *desc, ctp_geom **out) {
     return s;
   }
   plan_back(g, plan, sm_count);
+  if (slices) {
+    // the largest row group that still launches two full waves of blocks
+    // (four resident per SM), unless the plan names one
+    const int want = plan ? plan->slice_rows : 0;
+    int rg = 1;
+    if (want > 0) {
+      rg = want;
+    } else {
+      for (int r : {4, 2}) {
+        const int64_t bands = (g->n_rows + 8 * r - 1) / (8 * r);
+        if (bands * g->n_views * f.n_col_tiles >= 2 * 4 * (int64_t)sm_count) {
+          rg = r;
+          break;
+        }
+      }
+    }
+    f.row_group = rg;
+    f.row_group_bands = (int32_t)((g->n_rows + 8 * rg - 1) / (8 * rg));
+  }
   if (ctp::back_brick_smem_bytes(g->back.brick) > 200 * 1024) {
     delete g;
     return fail(CTP_ERR_INVALID_ARGUMENT, "adjoint brick needs more than 200 KB of shared memory");
@@ -593,7 +624,7 @@ ctp_status ctp_geom_create(const ctp_geom_desc *desc, ctp_geom **out) {
   if (forced == CTP_ADJOINT_BRICK || forced == CTP_ADJOINT_SORT || forced == CTP_ADJOINT_SCATTER)
     g->adjoint_variant = forced;
   else
-    g->adjoint_variant = g->collision_ratio >= kSortMinCollisionRatio ? CTP_ADJOINT_SORT : CTP_ADJOINT_BRICK;
+    g->adjoint_variant = g->collision_ratio >= kSortMinCollisionRatio ? CTP_ADJOINT_SORT : CTP_ADJOINT_SCATTER;
   *out = g;
   return CTP_OK;
 }
@@ -616,7 +647,7 @@ ctp_status ctp_geom_query(const ctp_geom *g, ctp_geom_info *info) {
   info->n_transposed_views = g->n_transposed;
   info->collision_ratio = g->collision_ratio;
   info->batch_chunk = g->batch_chunk;
-  info->reserved = 0;
+  info->slice_rows = g->fwd.row_group;
   return CTP_OK;
 }
 
@@ -636,7 +667,10 @@ ctp_status ctp_forward(const ctp_geom *g, const float *vol, float *sino, void *s
     e = ctp::launch_transpose_xy(vol, g->d_volT, g->vol, s);
     if (e != cudaSuccess) return cuda_fail(e, "transpose launch");
   }
-  e = ctp::launch_forward(g->fwd, g->d_views, g->d_trig, vol, g->d_volT, sino, 1, g->wide_index, s);
+  if (g->fwd.row_group > 1)
+    e = ctp::launch_forward_rows(g->fwd, g->d_views, vol, g->d_volT, sino, g->wide_index, s);
+  else
+    e = ctp::launch_forward(g->fwd, g->d_views, g->d_trig, vol, g->d_volT, sino, 1, g->wide_index, s);
   if (e != cudaSuccess) return cuda_fail(e, "forward launch");
   return CTP_OK;
 }

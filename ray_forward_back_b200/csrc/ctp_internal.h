@@ -55,6 +55,11 @@ struct FwdLaunch {
   VolDesc vol;
   int32_t n_col_tiles, n_row_bands;
   int32_t any_transposed;
+  // Rays in z-planes with rows stepping along z: each thread walks one (x, y)
+  // path for row_group rows (1 = one walk per ray); row_group_bands bands of
+  // 8 * row_group rows.  Used by the single-volume forward and the scatter
+  // adjoint.
+  int32_t row_group, row_group_bands;
 };
 
 struct BackLaunch {
@@ -76,6 +81,9 @@ cudaError_t launch_forward(const FwdLaunch& p, const ViewRec* views, const doubl
                            const float* volT, float* sino, int kb, bool wide_index, cudaStream_t stream);
 // Brick adjoint of kb (1 or 2) batch members: sinograms at sino, sino + n_rays,
 // volumes at vol, vol + n_vox.
+// The single-volume forward with one (x, y) walk per p.row_group rows.
+cudaError_t launch_forward_rows(const FwdLaunch& p, const ViewRec* views, const float* vol, const float* volT,
+                                float* sino, bool wide_index, cudaStream_t stream);
 cudaError_t launch_back_brick(const BackLaunch& p, const ViewRec* views, const double* trig, const float* sino,
                               float* vol, int power, int kb, bool wide_index, cudaStream_t stream);
 cudaError_t launch_count(const FwdLaunch& p, const ViewRec* views, const double* trig,

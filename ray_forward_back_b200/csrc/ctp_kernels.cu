@@ -1222,9 +1222,174 @@ __global__ void __launch_bounds__(256) transpose_add_kernel(const float* __restr
   }
 }
 
+// ------------------------------------------ parallel slices: shared (x, y) walks --
+//
+// When every ray lies in a plane of constant z (a parallel beam whose
+// direction has no z component) and detector rows step along z only, the rays
+// of one detector column in one view all follow the same (x, y) path, each in
+// the slice of its own row (the slices decouple; MBIRJAX "Sharding overview",
+// section "Why cone beam").  A thread then sets up and walks that path once
+// for kR consecutive rows and applies every segment to the kR slices.  Each
+// row's FP64 set-up equals that of its own ray in the x and y components (the
+// pixel centres differ in z only), so every row sees exactly the segments,
+// in the same order, that a walk of its own ray would give.
+
+#ifndef CTP_ROWS_MIN_BLOCKS
+#define CTP_ROWS_MIN_BLOCKS 4
+#endif
+
+// Slice offsets of rows r0 .. r0 + kR - 1 of column c: bit j of the result is
+// set where row r0 + j exists and its rays' height falls inside the volume
+// (the z test of the ray's slab clip); zoff[j] is then that slice's offset.
+template <int kR, typename Off>
+__device__ __forceinline__ unsigned row_slices(const ViewRec& V, const VolDesc& G, int r0, int c, int n_rows, Off sz,
+                                               Off zoff[kR]) {
+  unsigned mask = 0u;
+#pragma unroll
+  for (int j = 0; j < kR; ++j) {
+    const int r = r0 + j;
+    // the z component of pixel_centre's flat-detector formula
+    const double pz = fma((double)r, V.dv[2], fma((double)c, V.du[2], V.p00[2]));
+    const double az = (pz - G.origin[2]) * G.inv_spacing[2];
+    const bool in = r < n_rows && az >= 0.0 && az < (double)G.n[2];
+    zoff[j] = in ? (Off)clampi((int)floor(az), 0, G.n[2] - 1) * sz : (Off)0;
+    mask |= in ? 1u << j : 0u;
+  }
+  return mask;
+}
+
+// Shared (x, y) set-up of column c: the ray of any row, lifted into the
+// volume's height (its direction has no z component, so only the x and y
+// slabs clip it) and walked as slice 0.
+__device__ __forceinline__ bool slice_ray(const ViewRec& V, const VolDesc& G, const Dims& dm, int v, int c, Ray& R,
+                                          double& t_in, double& t_out) {
+  make_ray(V, G, nullptr, dm, v, 0, c, R);
+  R.A[2] = 0.5;
+  const int lo[3] = {0, 0, 0};
+  const int hi[3] = {G.n[0], G.n[1], G.n[2]};
+  return clip(R, lo, hi, t_in, t_out);
+}
+
+template <typename Off, int kR>
+__global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_ROWS_MIN_BLOCKS)
+    forward_rows_kernel(FwdLaunch P, const ViewRec* __restrict__ views, const float* __restrict__ vol,
+                        const float* __restrict__ volT, float* __restrict__ sino) {
+  const int per_band = P.dims.n_views * P.n_col_tiles;
+  const int band = blockIdx.x / per_band;
+  const int rem = blockIdx.x - band * per_band;
+  const int v = rem / P.n_col_tiles;
+  const int ct = rem - v * P.n_col_tiles;
+  const int c = ct * kFwdCols + threadIdx.x;
+  const int r0 = (band * kFwdRows + threadIdx.y) * kR;
+  const bool cvalid = c < P.dims.n_cols;
+  const ViewRec& V = views[v];
+  const Off nx = P.vol.n[0], ny = P.vol.n[1];
+  const Off sz = nx * ny;
+  Off zoff[kR];
+  const unsigned rows = cvalid ? row_slices<kR, Off>(V, P.vol, r0, c, P.dims.n_rows, sz, zoff) : 0u;
+  Ray R;
+  double t_in = 0.0, t_out = 0.0;
+  const bool hit = slice_ray(V, P.vol, P.dims, v, cvalid ? c : 0, R, t_in, t_out) && rows != 0u;
+  const int lo[3] = {0, 0, 0};
+  const int hi[3] = {P.vol.n[0], P.vol.n[1], P.vol.n[2]};
+  Walk W = {};
+  if (hit) entry(R, t_in, t_out, lo, hi, W);
+  const bool yfast = V.layout != 0;
+  const float* __restrict__ base = yfast ? volT : vol;
+  const Off sx = yfast ? ny : (Off)1;
+  const Off sy = yfast ? (Off)1 : nx;
+  const Off off = (Off)W.i[1] * sy + (Off)W.i[0] * sx;
+  float acc[kR];
+#pragma unroll
+  for (int j = 0; j < kR; ++j) acc[j] = 0.f;
+  walk<true, false, 0, Off>(hit, W, lo, hi, off, W.step[0] * sx, W.step[1] * sy, (Off)0, nullptr,
+                            [&](Off o, float len, bool) {
+#pragma unroll
+                              for (int j = 0; j < kR; ++j)
+                                if (rows & (1u << j)) acc[j] = fmaf(len, __ldg(base + o + zoff[j]), acc[j]);
+                            });
+  if (cvalid) {
+#pragma unroll
+    for (int j = 0; j < kR; ++j) {
+      const int r = r0 + j;
+      if (r < P.dims.n_rows) sino[((size_t)v * P.dims.n_rows + r) * P.dims.n_cols + c] = acc[j];
+    }
+  }
+}
+
+template <int kPower, typename Off, int kR>
+__global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_ROWS_MIN_BLOCKS)
+    back_scatter_rows_kernel(FwdLaunch P, const ViewRec* __restrict__ views, const float* __restrict__ sino,
+                             float* __restrict__ vol, float* __restrict__ volT) {
+  const int per_band = P.dims.n_views * P.n_col_tiles;
+  const int band = blockIdx.x / per_band;
+  const int rem = blockIdx.x - band * per_band;
+  const int v = rem / P.n_col_tiles;
+  const int ct = rem - v * P.n_col_tiles;
+  const int c = ct * kFwdCols + threadIdx.x;
+  const int r0 = (band * kFwdRows + threadIdx.y) * kR;
+  const bool cvalid = c < P.dims.n_cols;
+  const ViewRec& V = views[v];
+  const Off nx = P.vol.n[0], ny = P.vol.n[1];
+  const Off sz = nx * ny;
+  Off zoff[kR];
+  unsigned rows = cvalid ? row_slices<kR, Off>(V, P.vol, r0, c, P.dims.n_rows, sz, zoff) : 0u;
+  float y[kR];
+#pragma unroll
+  for (int j = 0; j < kR; ++j) {
+    y[j] = (rows & (1u << j)) ? __ldg(sino + ((size_t)v * P.dims.n_rows + r0 + j) * P.dims.n_cols + c) : 0.f;
+    if (!(y[j] != 0.f)) rows &= ~(1u << j);  // zero rows add nothing (NaN stays)
+  }
+  Ray R;
+  double t_in = 0.0, t_out = 0.0;
+  const bool hit = slice_ray(V, P.vol, P.dims, v, cvalid ? c : 0, R, t_in, t_out) && rows != 0u;
+  const int lo[3] = {0, 0, 0};
+  const int hi[3] = {P.vol.n[0], P.vol.n[1], P.vol.n[2]};
+  Walk W = {};
+  __shared__ double s_anc[7 * kAncStride];
+  double* const anc = s_anc + threadIdx.y * kFwdCols + threadIdx.x;
+  if (hit) entry(R, t_in, t_out, lo, hi, W, anc, kAncStride);
+  const bool yfast = V.layout != 0;
+  float* const base = yfast ? volT : vol;
+  const Off sx = yfast ? ny : (Off)1;
+  const Off sy = yfast ? (Off)1 : nx;
+  const Off off = (Off)W.i[1] * sy + (Off)W.i[0] * sx;
+  walk<true, false, kWalkAnchor, Off>(hit, W, lo, hi, off, W.step[0] * sx, W.step[1] * sy, (Off)0, anc,
+                                      [&](Off o, float len, bool) {
+                                        if (len > 0.f) {
+                                          const float w = coef<kPower>(len);
+#pragma unroll
+                                          for (int j = 0; j < kR; ++j)
+                                            if (rows & (1u << j)) atomicAdd(base + o + zoff[j], w * y[j]);
+                                        }
+                                      });
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------- launchers --
+
+cudaError_t launch_forward_rows(const FwdLaunch& p, const ViewRec* views, const float* vol, const float* volT,
+                                float* sino, bool wide_index, cudaStream_t stream) {
+  const long long blocks = (long long)p.row_group_bands * p.dims.n_views * p.n_col_tiles;
+  if (blocks <= 0) return cudaSuccess;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  dim3 block(kFwdCols, kFwdRows);
+  const unsigned nb = (unsigned)blocks;
+#define CTP_ROWS_LAUNCH(OFF, R) forward_rows_kernel<OFF, R><<<nb, block, 0, stream>>>(p, views, vol, volT, sino)
+  switch (p.row_group) {
+    case 2:
+      if (wide_index) CTP_ROWS_LAUNCH(long long, 2); else CTP_ROWS_LAUNCH(int, 2);
+      break;
+    case 4:
+      if (wide_index) CTP_ROWS_LAUNCH(long long, 4); else CTP_ROWS_LAUNCH(int, 4);
+      break;
+    default:
+      return cudaErrorInvalidValue;
+  }
+#undef CTP_ROWS_LAUNCH
+  return cudaGetLastError();
+}
 
 cudaError_t launch_back_scatter(const FwdLaunch& p, const ViewRec* views, const double* trig, const float* sino,
                                 float* vol, float* volT, int power, bool wide_index, cudaStream_t stream) {
@@ -1233,7 +1398,28 @@ cudaError_t launch_back_scatter(const FwdLaunch& p, const ViewRec* views, const 
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   dim3 block(kFwdCols, kFwdRows);
   const unsigned nb = (unsigned)blocks;
-  if (power == 2) {
+  if (p.row_group > 1) {
+    const long long rb = (long long)p.row_group_bands * p.dims.n_views * p.n_col_tiles;
+    if (rb > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    const unsigned nr = (unsigned)rb;
+#define CTP_SROWS(KP, OFF, R) back_scatter_rows_kernel<KP, OFF, R><<<nr, block, 0, stream>>>(p, views, sino, vol, volT)
+    if (p.row_group == 4) {
+      if (power == 2) {
+        if (wide_index) CTP_SROWS(2, long long, 4); else CTP_SROWS(2, int, 4);
+      } else {
+        if (wide_index) CTP_SROWS(1, long long, 4); else CTP_SROWS(1, int, 4);
+      }
+    } else if (p.row_group == 2) {
+      if (power == 2) {
+        if (wide_index) CTP_SROWS(2, long long, 2); else CTP_SROWS(2, int, 2);
+      } else {
+        if (wide_index) CTP_SROWS(1, long long, 2); else CTP_SROWS(1, int, 2);
+      }
+    } else {
+      return cudaErrorInvalidValue;
+    }
+#undef CTP_SROWS
+  } else if (power == 2) {
     if (wide_index) back_scatter_kernel<2, long long><<<nb, block, 0, stream>>>(p, views, trig, sino, vol, volT);
     else back_scatter_kernel<2, int><<<nb, block, 0, stream>>>(p, views, trig, sino, vol, volT);
   } else {

@@ -45,7 +45,7 @@ CTP_SOLVER_SIRT = 2
 class ctp_plan(ctypes.Structure):
     _fields_ = [("adjoint_variant", ctypes.c_int32), ("brick", ctypes.c_int32 * 3),
                 ("view_groups", ctypes.c_int32), ("forward_layout", ctypes.c_int32),
-                ("batch_chunk", ctypes.c_int32), ("reserved", ctypes.c_int32 * 9)]
+                ("batch_chunk", ctypes.c_int32), ("slice_rows", ctypes.c_int32), ("reserved", ctypes.c_int32 * 8)]
 
 
 class ctp_geom_desc(ctypes.Structure):
@@ -64,7 +64,7 @@ class ctp_geom_info(ctypes.Structure):
                 ("adjoint_variant", ctypes.c_int32), ("brick", ctypes.c_int32 * 3),
                 ("view_groups", ctypes.c_int32), ("n_transposed_views", ctypes.c_int32),
                 ("collision_ratio", ctypes.c_double), ("batch_chunk", ctypes.c_int32),
-                ("reserved", ctypes.c_int32)]
+                ("slice_rows", ctypes.c_int32)]
 
 
 class ctp_solver_options(ctypes.Structure):
@@ -190,6 +190,7 @@ class _Desc:
             p.view_groups = int(plan.get("view_groups", 0))
             p.forward_layout = int(plan.get("forward_layout", 0))
             p.batch_chunk = int(plan.get("batch_chunk", 0))
+            p.slice_rows = int(plan.get("slice_rows", 0))
             self.plan = p
             d.plan = ctypes.pointer(p)
         self.desc = d
@@ -215,7 +216,7 @@ def ctp_geom_query(handle: int) -> dict:
     return {"n_rays": info.n_rays, "n_vox": info.n_vox, "scratch_bytes": info.scratch_bytes,
             "adjoint_variant": info.adjoint_variant, "brick": tuple(info.brick), "view_groups": info.view_groups,
             "n_transposed_views": info.n_transposed_views, "collision_ratio": info.collision_ratio,
-            "batch_chunk": info.batch_chunk}
+            "batch_chunk": info.batch_chunk, "slice_rows": info.slice_rows}
 
 
 def ctp_forward(handle: int, vol, sino, stream=None) -> None:

@@ -118,6 +118,8 @@ def test_bad_plan(lib):
     _expect(ctp.CTP_ERR_INVALID_ARGUMENT, _cone(), {"brick": (0, -1, 0)})
     for chunk in (-1, 3, 8):
         _expect(ctp.CTP_ERR_INVALID_ARGUMENT, _cone(), {"batch_chunk": chunk})
+    for rows in (-1, 3, 8):
+        _expect(ctp.CTP_ERR_INVALID_ARGUMENT, _cone(), {"slice_rows": rows})
 
 
 def test_valid_geometry_without_a_gpu_fails_with_cuda_status(lib):

@@ -1,10 +1,10 @@
-"""The threaded oracle driver (tests/oracle_pool.py) against the plain
+"""The threaded oracle driver (oracle/pool.py) against the plain
 single-threaded oracle: the forward is the same ray by ray, the back
 projection the same up to the order in which view ranges are summed."""
 import numpy as np
 
 import oracle
-from tests import oracle_pool
+from oracle import pool as oracle_pool
 from tests.helpers import small_geometries
 
 

@@ -7,7 +7,7 @@ configuration of the whole workload (the brick and view groups the full
 geometry plans are forced on the subset).  The whole sinogram of the
 workload's phantom and the back projection of a dense U[0, 1) sinogram are
 compared with the FP64 oracle, run over the host's cores by
-``tests/oracle_pool.py``.  Every adjoint variant (brick, sort, scatter) is
+``oracle/pool.py``.  Every adjoint variant (brick, sort, scatter) is
 checked against the same oracle volume.
 
 Tolerances (the required bounds):
@@ -26,7 +26,7 @@ import numpy as np
 import pytest
 
 from ray_forward_back_b200 import workloads as W
-from tests import oracle_pool
+from oracle import pool as oracle_pool
 from tests.gpu_helpers import back_errors, forward_errors, gpu_back, gpu_forward, projector
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]

@@ -37,9 +37,12 @@ def test_single_rank_nccl_sharded_equals_projector():
         sino = torch.rand(g.sino_shape, device=dev)
         assert torch.equal(S.forward(vol), P.forward(vol))
         x_ref = P.back(sino)
-        assert torch.equal(S.back(sino), x_ref)
+        # the adjoint adds FP32 contributions in whatever order the atomics land
+        tol = dict(rtol=1e-5, atol=1e-6 * float(x_ref.abs().max()))
+        torch.testing.assert_close(S.back(sino), x_ref, **tol)
         z0, z1, slab = S.back_slab(sino)
-        assert (z0, z1) == (0, g.nz) and torch.equal(slab, x_ref)
+        assert (z0, z1) == (0, g.nz)
+        torch.testing.assert_close(slab, x_ref, **tol)
         torch.cuda.synchronize()
     finally:
         dist.destroy_process_group()
@@ -50,8 +53,7 @@ def test_slice_sharded_gpu_projection_equals_the_whole(world):
     """Slice sharding (no collective): ranks emulated one after another on
     this GPU.  The forward rows are bit-identical to the whole-volume
     forward (the rays' x-y walks are the same); the adjoint slabs agree to
-    FP32 accumulation (the brick adjoint's per-stage scale may see a
-    slightly different set of footprint rays)."""
+    FP32 accumulation order."""
     import torch
     from ray_forward_back_b200 import workloads as W
     from ray_forward_back_b200.sharded import SliceShardedProjector
