@@ -5,11 +5,15 @@
 A step is one forward projection and one back projection of the workload
 (default: parallel beam, 512^3 volume, 900 views, 512x736 detector), inputs
 resident in HBM.  value = (forward updates + back updates) / step time, in
-Gupdates/s (ray-voxel updates), summed over ranks; with N > 1 every rank runs
-its own copy of the workload (independent problems, weak scaling, no
-collective on the data path).  Rank 0 prints one JSON line.  The geometry
-gradient is timed on its own after the step and reported
-under "geometry_gradient"; it is not part of the step.
+Gupdates/s (ray-voxel updates).  With N > 1 processes (one per GPU) the
+workload is split (strong scaling): --split views (the default) shards the
+views, the adjoint's partial volumes reduce-scattered by NCCL into z-slabs;
+--split slices shards z-slabs with their detector rows where the slices
+decouple (no collective); --split replicas runs a whole copy per rank
+(independent problems, weak scaling).  Timings are CUDA events, max over
+ranks; rank 0 prints one JSON line.  The geometry gradient is timed on its
+own after the single-GPU step and reported under "geometry_gradient"; it is
+not part of the step.
 
 --impl reference times the FP64 CPU oracle on a bounded sample of the same
 workload (the reference arm; slow by design).  --solver cgls|sirt prints the
@@ -633,6 +637,165 @@ def run_ours(args, rank, world, local_rank):
     return 0
 
 
+def run_sharded(args, rank, world, local_rank):
+    """The workload split over `world` GPUs, one process each (strong
+    scaling: the job is the whole workload).
+
+    --split views: each rank projects a balanced contiguous shard of the
+    views; the forward needs no collective (the volume is replicated); the
+    adjoint back-projects the rank's views into a partial volume that NCCL
+    reduce-scatters into z-slabs, one per rank.  --split slices (geometries
+    whose slices decouple, as workload 4's): each rank owns a z-slab of the
+    volume and the detector rows that fall in it; no collective at all.
+    Every timing is CUDA events on the rank's stream, then the max over
+    ranks; value = all updates of the workload / the slowest rank's step."""
+    import torch
+    import torch.distributed as dist
+
+    from ray_forward_back_b200 import ctp
+    from ray_forward_back_b200.sharded import ShardedProjector, SliceShardedProjector
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = select_workload(args)
+    g = wl.geom
+    make = lambda geom: ctp.Projector(geom, device=local_rank)
+    stream = torch.cuda.Stream(device=dev)
+    vol_host = wl.phantom()
+    sino_host = wl.sinogram()
+    if args.split == "views":
+        S = ShardedProjector(g, device=local_rank, make_projector=make)
+        vol_in = vol_host                                   # replicated
+        sino_part = sino_host[S.v0:S.v1]
+        scaling = "strong (view shards + reduce-scatter)"
+        shard = {"views": [S.v0, S.v1]}
+    else:
+        S = SliceShardedProjector(g, make_projector=make)
+        vol_in = vol_host[S.z0:S.z1]
+        sino_part = sino_host[:, S.r0:S.r1]
+        scaling = "strong (slice shards, no collective)"
+        shard = {"slices": [S.z0, S.z1], "rows": [S.r0, S.r1]}
+    with torch.cuda.stream(stream):
+        vol = torch.from_numpy(np.ascontiguousarray(vol_in)).to(dev)
+        sino = torch.from_numpy(np.ascontiguousarray(sino_part)).to(dev)
+    stream.synchronize()
+    U_local = S.local.count_updates(stream=stream) if S.local is not None else 0
+    t = torch.tensor([float(U_local)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    U = int(round(t.item()))
+    info = S.local.info() if S.local is not None else None
+
+    def step(ev=None):
+        with torch.cuda.stream(stream):
+            if ev:
+                ev[0].record(stream)
+            y = S.forward(vol)
+            if ev:
+                ev[1].record(stream)
+            if args.split == "views":
+                part = S._partial_back(sino, dev)
+                if ev:
+                    ev[2].record(stream)
+                nz, ny, nx = g.vol_shape
+                from ray_forward_back_b200.sharded import z_slab
+                z0, z1, h = z_slab(nz, S.rank, S.world)
+                if h * S.world != nz:
+                    padded = torch.zeros((h * S.world, ny, nx), dtype=part.dtype, device=dev)
+                    padded[:nz] = part
+                    part = padded
+                out = torch.empty((h, ny, nx), dtype=part.dtype, device=dev)
+                dist.reduce_scatter_tensor(out, part, op=dist.ReduceOp.SUM)
+            else:
+                out = S.back(sino)
+                if ev:
+                    ev[2].record(stream)
+            if ev:
+                ev[3].record(stream)
+        return y, out
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    clocks = ClockSampler(local_rank)
+    if rank == 0:
+        clocks.start()
+        time.sleep(0.3)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    start.record(stream)
+    for k in range(args.steps):
+        step(ev[k])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    clk = clocks.stop() if rank == 0 else None
+    # end to end: every step copies this rank's inputs in from pinned host
+    # memory and its outputs (sinogram shard, volume slab) back out
+    e2e = None
+    if not args.no_e2e:
+        vin = torch.from_numpy(np.ascontiguousarray(vol_in)).pin_memory()
+        sin = torch.from_numpy(np.ascontiguousarray(sino_part)).pin_memory()
+        y0, x0 = step()
+        yout = torch.empty(tuple(y0.shape), dtype=torch.float32).pin_memory()
+        xout = torch.empty(tuple(x0.shape), dtype=torch.float32).pin_memory()
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            with torch.cuda.stream(stream):
+                vol.copy_(vin, non_blocking=True)
+                sino.copy_(sin, non_blocking=True)
+            yk, xk = step()
+            with torch.cuda.stream(stream):
+                yout.copy_(yk, non_blocking=True)
+                xout.copy_(xk, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = aggregate_over_ranks([e0.elapsed_time(e1) / args.steps], world, dev)[0]
+        e2e = {"value": 2 * U / (e2e_ms * 1e-3) / 1e9, "unit": UNIT, "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": int(4 * (vin.numel() + sin.numel())),
+               "d2h_bytes_per_step": int(4 * (yout.numel() + xout.numel())),
+               "pipelining": "none: copies and projections in order on one stream per rank; bytes of rank 0"}
+    fwd = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
+    back = float(np.mean([e[1].elapsed_time(e[2]) for e in ev]))
+    coll = float(np.mean([e[2].elapsed_time(e[3]) for e in ev]))
+    total, fwd, back, coll = aggregate_over_ranks([start.elapsed_time(end), fwd, back, coll], world, dev)
+    ms_per_step = total / args.steps
+    if rank != 0:
+        return 0
+    n_vox_local = int(np.prod(vol.shape))
+    B_local = algorithmic_bytes(U / world, n_vox_local, g.n_rays / world)
+    peak, peak_kind = measured_hbm_peak()
+    dom_ms = max(fwd, back)
+    fwd_kernel, back_kernel = kernel_names(info) if info else ("forward_kernel", "back_scatter_kernel")
+    line = {
+        "metric": METRIC, "value": 2 * U / (ms_per_step * 1e-3) / 1e9, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": scaling, "vs_baseline": None, "dtype": "f32 (fp64 ray setup)", "data": "synthetic",
+        "config": dict(workload_config(wl), split=args.split, parallelism=f"{args.split} x{world}"),
+        "updates_per_direction": U,
+        "per_rank_max": {"forward_ms": fwd, "back_kernel_ms": back, "collective_ms": coll,
+                         "rank0_shard": shard,
+                         "collective_bytes_per_rank": int(4 * g.n_vox * (world - 1) / world)
+                         if args.split == "views" else 0},
+        "roofline": {"kernel": back_kernel if back >= fwd else fwd_kernel, "bound": "hbm",
+                     "achieved": B_local / (dom_ms * 1e-3) / 1e9, "peak": peak,
+                     "peak_kind": f"{peak_kind} hbm_gbs", "unit": "GB/s",
+                     "frac": B_local / (dom_ms * 1e-3) / 1e9 / peak, "traffic": None,
+                     "algorithmic_bytes_per_launch": B_local},
+        "clocks": clk, "e2e": e2e,
+        "gpu_launches": args.steps * (launches_per_step(info) if info else 0),
+        "cpu_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -649,13 +812,19 @@ def main():
                     help="time the batched calls on this many members against single calls instead")
     ap.add_argument("--solver", choices=["cgls", "sirt"], default=None,
                     help="time solver iterations (against one forward + back) instead of the projector step")
+    ap.add_argument("--split", choices=["views", "slices", "replicas"], default=None,
+                    help="with several processes: view shards + reduce-scatter (default), z-slab shards "
+                         "(slices that decouple), or independent replicas of the whole workload")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank, world)
-    if world > 1:
+    split = args.split or ("views" if world > 1 else "replicas")
+    args.split = split
+    grouped = world > 1 or (split != "replicas" and "RANK" in os.environ)
+    if grouped:
         import datetime
 
         import torch
@@ -668,9 +837,11 @@ def main():
             return run_solver(args, rank, world, local_rank)
         if args.batch > 0:
             return run_batch(args, rank, world, local_rank)
+        if split != "replicas" and grouped:
+            return run_sharded(args, rank, world, local_rank)
         return run_ours(args, rank, world, local_rank)
     finally:
-        if world > 1:
+        if grouped:
             import torch.distributed as dist
             dist.destroy_process_group()
 

@@ -87,7 +87,7 @@ typedef struct {
                                 y-fastest scratch copy (if any view uses it) grows by this factor.
                                 2 or 4 also lets ctp_back_batch take member pairs in one launch. */
   int32_t slice_rows;        /* parallel beams whose rays lie in z-planes and whose rows step along z:
-                                detector rows that share one (x, y) path per thread, 2 or 4 (one walk
+                                detector rows that share one (x, y) path per thread, 2, 4 or 8 (one walk
                                 serves that many slices); 1 = one walk per ray; 0 = automatic */
   int32_t reserved[8];
 } ctp_plan;
@@ -254,13 +254,19 @@ ctp_status ctp_count_updates(const ctp_geom *geom, int64_t *host_out, void *stre
  * some view's detector columns run mostly along y) exceed that size is
  * rejected with CTP_ERR_OUT_OF_RANGE and a detail message giving the sizes.
  *
- * The first call on a device looks the array's device address up
- * (cudaGetSymbolAddress); make that first call before any stream capture.
- * The records are copied from host stack memory with cudaMemcpyAsync, so the
- * call may wait for earlier work on `stream` before returning.  All calls on a
- * device share the one array and it keeps the last call's contents: calls
- * that overlap on the GPU (different streams, or different host threads) race
- * and corrupt each other's results; serialise them on one stream.
+ * Every call looks the array's device address up on the current device
+ * (cudaGetSymbolAddress, which allocates nothing), so the address is never
+ * stale, even after the caller resets the device.  The records and column
+ * rows are copied with cudaMemcpyAsync from host memory of this call (a
+ * stack buffer and a static staging array, not the heap), so the call may
+ * wait for earlier work on `stream` before returning; for the same reason it
+ * returns CTP_ERR_UNSUPPORTED, enqueuing nothing, while `stream` is being
+ * captured into a graph (a replay would copy from memory the call no longer
+ * owns).  All calls on a device share the one array and it keeps the last
+ * call's contents: calls that overlap on the GPU (different streams, or
+ * different host threads) race and corrupt each other's results; serialise
+ * them on one stream (host threads are serialised inside the call, the GPU
+ * work they enqueue is not).
  * vol, sino: as for ctp_forward.  The plan's forward_layout is honoured; the
  * other plan fields do not apply.
  */
@@ -308,6 +314,21 @@ size_t ctp_solver_workspace_bytes(const ctp_geom *geom, int32_t method);
 ctp_status ctp_solve(const ctp_geom *geom, const float *sino, float *vol, const ctp_solver_options *opts,
                      void *workspace, size_t workspace_bytes, double *history, ctp_solver_result *result,
                      void *stream);
+
+/*
+ * ctp_debug_error_word — the bounds-check record of a CTP_DEBUG build of this
+ * library (built with -DCTP_DEBUG; a test and diagnosis build, not the
+ * default).  In that build every global and shared-memory index of the
+ * projector kernels is checked against its array's extent before the
+ * access; a failing index is recorded (site number in the top 16 bits, the
+ * index in the low 48) and the access skipped, and the next ctp_forward /
+ * ctp_back / ctp_back_power / ctp_forward_batch / ctp_geometry_gradient call
+ * returns CTP_ERR_OUT_OF_RANGE.  This call waits for the device, stores the
+ * record (0 if every index was in bounds) in *word and clears it.
+ * Other builds: *word = 0 and CTP_ERR_UNSUPPORTED.  The pages have no
+ * counterpart; this is the library's memory-safety check.
+ */
+ctp_status ctp_debug_error_word(uint64_t *word);
 
 /* Static description of a status code. */
 const char *ctp_status_string(ctp_status status);

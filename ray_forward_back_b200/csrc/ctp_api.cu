@@ -5,6 +5,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -164,8 +165,8 @@ ctp_status validate_desc(const ctp_geom_desc *d) {
     if (p->forward_layout < 0 || p->forward_layout > 2) return fail(CTP_ERR_INVALID_ARGUMENT, "plan.forward_layout");
     if (p->batch_chunk != 0 && p->batch_chunk != 1 && p->batch_chunk != 2 && p->batch_chunk != 4)
       return fail(CTP_ERR_INVALID_ARGUMENT, "plan.batch_chunk %d is not 0, 1, 2 or 4", p->batch_chunk);
-    if (p->slice_rows != 0 && p->slice_rows != 1 && p->slice_rows != 2 && p->slice_rows != 4)
-      return fail(CTP_ERR_INVALID_ARGUMENT, "plan.slice_rows %d is not 0, 1, 2 or 4", p->slice_rows);
+    if (p->slice_rows != 0 && p->slice_rows != 1 && p->slice_rows != 2 && p->slice_rows != 4 && p->slice_rows != 8)
+      return fail(CTP_ERR_INVALID_ARGUMENT, "plan.slice_rows %d is not 0, 1, 2, 4 or 8", p->slice_rows);
   }
   return CTP_OK;
 }
@@ -465,6 +466,31 @@ ctp_status measure_collision_ratio(ctp_geom *g, const std::vector<ViewRec> &view
 
 }  // namespace
 
+// CTP_DEBUG builds: a bounds check that failed in an earlier kernel makes the
+// next call return CTP_ERR_OUT_OF_RANGE (the record stays until
+// ctp_debug_error_word reads and clears it).  Synchronous in those builds only.
+#ifdef CTP_DEBUG
+std::mutex g_debug_mu;
+unsigned long long g_debug_pending = 0;
+
+unsigned long long debug_collect() {
+  std::lock_guard<std::mutex> lock(g_debug_mu);
+  if (!g_debug_pending) g_debug_pending = ctp::debug_take_word_kernels();
+  if (!g_debug_pending) g_debug_pending = ctp::debug_take_word_grad();
+  return g_debug_pending;
+}
+#endif
+
+ctp_status debug_check() {
+#ifdef CTP_DEBUG
+  const unsigned long long w = debug_collect();
+  if (w)
+    return fail(CTP_ERR_OUT_OF_RANGE, "bounds check failed in an earlier kernel: site %llu, index %llu", w >> 48,
+                w & 0xffffffffffffull);
+#endif
+  return CTP_OK;
+}
+
 // Host helpers shared with the entry point that allocates nothing
 // (ctp_noalloc.cu); thin wrappers over the functions above.
 namespace ctp {
@@ -480,7 +506,22 @@ void host_clear_error() { g_detail[0] = '\0'; }
 
 extern "C" {
 
-const char *ctp_version(void) { return "0.1.0"; }
+const char *ctp_version(void) { return "0.2.0"; }
+
+ctp_status ctp_debug_error_word(uint64_t *word) {
+  g_detail[0] = '\0';
+  if (!word) return fail(CTP_ERR_INVALID_ARGUMENT, "word is NULL");
+#ifdef CTP_DEBUG
+  debug_collect();
+  std::lock_guard<std::mutex> lock(g_debug_mu);
+  *word = (uint64_t)g_debug_pending;
+  g_debug_pending = 0;
+  return CTP_OK;
+#else
+  *word = 0;
+  return fail(CTP_ERR_UNSUPPORTED, "bounds checks are compiled only into CTP_DEBUG builds");
+#endif
+}
 
 const char *ctp_status_string(ctp_status s) {
   switch (s) {
@@ -660,6 +701,10 @@ ctp_status ctp_forward(const ctp_geom *g, const float *vol, float *sino, void *s
     return fail(CTP_ERR_INVALID_ARGUMENT, "vol is not device memory of device %d", g->device);
   if (!is_device_pointer(sino, g->device))
     return fail(CTP_ERR_INVALID_ARGUMENT, "sino is not device memory of device %d", g->device);
+  {
+    const ctp_status dbg = debug_check();
+    if (dbg != CTP_OK) return dbg;
+  }
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pending error before ctp_forward");
@@ -696,6 +741,10 @@ ctp_status ctp_forward_batch(const ctp_geom *g, const float *vol, float *sino, i
     return fail(CTP_ERR_INVALID_ARGUMENT, "vol is not device memory of device %d", g->device);
   if (!is_device_pointer(sino, g->device))
     return fail(CTP_ERR_INVALID_ARGUMENT, "sino is not device memory of device %d", g->device);
+  {
+    const ctp_status dbg = debug_check();
+    if (dbg != CTP_OK) return dbg;
+  }
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pending error before ctp_forward_batch");
@@ -764,6 +813,10 @@ ctp_status ctp_back_power(const ctp_geom *g, const float *sino, float *vol, int 
     return fail(CTP_ERR_INVALID_ARGUMENT, "sino is not device memory of device %d", g->device);
   if (!is_device_pointer(vol, g->device))
     return fail(CTP_ERR_INVALID_ARGUMENT, "vol is not device memory of device %d", g->device);
+  {
+    const ctp_status dbg = debug_check();
+    if (dbg != CTP_OK) return dbg;
+  }
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pending error before ctp_back");
@@ -794,6 +847,10 @@ ctp_status ctp_geometry_gradient(const ctp_geom *g, const float *vol, const floa
   if (!is_device_pointer(vol, g->device) || !is_device_pointer(sino_grad, g->device) ||
       !is_device_pointer(grad, g->device))
     return fail(CTP_ERR_INVALID_ARGUMENT, "vol, sino_grad and grad must be device memory of device %d", g->device);
+  {
+    const ctp_status dbg = debug_check();
+    if (dbg != CTP_OK) return dbg;
+  }
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pending error before ctp_geometry_gradient");

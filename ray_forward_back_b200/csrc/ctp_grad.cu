@@ -111,7 +111,8 @@ __device__ __forceinline__ bool clip_faces(const Ray& R, const int hi[3], double
 template <typename Off>
 __device__ __forceinline__ float crossing_sums(bool active, const Walk& W, const int hi[3],
                                                const float* __restrict__ vol, Off off, Off s0, Off s1, Off s2,
-                                               float x0, float S0[3], float Sl[3]) {
+                                               float x0, float S0[3], float Sl[3],
+                                               [[maybe_unused]] long long n_vox) {
   constexpr unsigned kFull = 0xffffffffu;
   int a, b, c;
   walk_axes(W, a, b, c);
@@ -154,9 +155,9 @@ __device__ __forceinline__ float crossing_sums(bool active, const Walk& W, const
         const float m1 = fmaxf(fminf(tb, tx), cur);
         const Off o2 = off + (cb ? sb : (Off)0);
         float x1 = x0;
-        if (cb) x1 = __ldg(vol + o2);
+        if (cb && CTP_IN_BOUNDS(o2, n_vox, 13)) x1 = __ldg(vol + o2);
         float x2 = x1;
-        if (ona) x2 = __ldg(vol + o2 + sa);
+        if (ona && CTP_IN_BOUNDS(o2 + sa, n_vox, 13)) x2 = __ldg(vol + o2 + sa);
         const float d1 = x0 - x1, d2 = x1 - x2;
         S0b += d1;
         Slb = fmaf(d1, m1, Slb);
@@ -188,11 +189,11 @@ __device__ __forceinline__ float crossing_sums(bool active, const Walk& W, const
         const Off o2 = off + (bfirst ? db : dc);
         const Off o3 = off + db + dc;
         float x1 = x0;
-        if (cb || cc) x1 = __ldg(vol + o2);
+        if ((cb || cc) && CTP_IN_BOUNDS(o2, n_vox, 13)) x1 = __ldg(vol + o2);
         float x2 = x1;
-        if (cb && cc) x2 = __ldg(vol + o3);
+        if (cb && cc && CTP_IN_BOUNDS(o3, n_vox, 13)) x2 = __ldg(vol + o3);
         float x3 = x2;
-        if (ona) x3 = __ldg(vol + o3 + sa);
+        if (ona && CTP_IN_BOUNDS(o3 + sa, n_vox, 13)) x3 = __ldg(vol + o3 + sa);
         const float d1 = x0 - x1, d2 = x1 - x2, d3 = x2 - x3;
         S0b += bfirst ? d1 : d2;
         S0c += bfirst ? d2 : d1;
@@ -314,10 +315,11 @@ __global__ void __launch_bounds__(kGradThreads, CTP_GRAD_MIN_BLOCKS) geometry_gr
   const float* __restrict__ base = yfast ? volT : vol;
   const Off sx = yfast ? ny : (Off)1, sy = yfast ? (Off)1 : nx, sz = nx * ny;
   const Off off = (Off)W.i[2] * sz + (Off)W.i[1] * sy + (Off)W.i[0] * sx;
-  const float first = hit ? __ldg(base + off) : 0.f;
+  const long long n_vox = (long long)P.vol.n[0] * P.vol.n[1] * P.vol.n[2];
+  const float first = hit && CTP_IN_BOUNDS(off, n_vox, 14) ? __ldg(base + off) : 0.f;
   float f0[3], fl[3];
   const float last =
-      crossing_sums<Off>(hit, W, hi, base, off, W.step[0] * sx, W.step[1] * sy, W.step[2] * sz, first, f0, fl);
+      crossing_sums<Off>(hit, W, hi, base, off, W.step[0] * sx, W.step[1] * sy, W.step[2] * sz, first, f0, fl, n_vox);
 
   // Pass 2: the same FP64 setup again (bit-identical), recomputed rather than
   // kept live through the walk so the walk runs with fewer registers; the
@@ -432,6 +434,19 @@ cudaError_t launch_geometry_gradient(const FwdLaunch& p, const ViewRec* views, c
     else geometry_gradient_kernel<int, false><<<nb, block, 0, stream>>>(p, views, trig, vol, volT, gsino, grad);
   }
   return cudaGetLastError();
+}
+
+// The bounds-check word of this file's kernel (CTP_DEBUG builds; 0
+// elsewhere), read and cleared.  Synchronous.
+unsigned long long debug_take_word_grad() {
+#ifdef CTP_DEBUG
+  unsigned long long w = 0, z = 0;
+  if (cudaMemcpyFromSymbol(&w, g_debug_word, sizeof(w)) != cudaSuccess) return ~0ull;
+  cudaMemcpyToSymbol(g_debug_word, &z, sizeof(z));
+  return w;
+#else
+  return 0;
+#endif
 }
 
 }  // namespace ctp

@@ -101,6 +101,11 @@ cudaError_t launch_geometry_gradient(const FwdLaunch& p, const ViewRec* views, c
                                      const float* volT, const float* gsino, double* grad, bool wide_index,
                                      cudaStream_t stream);
 
+// Bounds-check words of the CTP_DEBUG build (ctp_kernels.cu, ctp_grad.cu):
+// read and cleared, synchronously; always 0 in other builds.
+unsigned long long debug_take_word_kernels();
+unsigned long long debug_take_word_grad();
+
 // Host helpers (ctp_api.cu).
 ctp_status host_validate(const ctp_geom_desc* d);
 ctp_status host_view_record(const ctp_geom_desc* d, int64_t v, ViewRec& V, double* trig_row);
@@ -108,6 +113,9 @@ ctp_status host_error(ctp_status s, const char* msg);
 ctp_status host_cuda_error(cudaError_t e, const char* where);
 bool host_is_device_pointer(const void* ptr, int device);
 void host_clear_error();
+// Raise the brick adjoint's dynamic shared-memory limit on the current
+// device to at least smem_bytes (kb members); never lowers it, so handles
+// with larger bricks stay launchable.  Called at create only.
 cudaError_t prepare_back_brick(size_t smem_bytes, int kb = 1);
 
 }  // namespace ctp

@@ -38,6 +38,10 @@
 //                      ray-voxel collisions (and, counting, the collision ratio).
 //   count_kernel       the forward traversal counting positive-length segments.
 //   transpose_xy       x-fastest -> y-fastest copy of the volume.
+#include <map>
+#include <mutex>
+#include <utility>
+
 #include "ctp_ray.cuh"
 
 namespace ctp {
@@ -460,7 +464,7 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows, kB == 1 ? CTP_FWD_MIN_BLOC
   make_ray(V, P.vol, trig, P.dims, v, valid ? r : 0, valid ? c : 0, R);
   const int lo[3] = {0, 0, 0};
   const int hi[3] = {P.vol.n[0], P.vol.n[1], P.vol.n[2]};
-  double t_in = 0.0, t_out = 0.0;
+  setup_t t_in = 0, t_out = 0;
   const bool hit = valid && clip(R, lo, hi, t_in, t_out);
   Walk W = {};
   if (hit) entry(R, t_in, t_out, lo, hi, W);
@@ -477,14 +481,18 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows, kB == 1 ? CTP_FWD_MIN_BLOC
   for (int j = 0; j < kB; ++j) acc[j] = 0.f;
   walk<true, false, 0, Off>(hit, W, lo, hi, off, W.step[0] * sx, W.step[1] * sy, W.step[2] * sz, nullptr,
                          [&](Off o, float len, bool) {
+                           if (CTP_IN_BOUNDS(o, n_vox, 1)) {
 #pragma unroll
-                           for (int j = 0; j < kB; ++j) acc[j] = fmaf(len, __ldg(base + j * n_vox + o), acc[j]);
+                             for (int j = 0; j < kB; ++j) acc[j] = fmaf(len, __ldg(base + j * n_vox + o), acc[j]);
+                           }
                          });
   if (valid) {
     const size_t n_rays = (size_t)P.dims.n_views * P.dims.n_rows * P.dims.n_cols;
     const size_t i = ((size_t)v * P.dims.n_rows + r) * P.dims.n_cols + c;
+    if (CTP_IN_BOUNDS(i, n_rays, 2)) {
 #pragma unroll
-    for (int j = 0; j < kB; ++j) sino[j * n_rays + i] = acc[j];
+      for (int j = 0; j < kB; ++j) sino[j * n_rays + i] = acc[j];
+    }
   }
 }
 
@@ -506,7 +514,7 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows) count_kernel(FwdLaunch P, 
   make_ray(views[v], P.vol, trig, P.dims, v, valid ? r : 0, valid ? c : 0, R);
   const int lo[3] = {0, 0, 0};
   const int hi[3] = {P.vol.n[0], P.vol.n[1], P.vol.n[2]};
-  double t_in = 0.0, t_out = 0.0;
+  setup_t t_in = 0, t_out = 0;
   const bool hit = valid && clip(R, lo, hi, t_in, t_out);
   Walk W = {};
   if (hit) entry(R, t_in, t_out, lo, hi, W);
@@ -899,17 +907,18 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
         v = vb + sl;
         const size_t i = ((size_t)v * nr + r) * nc + c;
         act = false;
+        const bool in = CTP_IN_BOUNDS(i, n_rays, 8) && CTP_IN_BOUNDS(v, P.dims.n_views, 9);
 #pragma unroll
         for (int m = 0; m < kB; ++m) {
           // a member whose stage scale is 0 or NaN adds nothing (its brick
           // is all zero, or written as NaN, at the flush); a single member
           // only gets here with a positive scale
-          y[m] = (kB == 1 || S[m] > 0.f) ? __ldg(sino + m * n_rays + i) : 0.f;
+          y[m] = in && (kB == 1 || S[m] > 0.f) ? __ldg(sino + m * n_rays + i) : 0.f;
           act |= y[m] != 0.f;
         }
       }
       Ray R;
-      double t_in = 0.0, t_out = 0.0;
+      setup_t t_in = 0, t_out = 0;
       if (act) {
         make_ray(views[v], P.vol, trig, P.dims, v, r, c, R);
         act = clip(R, lo, hi, t_in, t_out);
@@ -931,6 +940,7 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
       // Elsewhere (few rays per voxel, a finer scale) a conversion does.
       const int mbytes = 4 * n_acc;  // byte distance between the members' bricks
       auto visit_fma = [&](int o, float len) {
+        if (!CTP_IN_BOUNDS(o >> 2, n_acc, 5)) return;
         const float w = coef<kPower>(len);
 #pragma unroll
         for (int m = 0; m < kB; ++m)
@@ -938,6 +948,7 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
                     __float_as_int(fmaf(w, yS[m], kRoundBias)) - kRoundBiasBits);
       };
       auto visit_cvt = [&](int o, float len) {
+        if (!CTP_IN_BOUNDS(o >> 2, n_acc, 5)) return;
         const float w = coef<kPower>(len);
 #pragma unroll
         for (int m = 0; m < kB; ++m)
@@ -1026,6 +1037,7 @@ __global__ void __launch_bounds__(kBackThreads, CTP_BACK_MIN_BLOCKS)
       const int z = t / ey;
       const int ai = (z * P.brick[1] + yy) * pitch + x;
       const Off gi = ((Off)(lo[2] + z) * ny + (Off)(lo[1] + yy)) * nx + (Off)(lo[0] + x);
+      if (!CTP_IN_BOUNDS(ai, n_acc, 6) || !CTP_IN_BOUNDS(gi, n_vox, 7)) continue;
 #pragma unroll
       for (int m = 0; m < kB; ++m) {
         const float val = nan_stage[m] ? CUDART_NAN_F : (float)acc[m * n_acc + ai] * inv[m];
@@ -1076,7 +1088,7 @@ __device__ __forceinline__ void warp_sort_pairs(Key& key, float& val, int lane) 
 // with one global atomic.  With kCount nothing is written; instead the
 // numbers of contributions and of runs are added to n_upd and n_runs.
 template <bool kCount, typename Key>
-__device__ __forceinline__ void warp_segment_reduce(Key key, float val, bool valid, float* __restrict__ vol,
+__device__ __forceinline__ void warp_segment_reduce(Key key, float val, bool valid, float* __restrict__ vol, size_t n_vox,
                                                     unsigned long long& n_upd, unsigned long long& n_runs) {
   constexpr unsigned kFull = 0xffffffffu;
   const Key kNone = (Key)(~(unsigned long long)0 >> 1);
@@ -1108,7 +1120,7 @@ __device__ __forceinline__ void warp_segment_reduce(Key key, float val, bool val
       n_runs += __popc(r);
     }
   } else if (tail && key != kNone) {
-    atomicAdd(vol + key, sum);
+    if (CTP_IN_BOUNDS(key, n_vox, 12)) atomicAdd(vol + key, sum);
   }
 }
 
@@ -1137,7 +1149,7 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_FWD_MIN_BLOCKS)
   make_ray(views[v], P.vol, trig, P.dims, v, valid ? r : 0, valid ? c : 0, R);
   const int lo[3] = {0, 0, 0};
   const int hi[3] = {P.vol.n[0], P.vol.n[1], P.vol.n[2]};
-  double t_in = 0.0, t_out = 0.0;
+  setup_t t_in = 0, t_out = 0;
   const bool hit = valid && y != 0.f && clip(R, lo, hi, t_in, t_out);
   Walk W = {};
   // the counting form only counts segments: no re-anchoring needed
@@ -1147,10 +1159,11 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_FWD_MIN_BLOCKS)
   if (hit) entry(R, t_in, t_out, lo, hi, W, kAnchor ? anc : nullptr, kAncStride);
   const Off nx = P.vol.n[0], sz = (Off)P.vol.n[0] * P.vol.n[1];
   const Off off = (Off)W.i[2] * sz + (Off)W.i[1] * nx + (Off)W.i[0];
+  const size_t n_vox = (size_t)P.vol.n[0] * P.vol.n[1] * P.vol.n[2];
   unsigned long long n_upd = 0, n_runs = 0;
   walk<true, true, kAnchor, Off>(hit, W, lo, hi, off, (Off)W.step[0], W.step[1] * nx, W.step[2] * sz, anc,
                         [&](Off o, float len, bool f) {
-                          warp_segment_reduce<kCount, Off>(o, coef<kPower>(len) * y, f, vol, n_upd, n_runs);
+                          warp_segment_reduce<kCount, Off>(o, coef<kPower>(len) * y, f, vol, n_vox, n_upd, n_runs);
                         });
   if (kCount && (threadIdx.x & 31) == 0 && (n_upd | n_runs)) {
     atomicAdd(counters, n_upd);
@@ -1186,7 +1199,7 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_SCATTER_MIN_BLOCKS)
   make_ray(V, P.vol, trig, P.dims, v, valid ? r : 0, valid ? c : 0, R);
   const int lo[3] = {0, 0, 0};
   const int hi[3] = {P.vol.n[0], P.vol.n[1], P.vol.n[2]};
-  double t_in = 0.0, t_out = 0.0;
+  setup_t t_in = 0, t_out = 0;
   const bool hit = valid && y != 0.f && clip(R, lo, hi, t_in, t_out);
   Walk W = {};
   __shared__ double s_anc[7 * kAncStride];
@@ -1199,9 +1212,10 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_SCATTER_MIN_BLOCKS)
   const Off sy = yfast ? (Off)1 : nx;
   const Off sz = nx * ny;
   const Off off = (Off)W.i[2] * sz + (Off)W.i[1] * sy + (Off)W.i[0] * sx;
+  [[maybe_unused]] const size_t n_vox = (size_t)P.vol.n[0] * P.vol.n[1] * P.vol.n[2];
   walk<true, false, kWalkAnchor, Off>(hit, W, lo, hi, off, W.step[0] * sx, W.step[1] * sy, W.step[2] * sz, anc,
                                       [&](Off o, float len, bool) {
-                           if (len > 0.f) atomicAdd(base + o, coef<kPower>(len) * y);
+                           if (len > 0.f && CTP_IN_BOUNDS(o, n_vox, 10)) atomicAdd(base + o, coef<kPower>(len) * y);
                          });
 }
 
@@ -1248,10 +1262,12 @@ __device__ __forceinline__ unsigned row_slices(const ViewRec& V, const VolDesc& 
 #pragma unroll
   for (int j = 0; j < kR; ++j) {
     const int r = r0 + j;
-    // the z component of pixel_centre's flat-detector formula
-    const double pz = fma((double)r, V.dv[2], fma((double)c, V.du[2], V.p00[2]));
-    const double az = (pz - G.origin[2]) * G.inv_spacing[2];
-    const bool in = r < n_rows && az >= 0.0 && az < (double)G.n[2];
+    // the z component of pixel_centre's flat-detector formula and make_ray's
+    // voxel-unit height, in the set-up's precision
+    using T = setup_t;
+    const T pz = fma((T)r, (T)V.dv[2], fma((T)c, (T)V.du[2], (T)V.p00[2]));
+    const T az = (pz - (T)G.origin[2]) * (T)G.inv_spacing[2];
+    const bool in = r < n_rows && az >= (T)0 && az < (T)G.n[2];
     zoff[j] = in ? (Off)clampi((int)floor(az), 0, G.n[2] - 1) * sz : (Off)0;
     mask |= in ? 1u << j : 0u;
   }
@@ -1262,9 +1278,9 @@ __device__ __forceinline__ unsigned row_slices(const ViewRec& V, const VolDesc& 
 // volume's height (its direction has no z component, so only the x and y
 // slabs clip it) and walked as slice 0.
 __device__ __forceinline__ bool slice_ray(const ViewRec& V, const VolDesc& G, const Dims& dm, int v, int c, Ray& R,
-                                          double& t_in, double& t_out) {
+                                          setup_t& t_in, setup_t& t_out) {
   make_ray(V, G, nullptr, dm, v, 0, c, R);
-  R.A[2] = 0.5;
+  R.A[2] = (setup_t)0.5;
   const int lo[3] = {0, 0, 0};
   const int hi[3] = {G.n[0], G.n[1], G.n[2]};
   return clip(R, lo, hi, t_in, t_out);
@@ -1288,7 +1304,7 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_ROWS_MIN_BLOCKS)
   Off zoff[kR];
   const unsigned rows = cvalid ? row_slices<kR, Off>(V, P.vol, r0, c, P.dims.n_rows, sz, zoff) : 0u;
   Ray R;
-  double t_in = 0.0, t_out = 0.0;
+  setup_t t_in = 0, t_out = 0;
   const bool hit = slice_ray(V, P.vol, P.dims, v, cvalid ? c : 0, R, t_in, t_out) && rows != 0u;
   const int lo[3] = {0, 0, 0};
   const int hi[3] = {P.vol.n[0], P.vol.n[1], P.vol.n[2]};
@@ -1299,6 +1315,7 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_ROWS_MIN_BLOCKS)
   const Off sx = yfast ? ny : (Off)1;
   const Off sy = yfast ? (Off)1 : nx;
   const Off off = (Off)W.i[1] * sy + (Off)W.i[0] * sx;
+  [[maybe_unused]] const size_t n_vox = (size_t)P.vol.n[0] * P.vol.n[1] * P.vol.n[2];
   float acc[kR];
 #pragma unroll
   for (int j = 0; j < kR; ++j) acc[j] = 0.f;
@@ -1306,13 +1323,16 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_ROWS_MIN_BLOCKS)
                             [&](Off o, float len, bool) {
 #pragma unroll
                               for (int j = 0; j < kR; ++j)
-                                if (rows & (1u << j)) acc[j] = fmaf(len, __ldg(base + o + zoff[j]), acc[j]);
+                                if ((rows & (1u << j)) && CTP_IN_BOUNDS(o + zoff[j], n_vox, 3))
+                                  acc[j] = fmaf(len, __ldg(base + o + zoff[j]), acc[j]);
                             });
   if (cvalid) {
 #pragma unroll
     for (int j = 0; j < kR; ++j) {
       const int r = r0 + j;
-      if (r < P.dims.n_rows) sino[((size_t)v * P.dims.n_rows + r) * P.dims.n_cols + c] = acc[j];
+      const size_t i = ((size_t)v * P.dims.n_rows + r) * P.dims.n_cols + c;
+      if (r < P.dims.n_rows && CTP_IN_BOUNDS(i, (size_t)P.dims.n_views * P.dims.n_rows * P.dims.n_cols, 4))
+        sino[i] = acc[j];
     }
   }
 }
@@ -1341,7 +1361,7 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_ROWS_MIN_BLOCKS)
     if (!(y[j] != 0.f)) rows &= ~(1u << j);  // zero rows add nothing (NaN stays)
   }
   Ray R;
-  double t_in = 0.0, t_out = 0.0;
+  setup_t t_in = 0, t_out = 0;
   const bool hit = slice_ray(V, P.vol, P.dims, v, cvalid ? c : 0, R, t_in, t_out) && rows != 0u;
   const int lo[3] = {0, 0, 0};
   const int hi[3] = {P.vol.n[0], P.vol.n[1], P.vol.n[2]};
@@ -1354,13 +1374,15 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_ROWS_MIN_BLOCKS)
   const Off sx = yfast ? ny : (Off)1;
   const Off sy = yfast ? (Off)1 : nx;
   const Off off = (Off)W.i[1] * sy + (Off)W.i[0] * sx;
+  [[maybe_unused]] const size_t n_vox = (size_t)P.vol.n[0] * P.vol.n[1] * P.vol.n[2];
   walk<true, false, kWalkAnchor, Off>(hit, W, lo, hi, off, W.step[0] * sx, W.step[1] * sy, (Off)0, anc,
                                       [&](Off o, float len, bool) {
                                         if (len > 0.f) {
                                           const float w = coef<kPower>(len);
 #pragma unroll
                                           for (int j = 0; j < kR; ++j)
-                                            if (rows & (1u << j)) atomicAdd(base + o + zoff[j], w * y[j]);
+                                            if ((rows & (1u << j)) && CTP_IN_BOUNDS(o + zoff[j], n_vox, 11))
+                                              atomicAdd(base + o + zoff[j], w * y[j]);
                                         }
                                       });
 }
@@ -1368,6 +1390,19 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_ROWS_MIN_BLOCKS)
 }  // namespace
 
 // ---------------------------------------------------------------- launchers --
+
+// The bounds-check word of this file's kernels (CTP_DEBUG builds; 0 elsewhere),
+// read and cleared.  Synchronous.
+unsigned long long debug_take_word_kernels() {
+#ifdef CTP_DEBUG
+  unsigned long long w = 0, z = 0;
+  if (cudaMemcpyFromSymbol(&w, g_debug_word, sizeof(w)) != cudaSuccess) return ~0ull;
+  cudaMemcpyToSymbol(g_debug_word, &z, sizeof(z));
+  return w;
+#else
+  return 0;
+#endif
+}
 
 cudaError_t launch_forward_rows(const FwdLaunch& p, const ViewRec* views, const float* vol, const float* volT,
                                 float* sino, bool wide_index, cudaStream_t stream) {
@@ -1383,6 +1418,9 @@ cudaError_t launch_forward_rows(const FwdLaunch& p, const ViewRec* views, const 
       break;
     case 4:
       if (wide_index) CTP_ROWS_LAUNCH(long long, 4); else CTP_ROWS_LAUNCH(int, 4);
+      break;
+    case 8:
+      if (wide_index) CTP_ROWS_LAUNCH(long long, 8); else CTP_ROWS_LAUNCH(int, 8);
       break;
     default:
       return cudaErrorInvalidValue;
@@ -1403,7 +1441,13 @@ cudaError_t launch_back_scatter(const FwdLaunch& p, const ViewRec* views, const 
     if (rb > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     const unsigned nr = (unsigned)rb;
 #define CTP_SROWS(KP, OFF, R) back_scatter_rows_kernel<KP, OFF, R><<<nr, block, 0, stream>>>(p, views, sino, vol, volT)
-    if (p.row_group == 4) {
+    if (p.row_group == 8) {
+      if (power == 2) {
+        if (wide_index) CTP_SROWS(2, long long, 8); else CTP_SROWS(2, int, 8);
+      } else {
+        if (wide_index) CTP_SROWS(1, long long, 8); else CTP_SROWS(1, int, 8);
+      }
+    } else if (p.row_group == 4) {
       if (power == 2) {
         if (wide_index) CTP_SROWS(2, long long, 4); else CTP_SROWS(2, int, 4);
       } else {
@@ -1547,7 +1591,18 @@ void launch_back_brick_kb(const BackLaunch& p, const ViewRec* views, const doubl
 }  // namespace
 
 cudaError_t prepare_back_brick(size_t smem_bytes, int kb) {
-  return kb == 2 ? set_back_smem<2>((int)smem_bytes) : set_back_smem<1>((int)smem_bytes);
+  // the limit set so far, per device and member count (one lock: create is rare)
+  static std::mutex mu;
+  static std::map<std::pair<int, int>, size_t> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  size_t& have = done[{dev, kb}];
+  if (smem_bytes <= have) return cudaSuccess;
+  e = kb == 2 ? set_back_smem<2>((int)smem_bytes) : set_back_smem<1>((int)smem_bytes);
+  if (e == cudaSuccess) have = smem_bytes;
+  return e;
 }
 
 cudaError_t launch_back_brick(const BackLaunch& p, const ViewRec* views, const double* trig, const float* sino,
@@ -1557,8 +1612,6 @@ cudaError_t launch_back_brick(const BackLaunch& p, const ViewRec* views, const d
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   const size_t smem = back_brick_smem_bytes(p.brick, kb);
-  cudaError_t e = prepare_back_brick(smem, kb);
-  if (e != cudaSuccess) return e;
   if (kb == 2) launch_back_brick_kb<2>(p, views, trig, sino, vol, power, wide_index, (unsigned)blocks, smem, stream);
   else launch_back_brick_kb<1>(p, views, trig, sino, vol, power, wide_index, (unsigned)blocks, smem, stream);
   return cudaGetLastError();

@@ -3,8 +3,9 @@
 // needs beyond the caller's volume and sinogram -- the per-view FP64 records,
 // the cylindrical column table and the y-fastest copy of the volume -- lives
 // in one file-scope device array of fixed size.  Nothing here allocates:
-// no cudaMalloc/cudaFree, no host heap; records are built in a stack buffer
-// and copied with cudaMemcpyAsync (pageable source, consumed before return).
+// no cudaMalloc/cudaFree, no host heap; records are built in a stack buffer,
+// column rows in a static staging array, and both are copied with
+// cudaMemcpyAsync (pageable source, consumed before the copy call returns).
 #include <cmath>
 #include <cstdio>
 #include <mutex>
@@ -14,27 +15,28 @@
 namespace {
 
 constexpr size_t kScratchBytes = CTP_NOALLOC_SCRATCH_BYTES;
-constexpr int kMaxDevices = 64;
 constexpr int kChunk = 32;  // view records built and copied per cudaMemcpyAsync
 
 // The scratch.  Every GPU that loads the library holds it until exit; all
 // calls on a device share it and it keeps the last call's contents.
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
+// Serialises the host part of the calls (the staging buffer below).
 std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
 
-// Device address of g_scratch on `device` (current).  The host-side name is
-// only a stand-in, so the address is looked up once per device.
-cudaError_t scratch_address(int device, unsigned char** out) {
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_ptr[device]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_ptr[device] = p;
-  }
-  *out = static_cast<unsigned char*>(g_scratch_ptr[device]);
+// Host staging for the cylindrical column table: whole views' rows of cos/sin
+// pairs are packed here and sent with one copy (a static array, not heap).
+constexpr size_t kTrigStage = 1 << 16;  // doubles (512 KiB)
+double g_trig_stage[kTrigStage];
+
+// Device address of g_scratch on the current device.  The host-side name is
+// only a stand-in; the address is looked up on every call (no allocation, and
+// no stale address after the caller resets the device).
+cudaError_t scratch_address(unsigned char** out) {
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_scratch);
+  if (e != cudaSuccess) return e;
+  *out = static_cast<unsigned char*>(p);
   return cudaSuccess;
 }
 
@@ -64,7 +66,7 @@ extern "C" ctp_status ctp_forward_noalloc(const ctp_geom_desc* desc, const float
   ctp_status st = host_validate(desc);
   if (st != CTP_OK) return st;
   const ctp_geom_desc& d = *desc;
-  if (d.device < 0 || d.device >= kMaxDevices) return host_error(CTP_ERR_INVALID_ARGUMENT, "device ordinal out of range");
+  if (d.device < 0) return host_error(CTP_ERR_INVALID_ARGUMENT, "device ordinal out of range");
 
   // pass 1 (host only): guards of every view and the layout plan
   ViewRec rec[kChunk];
@@ -90,45 +92,71 @@ extern "C" ctp_status ctp_forward_noalloc(const ctp_geom_desc* desc, const float
 
   CurrentDevice cd(d.device);
   if (cd.err != cudaSuccess) return host_cuda_error(cd.err, "cudaSetDevice");
+  cudaStream_t s = (cudaStream_t)stream;
+  // The uploads below copy from this call's host memory, which is gone (or
+  // reused) once the call returns: a graph captured from them would replay
+  // stale copies, so a capturing stream is refused before anything is enqueued.
+  cudaStreamCaptureStatus capturing = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(s, &capturing);
+  if (e != cudaSuccess) return host_cuda_error(e, "cudaStreamIsCapturing");
+  if (capturing != cudaStreamCaptureStatusNone)
+    return host_error(CTP_ERR_UNSUPPORTED, "ctp_forward_noalloc does not run on a stream that is capturing");
   if (!host_is_device_pointer(vol, d.device))
     return host_error(CTP_ERR_INVALID_ARGUMENT, "vol is not device memory of the described device");
   if (!host_is_device_pointer(sino, d.device))
     return host_error(CTP_ERR_INVALID_ARGUMENT, "sino is not device memory of the described device");
+  std::lock_guard<std::mutex> lock(g_mu);
   unsigned char* base = nullptr;
-  cudaError_t e = scratch_address(d.device, &base);
+  e = scratch_address(&base);
   if (e != cudaSuccess) return host_cuda_error(e, "cudaGetSymbolAddress");
   ViewRec* d_views = reinterpret_cast<ViewRec*>(base);
   double* d_trig = trig_bytes ? reinterpret_cast<double*>(base + rec_bytes) : nullptr;
   float* d_copy = copy_bytes ? reinterpret_cast<float*>(base + rec_bytes + trig_bytes) : nullptr;
-  cudaStream_t s = (cudaStream_t)stream;
   e = cudaGetLastError();
   if (e != cudaSuccess) return host_cuda_error(e, "pending error before ctp_forward_noalloc");
 
-  // pass 2: records (and column rows) to the scratch, chunk by chunk
-  double trig_row[2 * 1024];
+  // pass 2: records to the scratch, kChunk views per copy; column rows of as
+  // many whole views as the staging buffer holds per copy (a row wider than
+  // the buffer goes in pieces)
+  const size_t row = 2 * (size_t)d.n_cols;  // doubles per view
+  int64_t staged_v0 = 0;
+  size_t staged = 0;
+  auto flush_trig = [&]() -> cudaError_t {
+    if (!staged) return cudaSuccess;
+    const cudaError_t err = cudaMemcpyAsync(d_trig + (size_t)staged_v0 * row, g_trig_stage, sizeof(double) * staged,
+                                            cudaMemcpyHostToDevice, s);
+    staged = 0;
+    return err;
+  };
   for (int64_t v0 = 0; v0 < d.n_views; v0 += kChunk) {
     const int n = (int)(d.n_views - v0 < kChunk ? d.n_views - v0 : kChunk);
     for (int i = 0; i < n; ++i) {
       const int64_t v = v0 + i;
-      double* row = nullptr;
-      if (d_trig && d.n_cols <= 1024) row = trig_row;
-      st = host_view_record(desc, v, rec[i], row);
+      st = host_view_record(desc, v, rec[i], nullptr);
       if (st != CTP_OK) return st;
-      if (d_trig) {
-        if (!row) {  // a wide cylindrical detector: the row is built in pieces below
-          for (int64_t c0 = 0; c0 < d.n_cols; c0 += 1024) {
-            const int64_t m = d.n_cols - c0 < 1024 ? d.n_cols - c0 : 1024;
-            for (int64_t c = 0; c < m; ++c) {
-              const double g = rec[i].gam0 + (double)(c0 + c) * rec[i].dgam;
-              trig_row[2 * c] = std::cos(g);
-              trig_row[2 * c + 1] = std::sin(g);
-            }
-            e = cudaMemcpyAsync(d_trig + 2 * (v * d.n_cols + c0), trig_row, sizeof(double) * 2 * (size_t)m,
-                                cudaMemcpyHostToDevice, s);
-            if (e != cudaSuccess) return host_cuda_error(e, "column table upload");
+      if (!d_trig) continue;
+      if (row <= kTrigStage) {
+        if (staged + row > kTrigStage) {
+          e = flush_trig();
+          if (e != cudaSuccess) return host_cuda_error(e, "column table upload");
+        }
+        if (!staged) staged_v0 = v;
+        for (int64_t c = 0; c < d.n_cols; ++c) {
+          const double g = rec[i].gam0 + (double)c * rec[i].dgam;
+          g_trig_stage[staged + 2 * c] = std::cos(g);
+          g_trig_stage[staged + 2 * c + 1] = std::sin(g);
+        }
+        staged += row;
+      } else {
+        const int64_t piece = (int64_t)(kTrigStage / 2);
+        for (int64_t c0 = 0; c0 < d.n_cols; c0 += piece) {
+          const int64_t m = d.n_cols - c0 < piece ? d.n_cols - c0 : piece;
+          for (int64_t c = 0; c < m; ++c) {
+            const double g = rec[i].gam0 + (double)(c0 + c) * rec[i].dgam;
+            g_trig_stage[2 * c] = std::cos(g);
+            g_trig_stage[2 * c + 1] = std::sin(g);
           }
-        } else {
-          e = cudaMemcpyAsync(d_trig + 2 * v * d.n_cols, trig_row, sizeof(double) * 2 * (size_t)d.n_cols,
+          e = cudaMemcpyAsync(d_trig + (size_t)v * row + 2 * (size_t)c0, g_trig_stage, sizeof(double) * 2 * (size_t)m,
                               cudaMemcpyHostToDevice, s);
           if (e != cudaSuccess) return host_cuda_error(e, "column table upload");
         }
@@ -137,6 +165,8 @@ extern "C" ctp_status ctp_forward_noalloc(const ctp_geom_desc* desc, const float
     e = cudaMemcpyAsync(d_views + v0, rec, sizeof(ViewRec) * (size_t)n, cudaMemcpyHostToDevice, s);
     if (e != cudaSuccess) return host_cuda_error(e, "view record upload");
   }
+  e = flush_trig();
+  if (e != cudaSuccess) return host_cuda_error(e, "column table upload");
 
   // same launch plan as ctp_forward
   FwdLaunch f{};

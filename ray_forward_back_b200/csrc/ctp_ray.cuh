@@ -12,12 +12,39 @@
 
 namespace ctp {
 
+// Working precision of the per-ray set-up: FP64.  The CTP_FP32_SETUP build
+// (an ablation for tests only, never the library's default) runs the same
+// set-up in FP32, the working precision the pages report for hardware
+// without FP64 (diffct "Execution", paragraph on Apple MPS).
+#ifdef CTP_FP32_SETUP
+using setup_t = float;
+#else
+using setup_t = double;
+#endif
+
+// Bounds checks of the CTP_DEBUG build: every global and shared-memory index
+// of the walks and flushes is tested against its array's extent; a failing
+// index is recorded (the first one per translation unit: check site in the
+// top 16 bits, the index in the low 48) and its access skipped, so a bad
+// index never reaches memory.  Ordinary builds compile the checks away.
+#ifdef CTP_DEBUG
+static __device__ unsigned long long g_debug_word;
+__device__ __forceinline__ bool in_bounds(long long i, long long n, unsigned site) {
+  if (i >= 0 && i < n) return true;
+  atomicCAS(&g_debug_word, 0ull, ((unsigned long long)site << 48) | ((unsigned long long)i & 0xffffffffffffull));
+  return false;
+}
+#define CTP_IN_BOUNDS(i, n, site) ::ctp::in_bounds((long long)(i), (long long)(n), (site))
+#else
+#define CTP_IN_BOUNDS(i, n, site) true
+#endif
+
 struct Ray {
-  double A[3];    // parameter origin, voxel units relative to the volume min corner
-  double D[3];    // direction, voxel units per unit t
-  double rcp[3];  // 1 / D (unused where D == 0)
-  double len;     // physical length per unit t
-  double t_lo, t_hi;
+  setup_t A[3];    // parameter origin, voxel units relative to the volume min corner
+  setup_t D[3];    // direction, voxel units per unit t
+  setup_t rcp[3];  // 1 / D (unused where D == 0)
+  setup_t len;     // physical length per unit t
+  setup_t t_lo, t_hi;
 };
 
 struct Walk {
@@ -30,15 +57,17 @@ struct Walk {
 };
 
 __device__ __forceinline__ void pixel_centre(const ViewRec& V, const double* __restrict__ trig, const Dims& dm, int v,
-                                             int r, int c, double p[3]) {
+                                             int r, int c, setup_t p[3]) {
+  using T = setup_t;
   if (dm.det == CTP_DET_FLAT) {
 #pragma unroll
-    for (int k = 0; k < 3; ++k) p[k] = fma((double)r, V.dv[k], fma((double)c, V.du[k], V.p00[k]));
+    for (int k = 0; k < 3; ++k) p[k] = fma((T)r, (T)V.dv[k], fma((T)c, (T)V.du[k], (T)V.p00[k]));
   } else {
     const size_t t = 2 * ((size_t)v * dm.n_cols + c);
-    const double cg = trig[t], sg = trig[t + 1];
+    const T cg = (T)trig[t], sg = (T)trig[t + 1];
 #pragma unroll
-    for (int k = 0; k < 3; ++k) p[k] = fma((double)r, V.dv[k], V.p00[k]) + V.R * fma(cg, V.w[k], sg * V.du[k]);
+    for (int k = 0; k < 3; ++k)
+      p[k] = fma((T)r, (T)V.dv[k], (T)V.p00[k]) + (T)V.R * fma(cg, (T)V.w[k], sg * (T)V.du[k]);
   }
 }
 
@@ -48,57 +77,59 @@ __device__ __forceinline__ void pixel_centre(const ViewRec& V, const double* __r
 // Returns true when the origin is the pixel (cone) or always (parallel).
 __device__ __forceinline__ bool make_ray(const ViewRec& V, const VolDesc& G, const double* __restrict__ trig,
                                          const Dims& dm, int v, int r, int c, Ray& R) {
-  double p[3];
+  using T = setup_t;
+  T p[3];
   pixel_centre(V, trig, dm, v, r, c, p);
   if (dm.beam == CTP_BEAM_PARALLEL) {
 #pragma unroll
     for (int k = 0; k < 3; ++k) {
-      R.A[k] = (p[k] - G.origin[k]) * G.inv_spacing[k];
-      R.D[k] = V.s[k] * G.inv_spacing[k];
-      R.rcp[k] = V.rcp_dir[k];
+      R.A[k] = (p[k] - (T)G.origin[k]) * (T)G.inv_spacing[k];
+      R.D[k] = (T)V.s[k] * (T)G.inv_spacing[k];
+      R.rcp[k] = (T)V.rcp_dir[k];
     }
-    R.len = 1.0;
-    R.t_lo = -CUDART_INF;
-    R.t_hi = CUDART_INF;
+    R.len = (T)1;
+    R.t_lo = -(T)CUDART_INF;
+    R.t_hi = (T)CUDART_INF;
     return true;
   } else {
-    double pv[3], sv[3], dp2 = 0.0, ds2 = 0.0;
+    T pv[3], sv[3], dp2 = 0, ds2 = 0;
 #pragma unroll
     for (int k = 0; k < 3; ++k) {
-      pv[k] = (p[k] - G.origin[k]) * G.inv_spacing[k];
-      sv[k] = (V.s[k] - G.origin[k]) * G.inv_spacing[k];
-      const double a = pv[k] - G.centre[k], b = sv[k] - G.centre[k];
+      pv[k] = (p[k] - (T)G.origin[k]) * (T)G.inv_spacing[k];
+      sv[k] = ((T)V.s[k] - (T)G.origin[k]) * (T)G.inv_spacing[k];
+      const T a = pv[k] - (T)G.centre[k], b = sv[k] - (T)G.centre[k];
       dp2 = fma(a, a, dp2);
       ds2 = fma(b, b, ds2);
     }
     const bool from_pixel = dp2 <= ds2;
-    double len2 = 0.0;
+    T len2 = 0;
 #pragma unroll
     for (int k = 0; k < 3; ++k) {
-      const double dw = from_pixel ? (V.s[k] - p[k]) : (p[k] - V.s[k]);
+      const T dw = from_pixel ? ((T)V.s[k] - p[k]) : (p[k] - (T)V.s[k]);
       len2 = fma(dw, dw, len2);
       R.A[k] = from_pixel ? pv[k] : sv[k];
-      R.D[k] = dw * G.inv_spacing[k];
-      R.rcp[k] = 1.0 / R.D[k];
+      R.D[k] = dw * (T)G.inv_spacing[k];
+      R.rcp[k] = (T)1 / R.D[k];
     }
     R.len = sqrt(len2);
-    R.t_lo = 0.0;
-    R.t_hi = 1.0;
+    R.t_lo = 0;
+    R.t_hi = 1;
     return from_pixel;
   }
 }
 
 // Slab clipping against the half-open box [lo, hi) (voxel units).
-__device__ __forceinline__ bool clip(const Ray& R, const int lo[3], const int hi[3], double& t_in, double& t_out) {
+__device__ __forceinline__ bool clip(const Ray& R, const int lo[3], const int hi[3], setup_t& t_in, setup_t& t_out) {
+  using T = setup_t;
   t_in = R.t_lo;
   t_out = R.t_hi;
 #pragma unroll
   for (int k = 0; k < 3; ++k) {
-    if (R.D[k] == 0.0) {
-      if (!(R.A[k] >= (double)lo[k] && R.A[k] < (double)hi[k])) return false;
+    if (R.D[k] == (T)0) {
+      if (!(R.A[k] >= (T)lo[k] && R.A[k] < (T)hi[k])) return false;
     } else {
-      const double ta = ((double)lo[k] - R.A[k]) * R.rcp[k];
-      const double tb = ((double)hi[k] - R.A[k]) * R.rcp[k];
+      const T ta = ((T)lo[k] - R.A[k]) * R.rcp[k];
+      const T tb = ((T)hi[k] - R.A[k]) * R.rcp[k];
       t_in = fmax(t_in, fmin(ta, tb));
       t_out = fmin(t_out, fmax(ta, tb));
     }
@@ -113,41 +144,42 @@ __device__ __forceinline__ int clampi(int x, int lo, int hi) { return x < lo ? l
 // With w64 (a per-lane record of 7 doubles at stride `stride`: l0[3],
 // inc[3], L) the FP64 values behind W's FP32 l0, inc and L are kept too, for
 // walks that re-anchor their local FP32 parameters along the ray.
-__device__ __forceinline__ void entry(const Ray& R, double t_in, double t_out, const int lo[3], const int hi[3],
+__device__ __forceinline__ void entry(const Ray& R, setup_t t_in, setup_t t_out, const int lo[3], const int hi[3],
                                       Walk& W, double* w64 = nullptr, int stride = 1) {
+  using T = setup_t;
 #pragma unroll
   for (int k = 0; k < 3; ++k) {
-    const double e = fma(t_in, R.D[k], R.A[k]);
-    const double x = fma(t_out, R.D[k], R.A[k]);
-    const double el = fmin(fmax(e, (double)lo[k]), (double)hi[k]);
-    const double xl = fmin(fmax(x, (double)lo[k]), (double)hi[k]);
-    if (R.D[k] > 0.0) {
+    const T e = fma(t_in, R.D[k], R.A[k]);
+    const T x = fma(t_out, R.D[k], R.A[k]);
+    const T el = fmin(fmax(e, (T)lo[k]), (T)hi[k]);
+    const T xl = fmin(fmax(x, (T)lo[k]), (T)hi[k]);
+    if (R.D[k] > (T)0) {
       const int i0 = clampi((int)floor(el), lo[k], hi[k] - 1);
       const int i1 = clampi((int)ceil(xl) - 1, lo[k], hi[k] - 1);
       W.i[k] = i0;
       W.N[k] = max(i1 - i0, 0);
       W.step[k] = 1;
-      const double tc = ((double)(i0 + 1) - R.A[k]) * R.rcp[k];
-      const double l0d = (tc - t_in) * R.len, incd = R.rcp[k] * R.len;
+      const T tc = ((T)(i0 + 1) - R.A[k]) * R.rcp[k];
+      const T l0d = (tc - t_in) * R.len, incd = R.rcp[k] * R.len;
       W.l0[k] = (float)l0d;
       W.inc[k] = (float)incd;
       if (w64) {
-        w64[k * stride] = l0d;
-        w64[(3 + k) * stride] = incd;
+        w64[k * stride] = (double)l0d;
+        w64[(3 + k) * stride] = (double)incd;
       }
-    } else if (R.D[k] < 0.0) {
+    } else if (R.D[k] < (T)0) {
       const int i0 = clampi((int)ceil(el) - 1, lo[k], hi[k] - 1);
       const int i1 = clampi((int)floor(xl), lo[k], hi[k] - 1);
       W.i[k] = i0;
       W.N[k] = max(i0 - i1, 0);
       W.step[k] = -1;
-      const double tc = ((double)i0 - R.A[k]) * R.rcp[k];
-      const double l0d = (tc - t_in) * R.len, incd = -R.rcp[k] * R.len;
+      const T tc = ((T)i0 - R.A[k]) * R.rcp[k];
+      const T l0d = (tc - t_in) * R.len, incd = -R.rcp[k] * R.len;
       W.l0[k] = (float)l0d;
       W.inc[k] = (float)incd;
       if (w64) {
-        w64[k * stride] = l0d;
-        w64[(3 + k) * stride] = incd;
+        w64[k * stride] = (double)l0d;
+        w64[(3 + k) * stride] = (double)incd;
       }
     } else {
       W.i[k] = clampi((int)floor(el), lo[k], hi[k] - 1);
@@ -161,9 +193,9 @@ __device__ __forceinline__ void entry(const Ray& R, double t_in, double t_out, c
       }
     }
   }
-  const double Ld = (t_out - t_in) * R.len;
+  const T Ld = (t_out - t_in) * R.len;
   W.L = (float)Ld;
-  if (w64) w64[6 * stride] = Ld;
+  if (w64) w64[6 * stride] = (double)Ld;
 }
 
 template <typename T>

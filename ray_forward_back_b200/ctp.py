@@ -37,7 +37,7 @@ CTP_ADJOINT_SORT = 2
 
 EXPORTED = ["ctp_geom_create", "ctp_geom_destroy", "ctp_geom_query", "ctp_forward", "ctp_back",
             "ctp_forward_batch", "ctp_back_batch", "ctp_back_power", "ctp_geometry_gradient", "ctp_count_updates", "ctp_forward_noalloc", "ctp_solve", "ctp_solver_workspace_bytes",
-            "ctp_status_string", "ctp_last_error_detail", "ctp_version"]
+            "ctp_debug_error_word", "ctp_status_string", "ctp_last_error_detail", "ctp_version"]
 CTP_SOLVER_CGLS = 1
 CTP_SOLVER_SIRT = 2
 
@@ -125,6 +125,8 @@ def load(path: str = None):
         lib.ctp_solve.argtypes = [vp, vp, vp, ctypes.POINTER(ctp_solver_options), vp, ctypes.c_size_t,
                                   ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctp_solver_result), vp]
         lib.ctp_solve.restype = ctypes.c_int
+        lib.ctp_debug_error_word.argtypes = [ctypes.POINTER(ctypes.c_uint64)]
+        lib.ctp_debug_error_word.restype = ctypes.c_int
         lib.ctp_status_string.argtypes = [ctypes.c_int]
         lib.ctp_status_string.restype = ctypes.c_char_p
         lib.ctp_last_error_detail.argtypes = []
@@ -283,6 +285,14 @@ def ctp_solve(handle: int, sino, vol, method: int, iterations: int, atol=0.0, rt
     _check(load().ctp_solve(handle, _ptr(sino), _ptr(vol), ctypes.byref(opts), base_aligned, size, hist,
                             ctypes.byref(res), _stream_handle(stream)))
     return [hist[i] for i in range(res.iterations + 1)], bool(res.converged)
+
+
+def ctp_debug_error_word() -> int:
+    """Bounds-check record of a CTP_DEBUG build (0: every index in bounds);
+    raises CtpError(CTP_ERR_UNSUPPORTED) in other builds."""
+    w = ctypes.c_uint64()
+    _check(load().ctp_debug_error_word(ctypes.byref(w)))
+    return int(w.value)
 
 
 def ctp_version() -> str:

@@ -118,7 +118,7 @@ def test_bad_plan(lib):
     _expect(ctp.CTP_ERR_INVALID_ARGUMENT, _cone(), {"brick": (0, -1, 0)})
     for chunk in (-1, 3, 8):
         _expect(ctp.CTP_ERR_INVALID_ARGUMENT, _cone(), {"batch_chunk": chunk})
-    for rows in (-1, 3, 8):
+    for rows in (-1, 3, 16):
         _expect(ctp.CTP_ERR_INVALID_ARGUMENT, _cone(), {"slice_rows": rows})
 
 

@@ -16,6 +16,7 @@ from tests.gpu_helpers import projector
 pytestmark = pytest.mark.gpu
 
 REL = 2e-4
+ELEMENT_FLOOR = 1e-6
 
 
 def _jitter(g, seed, scale=0.03):
@@ -46,8 +47,15 @@ def _check(g, seed, vol=None, h=1e-6, rel=REL):
     assert got.shape == (g.n_views, 4, 3)
     scale = np.abs(ref).max()
     assert scale > 0
-    err = np.abs(got - ref).max()
-    assert err <= rel * scale, (err, scale)
+    err = np.abs(got - ref)
+    assert err.max() <= rel * scale, (err.max(), scale)
+    # entry by entry: relative to the entry, plus a floor relative to the
+    # largest entry of the view set (the FP32 crossing positions carry a few
+    # ulp of the ray length whatever the entry's own size)
+    floor = ELEMENT_FLOOR * scale
+    worst = float(((err - 1e-4 * np.abs(ref)) / scale).max())
+    print(f"element floor used: {worst:.2e} of the largest entry")
+    assert np.all(err <= 1e-4 * np.abs(ref) + floor), worst
     return ref, got
 
 

@@ -87,6 +87,33 @@ def test_cgls_on_workload1_against_matrix_free_reference():
     assert np.linalg.norm(x - x_ref) <= 1e-3 * np.linalg.norm(x_ref)
 
 
+@pytest.mark.slow
+def test_solvers_on_workload2_view_subset_against_matrix_free_reference():
+    """Workload 2 at its full size (256^3 volume, 384 x 384 detector) on 12
+    evenly spaced views: five CGLS and five SIRT iterations against the
+    reference solvers run matrix-free on the oracle's forward and adjoint
+    (spread over the host's cores).  The reference casts its iterates to FP32
+    before each projection, as the GPU stores them."""
+    from oracle import pool
+    wl = W.workload(2)
+    g = wl.geom.subset_views(np.linspace(0, wl.geom.n_views - 1, 12).round().astype(np.int64))
+    y = pool.forward(g, wl.phantom()).astype(np.float32)
+    fwd = lambda x: pool.forward(g, x.reshape(g.vol_shape).astype(np.float32)).reshape(-1)
+    adj = lambda s: pool.back(g, s.reshape(g.sino_shape).astype(np.float32)).reshape(-1)
+    y64 = y.astype(np.float64).reshape(-1)
+    x_ref, h_ref, _ = solvers.cgls((fwd, adj, g.n_vox), y64, 5)
+    x, h, _ = _gpu_solve(g, y, "cgls", 5)
+    assert len(h) == len(h_ref) == 6
+    np.testing.assert_allclose(h, h_ref, rtol=1e-4)
+    assert np.linalg.norm(x - x_ref) <= 1e-3 * np.linalg.norm(x_ref)
+    x_ref, h_ref, _ = solvers.sirt((fwd, adj, g.n_vox), y64, 5, relaxation=1.0, nonnegative=True)
+    x, h, _ = _gpu_solve(g, y, "sirt", 5, relaxation=1.0, nonnegative=True)
+    assert len(h) == len(h_ref) == 6
+    np.testing.assert_allclose(h, h_ref, rtol=1e-4)
+    assert np.linalg.norm(x - x_ref) <= 1e-4 * np.linalg.norm(x_ref)
+    assert x.min() >= 0.0
+
+
 def test_workspace_contract():
     import torch
     from ray_forward_back_b200 import ctp

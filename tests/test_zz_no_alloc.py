@@ -7,16 +7,18 @@ is owned by another framework -- so they cannot create a geometry handle
 either.  For them the library offers one entry point that takes the
 acquisition description directly and keeps everything it needs in a fixed
 device array built into the library.  These tests call it through the C ABI
-and compare it with the ordinary handle-based ctp_forward.
+and compare it with the ordinary handle-based ctp_forward and with the FP64
+oracle.
 
 This file is named so that pytest collects it last.
 """
 import numpy as np
 import pytest
 
+import oracle
 from ray_forward_back_b200 import ctp
 from ray_forward_back_b200 import workloads as W
-from tests.gpu_helpers import projector, rel_l2
+from tests.gpu_helpers import check_forward, oracle_chords, projector, rel_l2
 from tests.helpers import small_geometries
 
 pytestmark = pytest.mark.gpu
@@ -31,12 +33,18 @@ def _close(got, ref):
     assert np.all(np.abs(got - ref) <= 1e-4 * np.abs(ref) + 1e-6 * np.abs(ref).max())
 
 
-def _noalloc_forward(geom, vol_t):
+def _noalloc_forward(geom, vol_t, stream=None):
     import torch
     out = torch.full(geom.sino_shape, float("nan"), dtype=torch.float32, device=vol_t.device)
-    ctp.ctp_forward_noalloc(geom, vol_t, out, device=vol_t.device.index or 0)
-    torch.cuda.synchronize()
-    return out.cpu().numpy()
+    ctp.ctp_forward_noalloc(geom, vol_t, out, device=vol_t.device.index or 0, stream=stream)
+    return out
+
+
+def _wide_cylindrical(n_cols):
+    """A cylindrical detector wider than one staged column row."""
+    pu = W.helical_fan_pitch(n_cols, 8.0, 60.0, 100.0)
+    return W.make_cone(16, 14, 12, 2, 2, n_cols, sid=60.0, sdd=100.0, pitch_u=pu, pitch_v=1.1,
+                       detector=W.DET_CYLINDRICAL, z_start=-1.3, z_end=1.1, start=0.21)
 
 
 def test_noalloc_matches_ctp_forward_on_two_calls_in_a_row():
@@ -49,13 +57,72 @@ def test_noalloc_matches_ctp_forward_on_two_calls_in_a_row():
     cases = [W.workload(1).geom, small_geometries()["helical_cyl"]]
     rng = np.random.default_rng(77)
     for g in cases:
-        vol = torch.from_numpy(rng.random(g.vol_shape).astype(np.float32)).to(dev)
+        vol_np = rng.random(g.vol_shape).astype(np.float32)
+        vol = torch.from_numpy(vol_np).to(dev)
         P = projector(g)
         ref = P.forward(vol)
-        torch.cuda.synchronize()
         got = _noalloc_forward(g, vol)
-        _close(got, ref.cpu().numpy())
+        torch.cuda.synchronize()
+        _close(got.cpu().numpy(), ref.cpu().numpy())
+        check_forward(got.cpu().numpy(), oracle.forward(g, vol_np), oracle_chords(g), min(g.spacing), "noalloc")
         P.close()
+
+
+def test_noalloc_two_geometries_queued_on_one_stream():
+    """Two calls enqueued back to back on one stream, one synchronisation:
+    the second call's uploads are ordered after the first call's kernels, so
+    both results stand."""
+    import torch
+    dev = torch.device("cuda", torch.cuda.current_device())
+    g1, g2 = small_geometries()["cone_flat"], small_geometries()["helical_cyl"]
+    rng = np.random.default_rng(78)
+    v1 = rng.random(g1.vol_shape).astype(np.float32)
+    v2 = rng.random(g2.vol_shape).astype(np.float32)
+    s = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(s):
+        t1, t2 = torch.from_numpy(v1).to(dev), torch.from_numpy(v2).to(dev)
+        y1 = _noalloc_forward(g1, t1, stream=s)
+        y2 = _noalloc_forward(g2, t2, stream=s)
+    s.synchronize()
+    check_forward(y1.cpu().numpy(), oracle.forward(g1, v1), oracle_chords(g1), min(g1.spacing), "first")
+    check_forward(y2.cpu().numpy(), oracle.forward(g2, v2), oracle_chords(g2), min(g2.spacing), "second")
+
+
+@pytest.mark.parametrize("n_cols", [1500, 33000])
+def test_noalloc_wide_cylindrical_detector(n_cols):
+    """Column rows packed several views to a copy (1500 columns) and a row
+    wider than the staging array, sent in pieces (33000 columns)."""
+    import torch
+    g = _wide_cylindrical(n_cols)
+    vol = np.random.default_rng(79).random(g.vol_shape).astype(np.float32)
+    got = _noalloc_forward(g, torch.from_numpy(vol).cuda())
+    torch.cuda.synchronize()
+    check_forward(got.cpu().numpy(), oracle.forward(g, vol), oracle_chords(g), min(g.spacing), f"{n_cols} cols")
+
+
+def test_noalloc_refuses_a_capturing_stream():
+    """Its uploads read host memory of the call itself, so a stream being
+    captured into a graph is refused before anything is enqueued."""
+    import torch
+    dev = torch.device("cuda", torch.cuda.current_device())
+    g = small_geometries()["cone_flat"]
+    vol = torch.rand(g.vol_shape, device=dev)
+    out = torch.zeros(g.sino_shape, dtype=torch.float32, device=dev)
+    s = torch.cuda.Stream(device=dev)
+    graph = torch.cuda.CUDAGraph()
+    torch.cuda.synchronize()
+    with torch.cuda.graph(graph, stream=s):
+        out.fill_(1.0)
+        with pytest.raises(ctp.CtpError) as ei:
+            ctp.ctp_forward_noalloc(g, vol, out, device=dev.index or 0, stream=s)
+    assert ei.value.status == ctp.CTP_ERR_UNSUPPORTED
+    graph.replay()
+    torch.cuda.synchronize()
+    assert bool((out == 1.0).all())
+    # outside the capture the same call works
+    got = _noalloc_forward(g, vol)
+    torch.cuda.synchronize()
+    assert torch.isfinite(got).all()
 
 
 def test_noalloc_rejects_a_description_beyond_its_scratch():
