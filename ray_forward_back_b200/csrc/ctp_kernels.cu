@@ -1319,13 +1319,25 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_ROWS_MIN_BLOCKS)
   float acc[kR];
 #pragma unroll
   for (int j = 0; j < kR; ++j) acc[j] = 0.f;
-  walk<true, false, 0, Off>(hit, W, lo, hi, off, W.step[0] * sx, W.step[1] * sy, (Off)0, nullptr,
-                            [&](Off o, float len, bool) {
+  // every row of the group inside the volume (the common case) takes the
+  // walk without per-row tests; the warp decides together
+  if (__all_sync(0xffffffffu, rows == (1u << kR) - 1u || !hit)) {
+    walk<true, false, 0, Off>(hit, W, lo, hi, off, W.step[0] * sx, W.step[1] * sy, (Off)0, nullptr,
+                              [&](Off o, float len, bool) {
 #pragma unroll
-                              for (int j = 0; j < kR; ++j)
-                                if ((rows & (1u << j)) && CTP_IN_BOUNDS(o + zoff[j], n_vox, 3))
-                                  acc[j] = fmaf(len, __ldg(base + o + zoff[j]), acc[j]);
-                            });
+                                for (int j = 0; j < kR; ++j)
+                                  if (CTP_IN_BOUNDS(o + zoff[j], n_vox, 3))
+                                    acc[j] = fmaf(len, __ldg(base + o + zoff[j]), acc[j]);
+                              });
+  } else {
+    walk<true, false, 0, Off>(hit, W, lo, hi, off, W.step[0] * sx, W.step[1] * sy, (Off)0, nullptr,
+                              [&](Off o, float len, bool) {
+#pragma unroll
+                                for (int j = 0; j < kR; ++j)
+                                  if ((rows & (1u << j)) && CTP_IN_BOUNDS(o + zoff[j], n_vox, 3))
+                                    acc[j] = fmaf(len, __ldg(base + o + zoff[j]), acc[j]);
+                              });
+  }
   if (cvalid) {
 #pragma unroll
     for (int j = 0; j < kR; ++j) {
@@ -1375,16 +1387,31 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_ROWS_MIN_BLOCKS)
   const Off sy = yfast ? (Off)1 : nx;
   const Off off = (Off)W.i[1] * sy + (Off)W.i[0] * sx;
   [[maybe_unused]] const size_t n_vox = (size_t)P.vol.n[0] * P.vol.n[1] * P.vol.n[2];
-  walk<true, false, kWalkAnchor, Off>(hit, W, lo, hi, off, W.step[0] * sx, W.step[1] * sy, (Off)0, anc,
-                                      [&](Off o, float len, bool) {
-                                        if (len > 0.f) {
-                                          const float w = coef<kPower>(len);
+  // every row of the group inside the volume with a non-zero value (the
+  // common case) takes the walk without per-row tests; the warp decides together
+  if (__all_sync(0xffffffffu, rows == (1u << kR) - 1u || !hit)) {
+    walk<true, false, kWalkAnchor, Off>(hit, W, lo, hi, off, W.step[0] * sx, W.step[1] * sy, (Off)0, anc,
+                                        [&](Off o, float len, bool) {
+                                          if (len > 0.f) {
+                                            const float w = coef<kPower>(len);
 #pragma unroll
-                                          for (int j = 0; j < kR; ++j)
-                                            if ((rows & (1u << j)) && CTP_IN_BOUNDS(o + zoff[j], n_vox, 11))
-                                              atomicAdd(base + o + zoff[j], w * y[j]);
-                                        }
-                                      });
+                                            for (int j = 0; j < kR; ++j)
+                                              if (CTP_IN_BOUNDS(o + zoff[j], n_vox, 11))
+                                                atomicAdd(base + o + zoff[j], w * y[j]);
+                                          }
+                                        });
+  } else {
+    walk<true, false, kWalkAnchor, Off>(hit, W, lo, hi, off, W.step[0] * sx, W.step[1] * sy, (Off)0, anc,
+                                        [&](Off o, float len, bool) {
+                                          if (len > 0.f) {
+                                            const float w = coef<kPower>(len);
+#pragma unroll
+                                            for (int j = 0; j < kR; ++j)
+                                              if ((rows & (1u << j)) && CTP_IN_BOUNDS(o + zoff[j], n_vox, 11))
+                                                atomicAdd(base + o + zoff[j], w * y[j]);
+                                          }
+                                        });
+  }
 }
 
 }  // namespace
