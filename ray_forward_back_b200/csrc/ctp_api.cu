@@ -591,7 +591,6 @@ ctp_status ctp_geom_create(const ctp_geom_desc *desc, ctp_geom **out) {
   for (const ViewRec &V : views)
     slices = slices && V.s[2] == 0.0 && V.dv[0] == 0.0 && V.dv[1] == 0.0;
   f.row_group = 1;
-  f.row_group_bands = f.n_row_bands;
   g->adjoint_variant = CTP_ADJOINT_BRICK;
   g->batch_chunk = plan && plan->batch_chunk > 0 ? plan->batch_chunk : 1;
 
@@ -622,7 +621,6 @@ ctp_status ctp_geom_create(const ctp_geom_desc *desc, ctp_geom **out) {
       }
     }
     f.row_group = rg;
-    f.row_group_bands = (int32_t)((g->n_rows + 8 * rg - 1) / (8 * rg));
   }
   if (ctp::back_brick_smem_bytes(g->back.brick) > 200 * 1024) {
     delete g;

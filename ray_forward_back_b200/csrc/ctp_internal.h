@@ -56,10 +56,9 @@ struct FwdLaunch {
   int32_t n_col_tiles, n_row_bands;
   int32_t any_transposed;
   // Rays in z-planes with rows stepping along z: each thread walks one (x, y)
-  // path for row_group rows (1 = one walk per ray); row_group_bands bands of
-  // 8 * row_group rows.  Used by the single-volume forward and the scatter
-  // adjoint.
-  int32_t row_group, row_group_bands;
+  // path for row_group rows (1 = one walk per ray).  Used by the
+  // single-volume forward and the scatter adjoint.
+  int32_t row_group, pad;
 };
 
 struct BackLaunch {

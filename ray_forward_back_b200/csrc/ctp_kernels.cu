@@ -1252,6 +1252,40 @@ __global__ void __launch_bounds__(256) transpose_add_kernel(const float* __restr
 #define CTP_ROWS_MIN_BLOCKS 4
 #endif
 
+// Block shape of the shared-slice kernels: 8 warps of 32 columns x kR rows,
+// kRowsGroups of them stacked along the rows and 8 / kRowsGroups side by side
+// along the columns.  A band (the rows of one block row) is kRowsGroups * kR
+// slices deep; blocks run band by band, every view of a band before the next,
+// so the slices the blocks in flight touch (the adjoint's accumulation
+// working set, in both volume layouts) stay few enough for L2.
+#ifndef CTP_ROWS_GROUPS
+#define CTP_ROWS_GROUPS 8
+#endif
+constexpr int kRowsGroups = CTP_ROWS_GROUPS;
+constexpr int kRowsColTiles = kFwdRows / kRowsGroups;
+static_assert(kRowsGroups * kRowsColTiles == kFwdRows, "row groups divide the block's warps");
+
+__host__ __device__ __forceinline__ int rows_col_tiles(int n_cols) {
+  return (n_cols + kFwdCols * kRowsColTiles - 1) / (kFwdCols * kRowsColTiles);
+}
+__host__ __device__ __forceinline__ int rows_bands(int n_rows, int r) {
+  return (n_rows + kRowsGroups * r - 1) / (kRowsGroups * r);
+}
+
+// View, column and first row of this thread in a shared-slice kernel.
+template <int kR>
+__device__ __forceinline__ void rows_block_position(const FwdLaunch& P, int& v, int& c, int& r0) {
+  const int ctiles = rows_col_tiles(P.dims.n_cols);
+  const int per_band = P.dims.n_views * ctiles;
+  const int band = blockIdx.x / per_band;
+  const int rem = blockIdx.x - band * per_band;
+  v = rem / ctiles;
+  const int ct = rem - v * ctiles;
+  const int w = threadIdx.y;
+  c = (ct * kRowsColTiles + w % kRowsColTiles) * kFwdCols + threadIdx.x;
+  r0 = (band * kRowsGroups + w / kRowsColTiles) * kR;
+}
+
 // Slice offsets of rows r0 .. r0 + kR - 1 of column c: bit j of the result is
 // set where row r0 + j exists and its rays' height falls inside the volume
 // (the z test of the ray's slab clip); zoff[j] is then that slice's offset.
@@ -1290,13 +1324,8 @@ template <typename Off, int kR>
 __global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_ROWS_MIN_BLOCKS)
     forward_rows_kernel(FwdLaunch P, const ViewRec* __restrict__ views, const float* __restrict__ vol,
                         const float* __restrict__ volT, float* __restrict__ sino) {
-  const int per_band = P.dims.n_views * P.n_col_tiles;
-  const int band = blockIdx.x / per_band;
-  const int rem = blockIdx.x - band * per_band;
-  const int v = rem / P.n_col_tiles;
-  const int ct = rem - v * P.n_col_tiles;
-  const int c = ct * kFwdCols + threadIdx.x;
-  const int r0 = (band * kFwdRows + threadIdx.y) * kR;
+  int v, c, r0;
+  rows_block_position<kR>(P, v, c, r0);
   const bool cvalid = c < P.dims.n_cols;
   const ViewRec& V = views[v];
   const Off nx = P.vol.n[0], ny = P.vol.n[1];
@@ -1353,13 +1382,8 @@ template <int kPower, typename Off, int kR>
 __global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_ROWS_MIN_BLOCKS)
     back_scatter_rows_kernel(FwdLaunch P, const ViewRec* __restrict__ views, const float* __restrict__ sino,
                              float* __restrict__ vol, float* __restrict__ volT) {
-  const int per_band = P.dims.n_views * P.n_col_tiles;
-  const int band = blockIdx.x / per_band;
-  const int rem = blockIdx.x - band * per_band;
-  const int v = rem / P.n_col_tiles;
-  const int ct = rem - v * P.n_col_tiles;
-  const int c = ct * kFwdCols + threadIdx.x;
-  const int r0 = (band * kFwdRows + threadIdx.y) * kR;
+  int v, c, r0;
+  rows_block_position<kR>(P, v, c, r0);
   const bool cvalid = c < P.dims.n_cols;
   const ViewRec& V = views[v];
   const Off nx = P.vol.n[0], ny = P.vol.n[1];
@@ -1433,7 +1457,8 @@ unsigned long long debug_take_word_kernels() {
 
 cudaError_t launch_forward_rows(const FwdLaunch& p, const ViewRec* views, const float* vol, const float* volT,
                                 float* sino, bool wide_index, cudaStream_t stream) {
-  const long long blocks = (long long)p.row_group_bands * p.dims.n_views * p.n_col_tiles;
+  const long long blocks =
+      (long long)rows_bands(p.dims.n_rows, p.row_group) * p.dims.n_views * rows_col_tiles(p.dims.n_cols);
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   dim3 block(kFwdCols, kFwdRows);
@@ -1464,7 +1489,8 @@ cudaError_t launch_back_scatter(const FwdLaunch& p, const ViewRec* views, const 
   dim3 block(kFwdCols, kFwdRows);
   const unsigned nb = (unsigned)blocks;
   if (p.row_group > 1) {
-    const long long rb = (long long)p.row_group_bands * p.dims.n_views * p.n_col_tiles;
+    const long long rb =
+        (long long)rows_bands(p.dims.n_rows, p.row_group) * p.dims.n_views * rows_col_tiles(p.dims.n_cols);
     if (rb > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     const unsigned nr = (unsigned)rb;
 #define CTP_SROWS(KP, OFF, R) back_scatter_rows_kernel<KP, OFF, R><<<nr, block, 0, stream>>>(p, views, sino, vol, volT)
