@@ -75,20 +75,20 @@ def code_digest(paths):
 
 
 def kernel_counters(kernel, workload_index):
-    """Committed ncu counters of `kernel` (profiles/kernel_counters.json),
-    captured on a view subset of the workload: DRAM bytes and warp
-    instructions per launch there, and the ray-voxel updates of that subset.
-    None when the capture is for another workload or the kernel's code has
-    changed since it was taken (a digest of its sources without comments or
-    whitespace)."""
+    """Committed ncu counters of `kernel` on workload `workload_index`
+    (profiles/kernel_counters.json), captured on a view subset of it: DRAM
+    bytes and warp instructions per launch there, and the ray-voxel updates
+    of that subset.  None when there is no capture for that workload or the
+    kernel's code has changed since it was taken (a digest of its sources
+    without comments or whitespace)."""
     path = os.path.join(ROOT, "profiles", "kernel_counters.json")
     try:
         with open(path) as f:
-            k = json.load(f)["kernels"][kernel]
+            k = json.load(f)["kernels"][kernel][str(workload_index)]
         digest = code_digest(k["sources"])
     except Exception:
         return None
-    if digest != k.get("code_sha256") or workload_index != k.get("workload"):
+    if digest != k.get("code_sha256"):
         return None
     return k
 
@@ -263,10 +263,22 @@ def select_workload(args):
     from ray_forward_back_b200 import workloads as W
     wl = W.workload(args.workload)
     if args.views and args.views < wl.geom.n_views:
-        views = np.linspace(0, wl.geom.n_views - 1, args.views).round().astype(np.int64)
-        wl = dataclasses.replace(wl, geom=wl.geom.subset_views(views),
-                                 name=f"{wl.name} (views subset: {args.views})")
+        if args.first >= 0:
+            views = np.arange(args.first, min(args.first + args.views, wl.geom.n_views))
+            what = f"views {views[0]}-{views[-1]}"
+        else:
+            views = np.linspace(0, wl.geom.n_views - 1, args.views).round().astype(np.int64)
+            what = f"views subset: {args.views}"
+        wl = dataclasses.replace(wl, geom=wl.geom.subset_views(views), name=f"{wl.name} ({what})")
     return wl
+
+
+VARIANTS = {"auto": 0, "brick": 1, "sort": 2, "scatter": 3}
+
+
+def plan_of(args):
+    """Plan overrides from the command line (none by default)."""
+    return {"adjoint_variant": VARIANTS[args.variant]} if args.variant != "auto" else None
 
 
 def run_reference(args, rank, world):
@@ -508,7 +520,7 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     wl = select_workload(args)
     g = wl.geom
-    P = ctp.Projector(g, device=local_rank)
+    P = ctp.Projector(g, device=local_rank, plan=plan_of(args))
     info = P.info()
     stream = torch.cuda.Stream(device=dev)
     vol_host = wl.phantom()
@@ -804,6 +816,10 @@ def main():
     ap.add_argument("--workload", type=int, default=4)
     ap.add_argument("--views", type=int, default=0,
                     help="use this many evenly spaced views of the workload (0 = all); for profiling")
+    ap.add_argument("--first", type=int, default=-1,
+                    help="with --views: take that many consecutive views from this one instead")
+    ap.add_argument("--variant", choices=sorted(VARIANTS), default="auto",
+                    help="force an adjoint variant (default: the plan's automatic choice)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
