@@ -14,11 +14,14 @@
  *
  * Precision: per-ray clipping and entry setup in FP64, traversal and data in
  * FP32 (same page, table row backend="numba", and its paragraph on segment
- * setup from the endpoint nearer the volume centre).  The adjoint sums its
- * contributions exactly as 32-bit fixed point inside each block of the
- * volume (scale chosen per stage of views so that no voxel can overflow) and
- * adds the stages into the FP32 volume, so its result does not depend on
- * thread scheduling; the forward projection is deterministic as well.
+ * setup from the endpoint nearer the volume centre); walks that run the
+ * whole volume re-derive their FP32 parameters from the FP64 set-up every 64
+ * slabs.  The forward projection is deterministic.  The automatic adjoints
+ * (ray scatter, sort / segment-reduce) add FP32 contributions with global
+ * atomics, so their last bits depend on scheduling (the pages promise no
+ * bitwise determinism for scatter accumulation, same page); the brick
+ * adjoint, available through the plan, sums exactly as 32-bit fixed point
+ * inside each block of the volume and is bitwise reproducible.
  *
  * Layouts (same page, "Batch dimensions and axis spacing"):
  *   volume    float32 [nz][ny][nx], x fastest, contiguous
@@ -74,7 +77,12 @@ typedef enum {
 enum { CTP_BEAM_PARALLEL = 0, CTP_BEAM_CONE = 1 };
 enum { CTP_DET_FLAT = 0, CTP_DET_CYLINDRICAL = 1 };
 
-/* Adjoint variants.  AUTO picks by the collision ratio measured at create. */
+/* Adjoint variants.  AUTO picks by the collision ratio measured at create:
+ * SCATTER (one global float add per ray-voxel segment, off the forward's
+ * walk) below 13.5 contributions per distinct voxel of a warp batch, SORT
+ * (warp sort and segmented sum, one add per distinct voxel) above.  BRICK
+ * (shared-memory fixed point per voxel block) is never chosen automatically;
+ * it is the bitwise-reproducible variant. */
 enum { CTP_ADJOINT_AUTO = 0, CTP_ADJOINT_BRICK = 1, CTP_ADJOINT_SORT = 2, CTP_ADJOINT_SCATTER = 3 };
 
 /* Optional plan overrides (all zero = library defaults). */
@@ -85,7 +93,8 @@ typedef struct {
   int32_t forward_layout;    /* 0 = automatic per view, 1 = always x-fastest volume, 2 = always y-fastest */
   int32_t batch_chunk;       /* ctp_forward_batch: volumes per fused launch, 1, 2 or 4; 0 = 1.  The
                                 y-fastest scratch copy (if any view uses it) grows by this factor.
-                                2 or 4 also lets ctp_back_batch take member pairs in one launch. */
+                                2 or 4 also lets the brick adjoint of ctp_back_batch take member pairs
+                                in one launch. */
   int32_t slice_rows;        /* parallel beams whose rays lie in z-planes and whose rows step along z:
                                 detector rows that share one (x, y) path per thread, 2, 4 or 8 (one walk
                                 serves that many slices); 1 = one walk per ray; 0 = automatic */
@@ -114,7 +123,7 @@ typedef struct {
 typedef struct {
   int64_t n_rays, n_vox;
   int64_t scratch_bytes;        /* device memory the handle owns */
-  int32_t adjoint_variant;      /* variant ctp_back will run (BRICK or SORT) */
+  int32_t adjoint_variant;      /* variant ctp_back will run (BRICK, SORT or SCATTER) */
   int32_t brick[3];
   int32_t view_groups;
   int32_t n_transposed_views;   /* views whose forward gathers from the y-fastest copy */
@@ -164,8 +173,10 @@ ctp_status ctp_forward(const ctp_geom *geom, const float *vol, float *sino, void
  * sino: device pointer, float32 [n_views][n_rows][n_cols], read only.
  * vol:  device pointer, float32 [nz][ny][nx], overwritten.
  * Same pointer, stream and synchronisation rules as ctp_forward.  A
- * non-finite sinogram value (NaN or infinity) is not dropped: every voxel of
- * each volume block whose detector footprint holds it is written as NaN.
+ * non-finite sinogram value (NaN or infinity) is not dropped: with the
+ * scatter and sort adjoints it reaches every voxel its ray crosses (NaN, or
+ * an infinity); with the brick adjoint every voxel of each volume block whose
+ * detector footprint holds it is written as NaN.
  */
 ctp_status ctp_back(const ctp_geom *geom, const float *sino, float *vol, void *stream);
 
@@ -183,8 +194,8 @@ ctp_status ctp_back(const ctp_geom *geom, const float *sino, float *vol, void *s
  * across the chunk; each member's sinogram is bit-identical to ctp_forward's.
  * With plan.batch_chunk >= 2 the brick adjoint takes member pairs in one
  * launch (its brick halved along y); their volumes then differ from
- * ctp_back's by fixed-point rounding only.  Otherwise, and for the sort
- * adjoint, it runs member by member.  n_batch < 0, or a
+ * ctp_back's by fixed-point rounding only.  Otherwise, and for the scatter
+ * and sort adjoints, it runs member by member.  n_batch < 0, or a
  * batch whose element count exceeds 2^62, gives CTP_ERR_INVALID_ARGUMENT.
  * Same pointer, stream and synchronisation rules as ctp_forward / ctp_back.
  */
