@@ -34,6 +34,9 @@ struct ctp_geom {
   ViewRec *d_views = nullptr;
   double *d_trig = nullptr;
   float *d_volT = nullptr;
+  float4 *d_vol4 = nullptr;   // volume interleaved by 4 slices (and its y-fastest twin), shared slice walks
+  int64_t n_vol4 = 0;         // float4 elements of one interleaved copy
+  bool wide4 = false;         // 64-bit offsets for the interleaved copies
   unsigned long long *d_counter = nullptr;
   int64_t scratch_bytes = 0;
   int batch_chunk = 1;  // volumes per fused batched forward launch (y-fastest copies held)
@@ -416,6 +419,7 @@ void free_geom(ctp_geom *g) {
   cudaFree(g->d_views);
   cudaFree(g->d_trig);
   cudaFree(g->d_volT);
+  cudaFree(g->d_vol4);
   cudaFree(g->d_counter);
   delete g;
 }
@@ -621,6 +625,12 @@ ctp_status ctp_geom_create(const ctp_geom_desc *desc, ctp_geom **out) {
       }
     }
     f.row_group = rg;
+#ifndef CTP_NO_INTERLEAVE
+    // four rows per walk read and add 16 bytes at once from slices interleaved by 4
+    f.interleaved = rg == 4;
+#endif
+    g->n_vol4 = (g->nz + 3) / 4 * g->nx * g->ny;
+    g->wide4 = g->wide_index || 4 * g->n_vol4 >= (int64_t)0x7fffffff;
   }
   if (ctp::back_brick_smem_bytes(g->back.brick) > 200 * 1024) {
     delete g;
@@ -642,6 +652,9 @@ ctp_status ctp_geom_create(const ctp_geom_desc *desc, ctp_geom **out) {
   if (st == CTP_OK && f.any_transposed)
     st = alloc((void **)&g->d_volT, sizeof(float) * (size_t)g->n_vox * (size_t)g->batch_chunk,
                "y-fastest volume copies");
+  if (st == CTP_OK && f.interleaved)
+    st = alloc((void **)&g->d_vol4, sizeof(float4) * (size_t)g->n_vol4 * (f.any_transposed ? 2 : 1),
+               "volumes interleaved by 4 slices");
   if (st == CTP_OK) st = alloc((void **)&g->d_counter, sizeof(unsigned long long), "counter");
   cudaError_t e = cudaSuccess;
   if (st == CTP_OK) {
@@ -706,6 +719,11 @@ ctp_status ctp_forward(const ctp_geom *g, const float *vol, float *sino, void *s
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pending error before ctp_forward");
+  if (g->fwd.interleaved) {
+    e = ctp::launch_forward_rows4(g->fwd, g->d_views, vol, g->d_vol4, g->d_vol4 + g->n_vol4, sino, g->wide4, s);
+    if (e != cudaSuccess) return cuda_fail(e, "forward launch");
+    return CTP_OK;
+  }
   if (g->fwd.any_transposed) {
     e = ctp::launch_transpose_xy(vol, g->d_volT, g->vol, s);
     if (e != cudaSuccess) return cuda_fail(e, "transpose launch");
@@ -820,6 +838,15 @@ ctp_status ctp_back_power(const ctp_geom *g, const float *sino, float *vol, int 
   if (e != cudaSuccess) return cuda_fail(e, "pending error before ctp_back");
   const bool sorted = g->adjoint_variant == CTP_ADJOINT_SORT;
   const bool scatter = g->adjoint_variant == CTP_ADJOINT_SCATTER;
+  if (scatter && g->fwd.interleaved) {
+    // accumulate into the zeroed interleaved copies; their sum overwrites vol
+    e = cudaMemsetAsync(g->d_vol4, 0, sizeof(float4) * (size_t)g->n_vol4 * (g->fwd.any_transposed ? 2 : 1), s);
+    if (e != cudaSuccess) return cuda_fail(e, "accumulator zero-fill");
+    e = ctp::launch_back_scatter_rows4(g->fwd, g->d_views, sino, vol, g->d_vol4, g->d_vol4 + g->n_vol4, power,
+                                       g->wide4, s);
+    if (e != cudaSuccess) return cuda_fail(e, "adjoint launch");
+    return CTP_OK;
+  }
   if (sorted || scatter || g->back.view_groups > 1) {
     e = cudaMemsetAsync(vol, 0, sizeof(float) * (size_t)g->n_vox, s);
     if (e == cudaSuccess && scatter && g->fwd.any_transposed)

@@ -58,7 +58,8 @@ struct FwdLaunch {
   // Rays in z-planes with rows stepping along z: each thread walks one (x, y)
   // path for row_group rows (1 = one walk per ray).  Used by the
   // single-volume forward and the scatter adjoint.
-  int32_t row_group, pad;
+  int32_t row_group;
+  int32_t interleaved;  // row_group 4 on volumes interleaved by 4 slices (the rows4 kernels)
 };
 
 struct BackLaunch {
@@ -83,6 +84,15 @@ cudaError_t launch_forward(const FwdLaunch& p, const ViewRec* views, const doubl
 // The single-volume forward with one (x, y) walk per p.row_group rows.
 cudaError_t launch_forward_rows(const FwdLaunch& p, const ViewRec* views, const float* vol, const float* volT,
                                 float* sino, bool wide_index, cudaStream_t stream);
+// Slices interleaved by 4 (element [g][y][x][s] = slice 4g + s; vol4T with x
+// and y swapped): the forward interleaves vol into vol4 (and vol4T if some
+// view gathers y-fastest), then walks 4 rows per thread reading 16 bytes per
+// segment; the adjoint adds into the zeroed acc4 / acc4T with 16-byte
+// reductions, then writes vol from them.
+cudaError_t launch_forward_rows4(const FwdLaunch& p, const ViewRec* views, const float* vol, float4* vol4,
+                                 float4* vol4T, float* sino, bool wide_index, cudaStream_t stream);
+cudaError_t launch_back_scatter_rows4(const FwdLaunch& p, const ViewRec* views, const float* sino, float* vol,
+                                      float4* acc4, float4* acc4T, int power, bool wide_index, cudaStream_t stream);
 cudaError_t launch_back_brick(const BackLaunch& p, const ViewRec* views, const double* trig, const float* sino,
                               float* vol, int power, int kb, bool wide_index, cudaStream_t stream);
 cudaError_t launch_count(const FwdLaunch& p, const ViewRec* views, const double* trig,

@@ -1286,12 +1286,12 @@ __device__ __forceinline__ void rows_block_position(const FwdLaunch& P, int& v, 
   r0 = (band * kRowsGroups + w / kRowsColTiles) * kR;
 }
 
-// Slice offsets of rows r0 .. r0 + kR - 1 of column c: bit j of the result is
-// set where row r0 + j exists and its rays' height falls inside the volume
-// (the z test of the ray's slab clip); zoff[j] is then that slice's offset.
-template <int kR, typename Off>
-__device__ __forceinline__ unsigned row_slices(const ViewRec& V, const VolDesc& G, int r0, int c, int n_rows, Off sz,
-                                               Off zoff[kR]) {
+// Slices of rows r0 .. r0 + kR - 1 of column c: bit j of the result is set
+// where row r0 + j exists and its rays' height falls inside the volume (the z
+// test of the ray's slab clip); ks[j] is then that slice.
+template <int kR>
+__device__ __forceinline__ unsigned row_slice_index(const ViewRec& V, const VolDesc& G, int r0, int c, int n_rows,
+                                                    int ks[kR]) {
   unsigned mask = 0u;
 #pragma unroll
   for (int j = 0; j < kR; ++j) {
@@ -1302,9 +1302,20 @@ __device__ __forceinline__ unsigned row_slices(const ViewRec& V, const VolDesc& 
     const T pz = fma((T)r, (T)V.dv[2], fma((T)c, (T)V.du[2], (T)V.p00[2]));
     const T az = (pz - (T)G.origin[2]) * (T)G.inv_spacing[2];
     const bool in = r < n_rows && az >= (T)0 && az < (T)G.n[2];
-    zoff[j] = in ? (Off)clampi((int)floor(az), 0, G.n[2] - 1) * sz : (Off)0;
+    ks[j] = in ? clampi((int)floor(az), 0, G.n[2] - 1) : 0;
     mask |= in ? 1u << j : 0u;
   }
+  return mask;
+}
+
+// The same, as offsets of the slices (zoff[j] = slice * sz).
+template <int kR, typename Off>
+__device__ __forceinline__ unsigned row_slices(const ViewRec& V, const VolDesc& G, int r0, int c, int n_rows, Off sz,
+                                               Off zoff[kR]) {
+  int ks[kR];
+  const unsigned mask = row_slice_index<kR>(V, G, r0, c, n_rows, ks);
+#pragma unroll
+  for (int j = 0; j < kR; ++j) zoff[j] = (mask & (1u << j)) ? (Off)ks[j] * sz : (Off)0;
   return mask;
 }
 
@@ -1438,9 +1449,263 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_ROWS_MIN_BLOCKS)
   }
 }
 
+// ------------------------------- parallel slices: volumes interleaved by 4 --
+//
+// Slices taken in groups of four and interleaved: element [g][y][x][s] holds
+// slice 4g + s ([g][x][y][s] for the copy whose fastest axes are swapped),
+// with ng = ceil(nz / 4) groups and the slices past nz zero.  A thread of a
+// shared (x, y) walk over 4 rows whose heights fall in the 4 slices of one
+// group (the common case, rows and slices of equal pitch) then reads its 4
+// values with one 16-byte load, or adds its 4 contributions with one 16-byte
+// reduction; any other row group addresses single elements.  Each row still
+// sees exactly its own segments, in the same order.
+
+// slices 4g .. 4g + 3 of the rows' heights, in order
+__device__ __forceinline__ bool one_group(unsigned rows, const int ks[4]) {
+  return rows == 0xfu && (ks[0] & 3) == 0 && ks[1] == ks[0] + 1 && ks[2] == ks[0] + 2 && ks[3] == ks[0] + 3;
+}
+
+template <typename Off>
+__global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_ROWS_MIN_BLOCKS)
+    forward_rows4_kernel(FwdLaunch P, const ViewRec* __restrict__ views, const float4* __restrict__ vol4,
+                         const float4* __restrict__ vol4T, float* __restrict__ sino) {
+  int v, c, r0;
+  rows_block_position<4>(P, v, c, r0);
+  const bool cvalid = c < P.dims.n_cols;
+  const ViewRec& V = views[v];
+  const Off nx = P.vol.n[0], ny = P.vol.n[1];
+  const Off plane = nx * ny;
+  [[maybe_unused]] const Off n4 = (Off)((P.vol.n[2] + 3) >> 2) * plane;  // float4 elements of one copy
+  int ks[4];
+  const unsigned rows = cvalid ? row_slice_index<4>(V, P.vol, r0, c, P.dims.n_rows, ks) : 0u;
+  Ray R;
+  setup_t t_in = 0, t_out = 0;
+  const bool hit = slice_ray(V, P.vol, P.dims, v, cvalid ? c : 0, R, t_in, t_out) && rows != 0u;
+  const int lo[3] = {0, 0, 0};
+  const int hi[3] = {P.vol.n[0], P.vol.n[1], P.vol.n[2]};
+  Walk W = {};
+  if (hit) entry(R, t_in, t_out, lo, hi, W);
+  const bool yfast = V.layout != 0;
+  const float4* __restrict__ base4 = yfast ? vol4T : vol4;
+  const float* __restrict__ base1 = reinterpret_cast<const float*>(base4);
+  const Off sx = yfast ? ny : (Off)1;
+  const Off sy = yfast ? (Off)1 : nx;
+  const Off off = (Off)W.i[1] * sy + (Off)W.i[0] * sx;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  if (__all_sync(0xffffffffu, one_group(rows, ks) || !hit)) {
+    const Off g = (Off)(ks[0] >> 2) * plane;
+    walk<true, false, 0, Off>(hit, W, lo, hi, off, W.step[0] * sx, W.step[1] * sy, (Off)0, nullptr,
+                              [&](Off o, float len, bool) {
+                                if (CTP_IN_BOUNDS(g + o, n4, 15)) {
+                                  const float4 q = __ldg(base4 + g + o);
+                                  acc[0] = fmaf(len, q.x, acc[0]);
+                                  acc[1] = fmaf(len, q.y, acc[1]);
+                                  acc[2] = fmaf(len, q.z, acc[2]);
+                                  acc[3] = fmaf(len, q.w, acc[3]);
+                                }
+                              });
+  } else {
+    Off e[4];  // float index of row j's slice at (x, y) = (0, 0)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) e[j] = ((Off)(ks[j] >> 2) * plane) * 4 + (ks[j] & 3);
+    walk<true, false, 0, Off>(hit, W, lo, hi, off, W.step[0] * sx, W.step[1] * sy, (Off)0, nullptr,
+                              [&](Off o, float len, bool) {
+#pragma unroll
+                                for (int j = 0; j < 4; ++j)
+                                  if ((rows & (1u << j)) && CTP_IN_BOUNDS(e[j] + 4 * o, 4 * n4, 16))
+                                    acc[j] = fmaf(len, __ldg(base1 + e[j] + 4 * o), acc[j]);
+                              });
+  }
+  if (cvalid) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int r = r0 + j;
+      const size_t i = ((size_t)v * P.dims.n_rows + r) * P.dims.n_cols + c;
+      if (r < P.dims.n_rows && CTP_IN_BOUNDS(i, (size_t)P.dims.n_views * P.dims.n_rows * P.dims.n_cols, 4))
+        sino[i] = acc[j];
+    }
+  }
+}
+
+template <int kPower, typename Off>
+__global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_ROWS_MIN_BLOCKS)
+    back_scatter_rows4_kernel(FwdLaunch P, const ViewRec* __restrict__ views, const float* __restrict__ sino,
+                              float4* __restrict__ acc4, float4* __restrict__ acc4T) {
+  int v, c, r0;
+  rows_block_position<4>(P, v, c, r0);
+  const bool cvalid = c < P.dims.n_cols;
+  const ViewRec& V = views[v];
+  const Off nx = P.vol.n[0], ny = P.vol.n[1];
+  const Off plane = nx * ny;
+  [[maybe_unused]] const Off n4 = (Off)((P.vol.n[2] + 3) >> 2) * plane;
+  int ks[4];
+  const unsigned inside = cvalid ? row_slice_index<4>(V, P.vol, r0, c, P.dims.n_rows, ks) : 0u;
+  float y[4];
+  unsigned rows = inside;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    y[j] = (inside & (1u << j)) ? __ldg(sino + ((size_t)v * P.dims.n_rows + r0 + j) * P.dims.n_cols + c) : 0.f;
+    if (!(y[j] != 0.f)) rows &= ~(1u << j);  // zero rows add nothing (NaN stays)
+  }
+  Ray R;
+  setup_t t_in = 0, t_out = 0;
+  const bool hit = slice_ray(V, P.vol, P.dims, v, cvalid ? c : 0, R, t_in, t_out) && rows != 0u;
+  const int lo[3] = {0, 0, 0};
+  const int hi[3] = {P.vol.n[0], P.vol.n[1], P.vol.n[2]};
+  Walk W = {};
+  __shared__ double s_anc[7 * kAncStride];
+  double* const anc = s_anc + threadIdx.y * kFwdCols + threadIdx.x;
+  if (hit) entry(R, t_in, t_out, lo, hi, W, anc, kAncStride);
+  const bool yfast = V.layout != 0;
+  float4* const base4 = yfast ? acc4T : acc4;
+  float* const base1 = reinterpret_cast<float*>(base4);
+  const Off sx = yfast ? ny : (Off)1;
+  const Off sy = yfast ? (Off)1 : nx;
+  const Off off = (Off)W.i[1] * sy + (Off)W.i[0] * sx;
+  // a group of 4 rows in the 4 slices of one group adds the 4 contributions
+  // of a segment with one 16-byte reduction (a zero row adds zeros)
+  if (__all_sync(0xffffffffu, one_group(inside, ks) || !hit)) {
+    const Off g = (Off)(ks[0] >> 2) * plane;
+    walk<true, false, kWalkAnchor, Off>(hit, W, lo, hi, off, W.step[0] * sx, W.step[1] * sy, (Off)0, anc,
+                                        [&](Off o, float len, bool) {
+                                          if (len > 0.f && CTP_IN_BOUNDS(g + o, n4, 17)) {
+                                            const float w = coef<kPower>(len);
+                                            atomicAdd(base4 + g + o, make_float4(w * y[0], w * y[1], w * y[2], w * y[3]));
+                                          }
+                                        });
+  } else {
+    Off e[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) e[j] = ((Off)(ks[j] >> 2) * plane) * 4 + (ks[j] & 3);
+    walk<true, false, kWalkAnchor, Off>(hit, W, lo, hi, off, W.step[0] * sx, W.step[1] * sy, (Off)0, anc,
+                                        [&](Off o, float len, bool) {
+                                          if (len > 0.f) {
+                                            const float w = coef<kPower>(len);
+#pragma unroll
+                                            for (int j = 0; j < 4; ++j)
+                                              if ((rows & (1u << j)) && CTP_IN_BOUNDS(e[j] + 4 * o, 4 * n4, 18))
+                                                atomicAdd(base1 + e[j] + 4 * o, w * y[j]);
+                                          }
+                                        });
+  }
+}
+
+// Slices of vol [nz][ny][nx] interleaved by 4 into out4 [ng][ny][nx] and, if
+// given, out4T [ng][nx][ny].  One block: a 32 x 32 (x, y) tile of one group.
+__global__ void __launch_bounds__(256) interleave_kernel(const float* __restrict__ in, float4* __restrict__ out4,
+                                                         float4* __restrict__ out4T, int nx, int ny, int nz) {
+  __shared__ float tile[4][32][33];
+  const int g = blockIdx.z, x0 = blockIdx.x * 32, y0 = blockIdx.y * 32;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    const int z = 4 * g + s;
+    for (int j = ty; j < 32; j += 8) {
+      const int x = x0 + tx, y = y0 + j;
+      tile[s][j][tx] = (x < nx && y < ny && z < nz) ? in[((size_t)z * ny + y) * nx + x] : 0.f;
+    }
+  }
+  __syncthreads();
+  for (int j = ty; j < 32; j += 8) {
+    const int x = x0 + tx, y = y0 + j;
+    if (x < nx && y < ny)
+      out4[((size_t)g * ny + y) * nx + x] = make_float4(tile[0][j][tx], tile[1][j][tx], tile[2][j][tx], tile[3][j][tx]);
+  }
+  if (out4T) {
+    for (int j = ty; j < 32; j += 8) {
+      const int y = y0 + tx, x = x0 + j;
+      if (x < nx && y < ny)
+        out4T[((size_t)g * nx + x) * ny + y] =
+            make_float4(tile[0][tx][j], tile[1][tx][j], tile[2][tx][j], tile[3][tx][j]);
+    }
+  }
+}
+
+// out [nz][ny][nx] = acc4 [ng][ny][nx] (+ acc4T [ng][nx][ny]), slice by slice.
+__global__ void __launch_bounds__(256) deinterleave_kernel(const float4* __restrict__ acc4,
+                                                           const float4* __restrict__ acc4T, float* __restrict__ out,
+                                                           int nx, int ny, int nz) {
+  __shared__ float tile[4][32][33];
+  const int g = blockIdx.z, x0 = blockIdx.x * 32, y0 = blockIdx.y * 32;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  for (int j = ty; j < 32; j += 8) {
+    const int x = x0 + tx, y = y0 + j;
+    const float4 a = (x < nx && y < ny) ? acc4[((size_t)g * ny + y) * nx + x] : make_float4(0.f, 0.f, 0.f, 0.f);
+    tile[0][j][tx] = a.x;
+    tile[1][j][tx] = a.y;
+    tile[2][j][tx] = a.z;
+    tile[3][j][tx] = a.w;
+  }
+  if (acc4T) {
+    __syncthreads();
+    for (int j = ty; j < 32; j += 8) {
+      const int y = y0 + tx, x = x0 + j;
+      const float4 b =
+          (x < nx && y < ny) ? acc4T[((size_t)g * nx + x) * ny + y] : make_float4(0.f, 0.f, 0.f, 0.f);
+      tile[0][tx][j] += b.x;
+      tile[1][tx][j] += b.y;
+      tile[2][tx][j] += b.z;
+      tile[3][tx][j] += b.w;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    const int z = 4 * g + s;
+    if (z >= nz) break;
+    for (int j = ty; j < 32; j += 8) {
+      const int x = x0 + tx, y = y0 + j;
+      if (x < nx && y < ny) out[((size_t)z * ny + y) * nx + x] = tile[s][j][tx];
+    }
+  }
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------- launchers --
+
+cudaError_t launch_forward_rows4(const FwdLaunch& p, const ViewRec* views, const float* vol, float4* vol4,
+                                 float4* vol4T, float* sino, bool wide_index, cudaStream_t stream) {
+  const int ng = (p.vol.n[2] + 3) / 4;
+  dim3 tgrid((p.vol.n[0] + 31) / 32, (p.vol.n[1] + 31) / 32, ng);
+  interleave_kernel<<<tgrid, dim3(32, 8), 0, stream>>>(vol, vol4, p.any_transposed ? vol4T : nullptr, p.vol.n[0],
+                                                      p.vol.n[1], p.vol.n[2]);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const long long blocks = (long long)rows_bands(p.dims.n_rows, 4) * p.dims.n_views * rows_col_tiles(p.dims.n_cols);
+  if (blocks <= 0) return cudaSuccess;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  if (wide_index)
+    forward_rows4_kernel<long long><<<(unsigned)blocks, dim3(kFwdCols, kFwdRows), 0, stream>>>(p, views, vol4, vol4T,
+                                                                                                sino);
+  else
+    forward_rows4_kernel<int><<<(unsigned)blocks, dim3(kFwdCols, kFwdRows), 0, stream>>>(p, views, vol4, vol4T, sino);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_back_scatter_rows4(const FwdLaunch& p, const ViewRec* views, const float* sino, float* vol,
+                                      float4* acc4, float4* acc4T, int power, bool wide_index, cudaStream_t stream) {
+  const long long blocks = (long long)rows_bands(p.dims.n_rows, 4) * p.dims.n_views * rows_col_tiles(p.dims.n_cols);
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  if (blocks > 0) {
+    const unsigned nb = (unsigned)blocks;
+    const dim3 block(kFwdCols, kFwdRows);
+    if (power == 2) {
+      if (wide_index) back_scatter_rows4_kernel<2, long long><<<nb, block, 0, stream>>>(p, views, sino, acc4, acc4T);
+      else back_scatter_rows4_kernel<2, int><<<nb, block, 0, stream>>>(p, views, sino, acc4, acc4T);
+    } else {
+      if (wide_index) back_scatter_rows4_kernel<1, long long><<<nb, block, 0, stream>>>(p, views, sino, acc4, acc4T);
+      else back_scatter_rows4_kernel<1, int><<<nb, block, 0, stream>>>(p, views, sino, acc4, acc4T);
+    }
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  const int ng = (p.vol.n[2] + 3) / 4;
+  dim3 tgrid((p.vol.n[0] + 31) / 32, (p.vol.n[1] + 31) / 32, ng);
+  deinterleave_kernel<<<tgrid, dim3(32, 8), 0, stream>>>(acc4, p.any_transposed ? acc4T : nullptr, vol, p.vol.n[0],
+                                                        p.vol.n[1], p.vol.n[2]);
+  return cudaGetLastError();
+}
 
 // The bounds-check word of this file's kernels (CTP_DEBUG builds; 0 elsewhere),
 // read and cleared.  Synchronous.
