@@ -119,9 +119,10 @@ def issue_fraction(kernel, workload_index, updates_per_s, sm_mhz, n_sm):
 def kernel_names(info):
     """Names of the step's forward and adjoint kernels for this plan."""
     rows = info.get("slice_rows", 1) > 1
-    fwd = "forward_rows_kernel" if rows else "forward_kernel"
+    inter = "4" if info.get("interleaved_slices") else ""
+    fwd = f"forward_rows{inter}_kernel" if rows else "forward_kernel"
     back = {1: "back_brick_kernel", 2: "back_sort_kernel",
-            3: "back_scatter_rows_kernel" if rows else "back_scatter_kernel"}[info["adjoint_variant"]]
+            3: f"back_scatter_rows{inter}_kernel" if rows else "back_scatter_kernel"}[info["adjoint_variant"]]
     return fwd, back
 
 
@@ -129,6 +130,10 @@ def launches_per_step(info):
     """Kernels of the library launched by one forward + one back projection
     (memsets are not kernels of the library)."""
     t = 1 if info["n_transposed_views"] > 0 else 0
+    if info.get("interleaved_slices") and info["adjoint_variant"] == 3:
+        return 4                      # interleave + forward, adjoint + deinterleave
+    if info.get("interleaved_slices"):
+        return 2 + 1                  # interleave + forward, adjoint
     fwd = 1 + t                       # transpose_xy + forward
     back = 1 + (t if info["adjoint_variant"] == 3 else 0)   # + transpose_add for the scatter adjoint
     return fwd + back
@@ -278,7 +283,12 @@ VARIANTS = {"auto": 0, "brick": 1, "sort": 2, "scatter": 3}
 
 def plan_of(args):
     """Plan overrides from the command line (none by default)."""
-    return {"adjoint_variant": VARIANTS[args.variant]} if args.variant != "auto" else None
+    plan = {}
+    if args.variant != "auto":
+        plan["adjoint_variant"] = VARIANTS[args.variant]
+    if args.slice_rows:
+        plan["slice_rows"] = args.slice_rows
+    return plan or None
 
 
 def run_reference(args, rank, world):
@@ -820,6 +830,8 @@ def main():
                     help="with --views: take that many consecutive views from this one instead")
     ap.add_argument("--variant", choices=sorted(VARIANTS), default="auto",
                     help="force an adjoint variant (default: the plan's automatic choice)")
+    ap.add_argument("--slice-rows", type=int, default=0, choices=[0, 1, 2, 4, 8],
+                    help="force the detector rows per shared (x, y) walk (default: automatic)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -130,6 +130,8 @@ typedef struct {
   double collision_ratio;       /* updates / distinct voxels per sort batch, measured at create */
   int32_t batch_chunk;          /* volumes per fused ctp_forward_batch launch */
   int32_t slice_rows;           /* detector rows per shared (x, y) walk (1 = one walk per ray) */
+  int32_t interleaved_slices;   /* 1: shared walks of 4 rows run on copies interleaved by 4 slices */
+  int32_t reserved;
 } ctp_geom_info;
 
 /*
@@ -191,7 +193,9 @@ ctp_status ctp_back(const ctp_geom *geom, const float *sino, float *vol, void *s
  * does nothing and returns CTP_OK without looking at the pointers).
  * The forward walks every ray once per chunk of plan.batch_chunk members and
  * gathers from all of them, so the per-ray set-up and walk control are shared
- * across the chunk; each member's sinogram is bit-identical to ctp_forward's.
+ * across the chunk (where the geometry's slices decouple and one walk already
+ * serves several detector rows, it runs member by member instead); each
+ * member's sinogram is bit-identical to ctp_forward's.
  * With plan.batch_chunk >= 2 the brick adjoint takes member pairs in one
  * launch (its brick halved along y); their volumes then differ from
  * ctp_back's by fixed-point rounding only.  Otherwise, and for the scatter

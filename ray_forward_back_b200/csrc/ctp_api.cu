@@ -700,6 +700,8 @@ ctp_status ctp_geom_query(const ctp_geom *g, ctp_geom_info *info) {
   info->collision_ratio = g->collision_ratio;
   info->batch_chunk = g->batch_chunk;
   info->slice_rows = g->fwd.row_group;
+  info->interleaved_slices = g->fwd.interleaved;
+  info->reserved = 0;
   return CTP_OK;
 }
 
@@ -764,6 +766,15 @@ ctp_status ctp_forward_batch(const ctp_geom *g, const float *vol, float *sino, i
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pending error before ctp_forward_batch");
+  if (g->fwd.row_group > 1) {
+    // decoupled slices: one (x, y) walk already serves several rows of one
+    // volume, faster per member than walks shared across members
+    for (int64_t b = 0; b < n_batch; ++b) {
+      st = ctp_forward(g, vol + (size_t)b * (size_t)g->n_vox, sino + (size_t)b * (size_t)g->n_rays, stream);
+      if (st != CTP_OK) return st;
+    }
+    return CTP_OK;
+  }
   for (int64_t b0 = 0; b0 < n_batch;) {
     // the largest supported chunk that fits the remaining members
     int kb = g->batch_chunk;

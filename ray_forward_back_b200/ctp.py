@@ -64,7 +64,7 @@ class ctp_geom_info(ctypes.Structure):
                 ("adjoint_variant", ctypes.c_int32), ("brick", ctypes.c_int32 * 3),
                 ("view_groups", ctypes.c_int32), ("n_transposed_views", ctypes.c_int32),
                 ("collision_ratio", ctypes.c_double), ("batch_chunk", ctypes.c_int32),
-                ("slice_rows", ctypes.c_int32)]
+                ("slice_rows", ctypes.c_int32), ("interleaved_slices", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 class ctp_solver_options(ctypes.Structure):
@@ -218,7 +218,8 @@ def ctp_geom_query(handle: int) -> dict:
     return {"n_rays": info.n_rays, "n_vox": info.n_vox, "scratch_bytes": info.scratch_bytes,
             "adjoint_variant": info.adjoint_variant, "brick": tuple(info.brick), "view_groups": info.view_groups,
             "n_transposed_views": info.n_transposed_views, "collision_ratio": info.collision_ratio,
-            "batch_chunk": info.batch_chunk, "slice_rows": info.slice_rows}
+            "batch_chunk": info.batch_chunk, "slice_rows": info.slice_rows,
+            "interleaved_slices": info.interleaved_slices}
 
 
 def ctp_forward(handle: int, vol, sino, stream=None) -> None:
