@@ -891,6 +891,15 @@ ctp_status ctp_geometry_gradient(const ctp_geom *g, const float *vol, const floa
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pending error before ctp_geometry_gradient");
   e = cudaMemsetAsync(grad, 0, sizeof(double) * 12 * (size_t)g->n_views, s);
+  if (e == cudaSuccess && g->fwd.interleaved) {
+    // decoupled slices: one (x, y) walk per 4 rows on the interleaved copies
+    e = ctp::launch_interleave(g->fwd, vol, g->d_vol4, g->d_vol4 + g->n_vol4, s);
+    if (e == cudaSuccess)
+      e = ctp::launch_geometry_gradient_rows4(g->fwd, g->d_views, g->d_vol4, g->d_vol4 + g->n_vol4, sino_grad, grad,
+                                              g->wide4, s);
+    if (e != cudaSuccess) return cuda_fail(e, "geometry gradient launch");
+    return CTP_OK;
+  }
   if (e == cudaSuccess && g->fwd.any_transposed) e = ctp::launch_transpose_xy(vol, g->d_volT, g->vol, s);
   if (e == cudaSuccess)
     e = ctp::launch_geometry_gradient(g->fwd, g->d_views, g->d_trig, vol, g->d_volT, sino_grad, grad,

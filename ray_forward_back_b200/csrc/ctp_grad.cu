@@ -274,6 +274,29 @@ __device__ __forceinline__ void cylinder_chain(const ViewRec& V, const double* _
   }
 }
 
+// Block reduction of the 12 per-thread gradient entries (warps by shuffles,
+// then one warp over the 8 warp sums) and one FP64 atomic per entry into
+// grad[v][4][3].  Every block covers one view.
+__device__ __forceinline__ void block_add_view_gradient(const double acc[12], double* __restrict__ grad, int v) {
+  __shared__ double part[kGradThreads / 32][12];
+  const int tid = threadIdx.y * kGradCols + threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+#pragma unroll
+  for (int i = 0; i < 12; ++i) {
+    double a = acc[i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+    if (lane == 0) part[warp][i] = a;
+  }
+  __syncthreads();
+  if (tid < 12) {
+    double a = 0.0;
+#pragma unroll
+    for (int w = 0; w < kGradThreads / 32; ++w) a += part[w][tid];
+    if (a != 0.0) atomicAdd(grad + (size_t)v * 12 + tid, a);
+  }
+}
+
 template <typename Off, bool kCyl>
 __global__ void __launch_bounds__(kGradThreads, CTP_GRAD_MIN_BLOCKS) geometry_gradient_kernel(FwdLaunch P,
                                                                          const ViewRec* __restrict__ views,
@@ -395,24 +418,222 @@ __global__ void __launch_bounds__(kGradThreads, CTP_GRAD_MIN_BLOCKS) geometry_gr
   } else {
     cylinder_chain(V, trig, P.dims, v, valid ? c : 0, rv, gs, gp, acc);
   }
-  // block reduction: warps by shuffles, then one warp over the 8 warp sums
-  __shared__ double part[kGradThreads / 32][12];
-  const int tid = threadIdx.y * kGradCols + threadIdx.x;
-  const int lane = tid & 31, warp = tid >> 5;
-#pragma unroll
-  for (int i = 0; i < 12; ++i) {
-    double a = acc[i];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-    if (lane == 0) part[warp][i] = a;
+  block_add_view_gradient(acc, grad, v);
+}
+
+// ------------------------------------------------ shared (x, y) slice walks --
+//
+// Rays in z-planes whose detector rows step along z (ctp_ray.cuh): one thread
+// walks the (x, y) path of a detector column once for 4 rows, reading the 4
+// rows' voxel values with one 16-byte load from the volume interleaved by 4
+// slices where the rows fall in one slice group (single elements otherwise).
+// The z axis is never crossed, so a slab is one or two segments; every row's
+// crossing sums are the ones its own walk would give, in the same order.
+
+__device__ __forceinline__ float4 f4sub(float4 p, float4 q) { return make_float4(p.x - q.x, p.y - q.y, p.z - q.z, p.w - q.w); }
+__device__ __forceinline__ float4 f4add(float4 p, float4 q) { return make_float4(p.x + q.x, p.y + q.y, p.z + q.z, p.w + q.w); }
+__device__ __forceinline__ float4 f4fma(float4 p, float t, float4 q) {
+  return make_float4(fmaf(p.x, t, q.x), fmaf(p.y, t, q.y), fmaf(p.z, t, q.z), fmaf(p.w, t, q.w));
+}
+__device__ __forceinline__ float f4get(float4 p, int j) { return j == 0 ? p.x : (j == 1 ? p.y : (j == 2 ? p.z : p.w)); }
+
+// crossing_sums for 4 rows at once (component j of every float4 is row j):
+// S0 / Sl of the major axis a (index 0) and of the other crossed axis b
+// (index 1).  load(offset) returns the 4 rows' values of the voxel column at
+// that (x, y) offset.  Returns the values of the voxel the segment ends in.
+#ifndef CTP_GRAD_ROWS_UNROLL
+#define CTP_GRAD_ROWS_UNROLL 2
+#endif
+constexpr int kGradRowsUnroll = CTP_GRAD_ROWS_UNROLL;
+
+template <typename Off, typename Load>
+__device__ __forceinline__ float4 crossing_sums4(bool active, const Walk& W, const int hi[3], Off off, Off s0, Off s1,
+                                                 float4 x0, float4 S0[2], float4 Sl[2], int& ka, int& kb,
+                                                 Load&& load) {
+  constexpr unsigned kFull = 0xffffffffu;
+  int a, b, c;
+  walk_axes(W, a, b, c);
+  ka = a;
+  kb = b;
+  const int Na = active ? pick3(a, W.N[0], W.N[1], W.N[2]) : 0;
+  const int Nb = pick3(b, W.N[0], W.N[1], W.N[2]);
+  const float l0a = pick3(a, W.l0[0], W.l0[1], W.l0[2]), inca = pick3(a, W.inc[0], W.inc[1], W.inc[2]);
+  const float l0b = pick3(b, W.l0[0], W.l0[1], W.l0[2]), incb = pick3(b, W.inc[0], W.inc[1], W.inc[2]);
+  const Off sa = pick3(a, s0, s1, (Off)0), sb = pick3(b, s0, s1, (Off)0);
+  const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+  float4 S0a = zero, S0b = zero, Sla = zero, Slb = zero;
+  float4 xe = x0;
+  const int ia = pick3(a, W.i[0], W.i[1], W.i[2]);
+  const int p = pick3(a, W.step[0], W.step[1], W.step[2]) > 0 ? ia : pick3(a, hi[0], hi[1], hi[2]) - 1 - ia;
+  const int span_plain = __reduce_max_sync(kFull, active ? Na : -1);
+  if (span_plain >= 0) {
+    const int pmin = __reduce_min_sync(kFull, active ? p : 0x7fffffff);
+    int d = active ? p - pmin : 0;
+    int kmax = __reduce_max_sync(kFull, active ? d + Na : -1);
+    if (kmax > 2 * span_plain + 8) {  // alignment would stretch the warp's loop too much
+      d = 0;
+      kmax = span_plain;
+    }
+    if (!active) d = 1 << 30;
+    float fs = -(float)d;
+    const float L = W.L;
+    const float fNb = (float)Nb;
+    float tb = Nb > 0 ? l0b : CUDART_INF_F;
+    float fjb = 1.f, cur = 0.f;
+#pragma unroll kGradRowsUnroll
+    for (int k = 0; k <= kmax; ++k, fs += 1.f) {
+      const int s = k - d;
+      const bool on = (unsigned)s <= (unsigned)Na;
+      const bool ona = (unsigned)s < (unsigned)Na;  // a major plane ends this slab
+      const float tx = ona ? fminf(fmaf(fs, inca, l0a), L) : L;
+      const bool cb = on && tb < tx;
+      const float m1 = fmaxf(fminf(tb, tx), cur);
+      const Off o2 = off + (cb ? sb : (Off)0);
+      float4 x1 = x0;
+      if (cb) x1 = load(o2);
+      float4 x2 = x1;
+      if (ona) x2 = load(o2 + sa);
+      const float4 d1 = f4sub(x0, x1), d2 = f4sub(x1, x2);
+      S0b = f4add(S0b, d1);
+      Slb = f4fma(d1, m1, Slb);
+      S0a = f4add(S0a, d2);
+      Sla = f4fma(d2, tx, Sla);
+      if (on) {
+        xe = x1;
+        x0 = x2;
+        off = o2 + sa;
+        cur = tx;
+      }
+      if (cb) {
+        tb = fjb < fNb ? fmaf(fjb, incb, l0b) : CUDART_INF_F;
+        fjb += 1.f;
+      }
+    }
   }
-  __syncthreads();
-  if (tid < 12) {
-    double a = 0.0;
+  S0[0] = S0a;
+  S0[1] = S0b;
+  Sl[0] = Sla;
+  Sl[1] = Slb;
+  return xe;
+}
+
+#ifndef CTP_GRAD_ROWS_MIN_BLOCKS
+#define CTP_GRAD_ROWS_MIN_BLOCKS 3
+#endif
+
+template <typename Off>
+__global__ void __launch_bounds__(kSliceCols* kSliceWarps, CTP_GRAD_ROWS_MIN_BLOCKS)
+    geometry_gradient_rows4_kernel(FwdLaunch P, const ViewRec* __restrict__ views, const float4* __restrict__ vol4,
+                                   const float4* __restrict__ vol4T, const float* __restrict__ gsino,
+                                   double* __restrict__ grad) {
+  static_assert(kSliceCols * kSliceWarps == kGradThreads, "one gradient block per shared-walk block");
+  int v, c, r0;
+  rows_block_position<4>(P, v, c, r0);
+  const bool cvalid = c < P.dims.n_cols;
+  const ViewRec& V = views[v];
+  const Off nx = P.vol.n[0], ny = P.vol.n[1];
+  const Off plane = nx * ny;
+  [[maybe_unused]] const Off n4 = (Off)((P.vol.n[2] + 3) >> 2) * plane;
+  int ks[4];
+  const unsigned inside = cvalid ? row_slice_index<4>(V, P.vol, r0, c, P.dims.n_rows, ks) : 0u;
+  // rows with a non-zero upstream gradient (their values are read again after
+  // the walk, so they hold no registers through it)
+  auto upstream = [&](int j) -> float {
+    return (inside & (1u << j)) ? __ldg(gsino + ((size_t)v * P.dims.n_rows + r0 + j) * P.dims.n_cols + c) : 0.f;
+  };
+  unsigned rows = inside;
 #pragma unroll
-    for (int w = 0; w < kGradThreads / 32; ++w) a += part[w][tid];
-    if (a != 0.0) atomicAdd(grad + (size_t)v * 12 + tid, a);
+  for (int j = 0; j < 4; ++j)
+    if (!(upstream(j) != 0.f)) rows &= ~(1u << j);
+  // the shared (x, y) ray, lifted into the volume's height: only the x and y
+  // slabs clip it, so t_in, t_out and the entry and exit faces are every row's
+  const int lo[3] = {0, 0, 0};
+  const int hi[3] = {P.vol.n[0], P.vol.n[1], P.vol.n[2]};
+  Walk W = {};
+  bool hit;
+  {
+    Ray R;
+    make_ray(V, P.vol, nullptr, P.dims, v, 0, cvalid ? c : 0, R);
+    R.A[2] = (setup_t)0.5;
+    double t_in = 0.0, t_out = 0.0;
+    int k_in, k_out;
+    hit = rows != 0u && clip_faces(R, hi, t_in, t_out, k_in, k_out);
+    if (hit) entry(R, (setup_t)t_in, (setup_t)t_out, lo, hi, W);
   }
+  const bool yfast = V.layout != 0;
+  const float4* __restrict__ base4 = yfast ? vol4T : vol4;
+  const float* __restrict__ base1 = reinterpret_cast<const float*>(base4);
+  const Off sx = yfast ? ny : (Off)1, sy = yfast ? (Off)1 : nx;
+  const Off off = (Off)W.i[1] * sy + (Off)W.i[0] * sx;
+  const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+  float4 S0[2], Sl[2], first, last;
+  int ka = 0, kb = 1;
+  if (__all_sync(0xffffffffu, one_group(inside, ks) || !hit)) {
+    const Off g0 = (Off)(ks[0] >> 2) * plane;
+    auto load = [&](Off o) -> float4 { return CTP_IN_BOUNDS(g0 + o, n4, 19) ? __ldg(base4 + g0 + o) : zero; };
+    first = hit ? load(off) : zero;
+    last = crossing_sums4<Off>(hit, W, hi, off, W.step[0] * sx, W.step[1] * sy, first, S0, Sl, ka, kb, load);
+  } else {
+    Off e[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) e[j] = ((Off)(ks[j] >> 2) * plane) * 4 + (ks[j] & 3);
+    auto load = [&](Off o) -> float4 {
+      float q[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        q[j] = (inside & (1u << j)) && CTP_IN_BOUNDS(e[j] + 4 * o, 4 * n4, 20) ? __ldg(base1 + e[j] + 4 * o) : 0.f;
+      return make_float4(q[0], q[1], q[2], q[3]);
+    };
+    first = hit ? load(off) : zero;
+    last = crossing_sums4<Off>(hit, W, hi, off, W.step[0] * sx, W.step[1] * sy, first, S0, Sl, ka, kb, load);
+  }
+  // per-row gradients of a parallel ray (as in geometry_gradient_kernel),
+  // weighted by the row's upstream gradient and summed over the 4 rows; the
+  // FP64 set-up is recomputed (bit-identical) rather than kept through the walk
+  const ViewRec* vp = views + v;
+  asm volatile("" : "+l"(vp));
+  Ray R;
+  make_ray(*vp, P.vol, nullptr, P.dims, v, 0, cvalid ? c : 0, R);
+  R.A[2] = (setup_t)0.5;
+  double t_in = 0.0, t_out = 0.0;
+  int k_in = -1, k_out = -1;
+  if (hit) clip_faces(R, hi, t_in, t_out, k_in, k_out);
+  double acc[12];
+#pragma unroll
+  for (int i = 0; i < 12; ++i) acc[i] = 0.0;
+  if (hit) {
+    const double Lseg = (t_out - t_in) * (double)R.len;
+    const double cu = (double)c - 0.5 * (double)(P.dims.n_cols - 1);
+    double q[3];
+#pragma unroll
+    for (int k = 0; k < 3; ++k) q[k] = V.s[k] != 0.0 ? -1.0 / V.s[k] : 0.0;  // V.s is the unit direction
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (!(rows & (1u << j))) continue;
+      const double fj = (double)f4get(first, j), lj = (double)f4get(last, j), gj = (double)upstream(j);
+      double gp[3], gu[3];
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        const double f0 = k == ka ? (double)f4get(S0[0], j) : (k == kb ? (double)f4get(S0[1], j) : 0.0);
+        const double fl = k == ka ? (double)f4get(Sl[0], j) : (k == kb ? (double)f4get(Sl[1], j) : 0.0);
+        const double s0 = f0 - (k == k_in ? fj : 0.0) + (k == k_out ? lj : 0.0);
+        const double sl = fl + (k == k_out ? lj * Lseg : 0.0);
+        const double s1 = fma(t_in, s0, sl / (double)R.len);
+        gp[k] = gj * q[k] * s0;
+        gu[k] = gj * q[k] * s1;
+      }
+      const double ud = V.s[0] * gu[0] + V.s[1] * gu[1] + V.s[2] * gu[2];
+      const double rv = (double)(r0 + j) - 0.5 * (double)(P.dims.n_rows - 1);
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        acc[k] += (gu[k] - V.s[k] * ud) / V.src_norm;
+        acc[3 + k] += gp[k];
+        acc[6 + k] += cu * gp[k];
+        acc[9 + k] += rv * gp[k];
+      }
+    }
+  }
+  block_add_view_gradient(acc, grad, v);
 }
 
 }  // namespace
@@ -433,6 +654,21 @@ cudaError_t launch_geometry_gradient(const FwdLaunch& p, const ViewRec* views, c
     if (cyl) geometry_gradient_kernel<int, true><<<nb, block, 0, stream>>>(p, views, trig, vol, volT, gsino, grad);
     else geometry_gradient_kernel<int, false><<<nb, block, 0, stream>>>(p, views, trig, vol, volT, gsino, grad);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_geometry_gradient_rows4(const FwdLaunch& p, const ViewRec* views, const float4* vol4,
+                                           const float4* vol4T, const float* gsino, double* grad, bool wide_index,
+                                           cudaStream_t stream) {
+  const long long blocks = (long long)rows_bands(p.dims.n_rows, 4) * p.dims.n_views * rows_col_tiles(p.dims.n_cols);
+  if (blocks <= 0) return cudaSuccess;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  const dim3 block(kSliceCols, kSliceWarps);
+  if (wide_index)
+    geometry_gradient_rows4_kernel<long long><<<(unsigned)blocks, block, 0, stream>>>(p, views, vol4, vol4T, gsino,
+                                                                                       grad);
+  else
+    geometry_gradient_rows4_kernel<int><<<(unsigned)blocks, block, 0, stream>>>(p, views, vol4, vol4T, gsino, grad);
   return cudaGetLastError();
 }
 

@@ -89,6 +89,13 @@ cudaError_t launch_forward_rows(const FwdLaunch& p, const ViewRec* views, const 
 // view gathers y-fastest), then walks 4 rows per thread reading 16 bytes per
 // segment; the adjoint adds into the zeroed acc4 / acc4T with 16-byte
 // reductions, then writes vol from them.
+cudaError_t launch_interleave(const FwdLaunch& p, const float* vol, float4* vol4, float4* vol4T,
+                              cudaStream_t stream);
+// Geometry gradients with one (x, y) walk per 4 rows on the interleaved copies
+// (written by launch_interleave first).
+cudaError_t launch_geometry_gradient_rows4(const FwdLaunch& p, const ViewRec* views, const float4* vol4,
+                                           const float4* vol4T, const float* gsino, double* grad, bool wide_index,
+                                           cudaStream_t stream);
 cudaError_t launch_forward_rows4(const FwdLaunch& p, const ViewRec* views, const float* vol, float4* vol4,
                                  float4* vol4T, float* sino, bool wide_index, cudaStream_t stream);
 cudaError_t launch_back_scatter_rows4(const FwdLaunch& p, const ViewRec* views, const float* sino, float* vol,

@@ -72,6 +72,7 @@ constexpr int kWalk3Unroll = CTP_WALK3_UNROLL;
 
 constexpr int kFwdCols = 32;  // threads along detector columns per block
 constexpr int kFwdRows = 8;   // detector rows per block (row band height)
+static_assert(kFwdCols == kSliceCols && kFwdRows == kSliceWarps, "shared slice walks use the forward's block");
 constexpr int kBackThreads = 256;
 #ifndef CTP_BACK_STAGE
 #define CTP_BACK_STAGE 64
@@ -1252,85 +1253,6 @@ __global__ void __launch_bounds__(256) transpose_add_kernel(const float* __restr
 #define CTP_ROWS_MIN_BLOCKS 4
 #endif
 
-// Block shape of the shared-slice kernels: 8 warps of 32 columns x kR rows,
-// kRowsGroups of them stacked along the rows and 8 / kRowsGroups side by side
-// along the columns.  A band (the rows of one block row) is kRowsGroups * kR
-// slices deep; blocks run band by band, every view of a band before the next,
-// so the slices the blocks in flight touch (the adjoint's accumulation
-// working set, in both volume layouts) stay few enough for L2.
-#ifndef CTP_ROWS_GROUPS
-#define CTP_ROWS_GROUPS 8
-#endif
-constexpr int kRowsGroups = CTP_ROWS_GROUPS;
-constexpr int kRowsColTiles = kFwdRows / kRowsGroups;
-static_assert(kRowsGroups * kRowsColTiles == kFwdRows, "row groups divide the block's warps");
-
-__host__ __device__ __forceinline__ int rows_col_tiles(int n_cols) {
-  return (n_cols + kFwdCols * kRowsColTiles - 1) / (kFwdCols * kRowsColTiles);
-}
-__host__ __device__ __forceinline__ int rows_bands(int n_rows, int r) {
-  return (n_rows + kRowsGroups * r - 1) / (kRowsGroups * r);
-}
-
-// View, column and first row of this thread in a shared-slice kernel.
-template <int kR>
-__device__ __forceinline__ void rows_block_position(const FwdLaunch& P, int& v, int& c, int& r0) {
-  const int ctiles = rows_col_tiles(P.dims.n_cols);
-  const int per_band = P.dims.n_views * ctiles;
-  const int band = blockIdx.x / per_band;
-  const int rem = blockIdx.x - band * per_band;
-  v = rem / ctiles;
-  const int ct = rem - v * ctiles;
-  const int w = threadIdx.y;
-  c = (ct * kRowsColTiles + w % kRowsColTiles) * kFwdCols + threadIdx.x;
-  r0 = (band * kRowsGroups + w / kRowsColTiles) * kR;
-}
-
-// Slices of rows r0 .. r0 + kR - 1 of column c: bit j of the result is set
-// where row r0 + j exists and its rays' height falls inside the volume (the z
-// test of the ray's slab clip); ks[j] is then that slice.
-template <int kR>
-__device__ __forceinline__ unsigned row_slice_index(const ViewRec& V, const VolDesc& G, int r0, int c, int n_rows,
-                                                    int ks[kR]) {
-  unsigned mask = 0u;
-#pragma unroll
-  for (int j = 0; j < kR; ++j) {
-    const int r = r0 + j;
-    // the z component of pixel_centre's flat-detector formula and make_ray's
-    // voxel-unit height, in the set-up's precision
-    using T = setup_t;
-    const T pz = fma((T)r, (T)V.dv[2], fma((T)c, (T)V.du[2], (T)V.p00[2]));
-    const T az = (pz - (T)G.origin[2]) * (T)G.inv_spacing[2];
-    const bool in = r < n_rows && az >= (T)0 && az < (T)G.n[2];
-    ks[j] = in ? clampi((int)floor(az), 0, G.n[2] - 1) : 0;
-    mask |= in ? 1u << j : 0u;
-  }
-  return mask;
-}
-
-// The same, as offsets of the slices (zoff[j] = slice * sz).
-template <int kR, typename Off>
-__device__ __forceinline__ unsigned row_slices(const ViewRec& V, const VolDesc& G, int r0, int c, int n_rows, Off sz,
-                                               Off zoff[kR]) {
-  int ks[kR];
-  const unsigned mask = row_slice_index<kR>(V, G, r0, c, n_rows, ks);
-#pragma unroll
-  for (int j = 0; j < kR; ++j) zoff[j] = (mask & (1u << j)) ? (Off)ks[j] * sz : (Off)0;
-  return mask;
-}
-
-// Shared (x, y) set-up of column c: the ray of any row, lifted into the
-// volume's height (its direction has no z component, so only the x and y
-// slabs clip it) and walked as slice 0.
-__device__ __forceinline__ bool slice_ray(const ViewRec& V, const VolDesc& G, const Dims& dm, int v, int c, Ray& R,
-                                          setup_t& t_in, setup_t& t_out) {
-  make_ray(V, G, nullptr, dm, v, 0, c, R);
-  R.A[2] = (setup_t)0.5;
-  const int lo[3] = {0, 0, 0};
-  const int hi[3] = {G.n[0], G.n[1], G.n[2]};
-  return clip(R, lo, hi, t_in, t_out);
-}
-
 template <typename Off, int kR>
 __global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_ROWS_MIN_BLOCKS)
     forward_rows_kernel(FwdLaunch P, const ViewRec* __restrict__ views, const float* __restrict__ vol,
@@ -1459,11 +1381,6 @@ __global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_ROWS_MIN_BLOCKS)
 // values with one 16-byte load, or adds its 4 contributions with one 16-byte
 // reduction; any other row group addresses single elements.  Each row still
 // sees exactly its own segments, in the same order.
-
-// slices 4g .. 4g + 3 of the rows' heights, in order
-__device__ __forceinline__ bool one_group(unsigned rows, const int ks[4]) {
-  return rows == 0xfu && (ks[0] & 3) == 0 && ks[1] == ks[0] + 1 && ks[2] == ks[0] + 2 && ks[3] == ks[0] + 3;
-}
 
 template <typename Off>
 __global__ void __launch_bounds__(kFwdCols* kFwdRows, CTP_ROWS_MIN_BLOCKS)
@@ -1664,13 +1581,18 @@ __global__ void __launch_bounds__(256) deinterleave_kernel(const float4* __restr
 
 // ---------------------------------------------------------------- launchers --
 
-cudaError_t launch_forward_rows4(const FwdLaunch& p, const ViewRec* views, const float* vol, float4* vol4,
-                                 float4* vol4T, float* sino, bool wide_index, cudaStream_t stream) {
+cudaError_t launch_interleave(const FwdLaunch& p, const float* vol, float4* vol4, float4* vol4T,
+                              cudaStream_t stream) {
   const int ng = (p.vol.n[2] + 3) / 4;
   dim3 tgrid((p.vol.n[0] + 31) / 32, (p.vol.n[1] + 31) / 32, ng);
   interleave_kernel<<<tgrid, dim3(32, 8), 0, stream>>>(vol, vol4, p.any_transposed ? vol4T : nullptr, p.vol.n[0],
                                                       p.vol.n[1], p.vol.n[2]);
-  cudaError_t e = cudaGetLastError();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_forward_rows4(const FwdLaunch& p, const ViewRec* views, const float* vol, float4* vol4,
+                                 float4* vol4T, float* sino, bool wide_index, cudaStream_t stream) {
+  cudaError_t e = launch_interleave(p, vol, vol4, vol4T, stream);
   if (e != cudaSuccess) return e;
   const long long blocks = (long long)rows_bands(p.dims.n_rows, 4) * p.dims.n_views * rows_col_tiles(p.dims.n_cols);
   if (blocks <= 0) return cudaSuccess;

@@ -220,4 +220,101 @@ __device__ __forceinline__ void walk_axes(const Walk& W, int& a, int& b, int& c)
   }
 }
 
+
+// ------------------------------------------------ shared (x, y) slice walks --
+//
+// Shared by the projector kernels (ctp_kernels.cu) and the geometry-gradient
+// kernel (ctp_grad.cu): when every ray lies in a plane of constant z (a
+// parallel beam whose direction has no z component) and detector rows step
+// along z only, the rays of one detector column in one view follow the same
+// (x, y) path, each in the slice of its own row (the slices decouple;
+// MBIRJAX "Sharding overview", section "Why cone beam").  Blocks of these
+// kernels are kSliceWarps warps of kSliceCols columns x kR rows.
+constexpr int kSliceCols = 32;
+constexpr int kSliceWarps = 8;
+
+// Block shape of the shared-slice kernels: 8 warps of 32 columns x kR rows,
+// kRowsGroups of them stacked along the rows and 8 / kRowsGroups side by side
+// along the columns.  A band (the rows of one block row) is kRowsGroups * kR
+// slices deep; blocks run band by band, every view of a band before the next,
+// so the slices the blocks in flight touch (the adjoint's accumulation
+// working set, in both volume layouts) stay few enough for L2.
+#ifndef CTP_ROWS_GROUPS
+#define CTP_ROWS_GROUPS 8
+#endif
+constexpr int kRowsGroups = CTP_ROWS_GROUPS;
+constexpr int kRowsColTiles = kSliceWarps / kRowsGroups;
+static_assert(kRowsGroups * kRowsColTiles == kSliceWarps, "row groups divide the block's warps");
+
+__host__ __device__ __forceinline__ int rows_col_tiles(int n_cols) {
+  return (n_cols + kSliceCols * kRowsColTiles - 1) / (kSliceCols * kRowsColTiles);
+}
+__host__ __device__ __forceinline__ int rows_bands(int n_rows, int r) {
+  return (n_rows + kRowsGroups * r - 1) / (kRowsGroups * r);
+}
+
+// View, column and first row of this thread in a shared-slice kernel.
+template <int kR>
+__device__ __forceinline__ void rows_block_position(const FwdLaunch& P, int& v, int& c, int& r0) {
+  const int ctiles = rows_col_tiles(P.dims.n_cols);
+  const int per_band = P.dims.n_views * ctiles;
+  const int band = blockIdx.x / per_band;
+  const int rem = blockIdx.x - band * per_band;
+  v = rem / ctiles;
+  const int ct = rem - v * ctiles;
+  const int w = threadIdx.y;
+  c = (ct * kRowsColTiles + w % kRowsColTiles) * kSliceCols + threadIdx.x;
+  r0 = (band * kRowsGroups + w / kRowsColTiles) * kR;
+}
+
+// Slices of rows r0 .. r0 + kR - 1 of column c: bit j of the result is set
+// where row r0 + j exists and its rays' height falls inside the volume (the z
+// test of the ray's slab clip); ks[j] is then that slice.
+template <int kR>
+__device__ __forceinline__ unsigned row_slice_index(const ViewRec& V, const VolDesc& G, int r0, int c, int n_rows,
+                                                    int ks[kR]) {
+  unsigned mask = 0u;
+#pragma unroll
+  for (int j = 0; j < kR; ++j) {
+    const int r = r0 + j;
+    // the z component of pixel_centre's flat-detector formula and make_ray's
+    // voxel-unit height, in the set-up's precision
+    using T = setup_t;
+    const T pz = fma((T)r, (T)V.dv[2], fma((T)c, (T)V.du[2], (T)V.p00[2]));
+    const T az = (pz - (T)G.origin[2]) * (T)G.inv_spacing[2];
+    const bool in = r < n_rows && az >= (T)0 && az < (T)G.n[2];
+    ks[j] = in ? clampi((int)floor(az), 0, G.n[2] - 1) : 0;
+    mask |= in ? 1u << j : 0u;
+  }
+  return mask;
+}
+
+// The same, as offsets of the slices (zoff[j] = slice * sz).
+template <int kR, typename Off>
+__device__ __forceinline__ unsigned row_slices(const ViewRec& V, const VolDesc& G, int r0, int c, int n_rows, Off sz,
+                                               Off zoff[kR]) {
+  int ks[kR];
+  const unsigned mask = row_slice_index<kR>(V, G, r0, c, n_rows, ks);
+#pragma unroll
+  for (int j = 0; j < kR; ++j) zoff[j] = (mask & (1u << j)) ? (Off)ks[j] * sz : (Off)0;
+  return mask;
+}
+
+// Shared (x, y) set-up of column c: the ray of any row, lifted into the
+// volume's height (its direction has no z component, so only the x and y
+// slabs clip it) and walked as slice 0.
+__device__ __forceinline__ bool slice_ray(const ViewRec& V, const VolDesc& G, const Dims& dm, int v, int c, Ray& R,
+                                          setup_t& t_in, setup_t& t_out) {
+  make_ray(V, G, nullptr, dm, v, 0, c, R);
+  R.A[2] = (setup_t)0.5;
+  const int lo[3] = {0, 0, 0};
+  const int hi[3] = {G.n[0], G.n[1], G.n[2]};
+  return clip(R, lo, hi, t_in, t_out);
+}
+
+// slices 4g .. 4g + 3 of the rows' heights, in order
+__device__ __forceinline__ bool one_group(unsigned rows, const int ks[4]) {
+  return rows == 0xfu && (ks[0] & 3) == 0 && ks[1] == ks[0] + 1 && ks[2] == ks[0] + 2 && ks[3] == ks[0] + 3;
+}
+
 }  // namespace ctp

@@ -154,3 +154,53 @@ def test_zero_inputs_give_zero():
     assert torch.count_nonzero(out).item() == 0
     with pytest.raises(ValueError):
         P.geometry_gradient(vol, gs, out=torch.empty((g.n_views, 4, 3), dtype=torch.float32, device="cuda"))
+
+
+def _slice_geometry(name):
+    """Parallel beams whose rays lie in z-planes and whose rows step along z
+    (decoupled slices), moved off the voxel lattice in x and y only, so they
+    keep that property; rows sit at half-integer heights."""
+    import dataclasses
+    if name == "workload0":
+        g = W.workload(0).geom
+    elif name == "ragged":
+        g = W.make_parallel(70, 45, 33, 9, 36, 77, pitch_u=1.1, pitch_v=1.0, spacing=(1.0, 1.1, 1.0), start=0.05)
+    else:
+        g = W.make_parallel(40, 36, 14, 7, 24, 45, pitch_u=1.0, pitch_v=1.0, start=0.3)
+        g.det_c = g.det_c + np.array([0.0, 0.0, 3.0])  # some rows above the volume
+    return dataclasses.replace(g, det_c=g.det_c + np.array([0.0131, -0.0217, 0.0]))
+
+
+@pytest.mark.parametrize("name", ["ragged", "rows_outside", "workload0"])
+def test_slice_rows_geometry_gradient_equals_one_walk_per_ray(name):
+    """Four rows per (x, y) walk on the interleaved volume: every row's
+    crossing sums are those of its own walk, so only the FP64 order of the
+    per-view sums differs from one walk per ray."""
+    import torch
+    g = _slice_geometry(name)
+    rng = np.random.default_rng(41)
+    vol = torch.from_numpy(rng.random(g.vol_shape).astype(np.float32)).cuda()
+    gs = torch.from_numpy(rng.standard_normal(g.sino_shape).astype(np.float32)).cuda()
+    P1 = projector(g, {"slice_rows": 1})
+    P4 = projector(g, {"slice_rows": 4})
+    assert P4.info()["interleaved_slices"] == 1 and P1.info()["slice_rows"] == 1
+    a = P1.geometry_gradient(vol, gs).cpu().numpy()
+    b = P4.geometry_gradient(vol, gs).cpu().numpy()
+    np.testing.assert_allclose(b, a, rtol=1e-9, atol=1e-12 * np.abs(a).max())
+
+
+def test_slice_rows_geometry_gradient_matches_finite_differences():
+    """The same path against central finite differences of the oracle."""
+    import torch
+    g = _slice_geometry("rows_outside")
+    rng = np.random.default_rng(42)
+    vol = rng.random(g.vol_shape).astype(np.float32)
+    gs = rng.standard_normal(g.sino_shape).astype(np.float32)
+    ref = geometry_gradient_fd(g, vol, gs.astype(np.float64), h=1e-6)
+    P = projector(g, {"slice_rows": 4})
+    assert P.info()["interleaved_slices"] == 1
+    got = P.geometry_gradient(torch.from_numpy(vol).cuda(), torch.from_numpy(gs).cuda()).cpu().numpy()
+    scale = np.abs(ref).max()
+    err = np.abs(got - ref)
+    assert err.max() <= REL * scale, (err.max(), scale)
+    assert np.all(err <= 1e-4 * np.abs(ref) + ELEMENT_FLOOR * scale)
