@@ -62,3 +62,24 @@ def test_code_digest_ignores_comments_and_whitespace_only(tmp_path, monkeypatch)
     a.write_text("int f(int x) {\\n  return x + 2;\\n}\\n")
     assert bench.code_digest(["a.cu"]) != d0
 
+
+
+def test_committed_kernel_counters_match_the_sources():
+    """Every entry of profiles/kernel_counters.json was captured on the kernel
+    code as it stands (the digest of its sources matches), so the bench line's
+    traffic and issue-rate fraction come from the current kernels."""
+    import json
+    import os
+
+    import bench
+    path = os.path.join(bench.ROOT, "profiles", "kernel_counters.json")
+    kernels = json.load(open(path))["kernels"]
+    assert {"forward_rows4_kernel", "back_scatter_rows4_kernel", "forward_kernel", "back_scatter_kernel"} <= set(kernels)
+    for name, per_workload in kernels.items():
+        for wl, k in per_workload.items():
+            assert bench.code_digest(k["sources"]) == k["code_sha256"], (name, wl)
+            assert bench.kernel_counters(name, int(wl)) is not None
+            assert k["updates"] > 0 and k["warp_instructions"] > 0
+    f = bench.issue_fraction("forward_rows4_kernel", 4, 3.0e12, 1965.0, 148)
+    assert 0.5 < f["frac"] < 1.0 and 0.2 < f["warp_instructions_per_update"] < 0.4
+    assert bench.measured_traffic("back_scatter_rows4_kernel", 4, 900) > 1e9
