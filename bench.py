@@ -401,8 +401,12 @@ def time_geometry_gradient(args, P, g, vol, sino_grad, stream, U, world, dev):
     t1.record(stream)
     torch.cuda.synchronize(dev)
     ms = aggregate_over_ranks([t0.elapsed_time(t1) / args.steps], world, dev)[0]
-    return {"ms": ms, "gupdates_s": U / (ms * 1e-3) / 1e9, "kernel": "geometry_gradient_kernel",
-            "launches_per_call": 1 + (1 if P.info()["n_transposed_views"] > 0 else 0)}
+    info = P.info()
+    if info.get("interleaved_slices"):
+        kernel, launches = "geometry_gradient_rows4_kernel", 2      # interleave + gradient
+    else:
+        kernel, launches = "geometry_gradient_kernel", 1 + (1 if info["n_transposed_views"] > 0 else 0)
+    return {"ms": ms, "gupdates_s": U / (ms * 1e-3) / 1e9, "kernel": kernel, "launches_per_call": launches}
 
 
 def run_solver(args, rank, world, local_rank):
@@ -599,7 +603,7 @@ def run_ours(args, rank, world, local_rank):
     if grad is not None:
         gb = algorithmic_bytes(U, g.n_vox, g.n_rays) / (grad["ms"] * 1e-3) / 1e9
         grad.update({"effective_gbs": gb, "frac_of_hbm": gb / peak,
-                     "traffic": measured_traffic("geometry_gradient_kernel", wl_key, g.n_views)})
+                     "traffic": measured_traffic(grad["kernel"], wl_key, g.n_views)})
     B = algorithmic_bytes(U, g.n_vox, g.n_rays)
     fwd_kernel, back_kernel = kernel_names(info)
     dominant = "back" if back_avg >= fwd_avg else "forward"
