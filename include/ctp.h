@@ -260,7 +260,8 @@ ctp_status ctp_count_updates(const ctp_geom *geom, int64_t *host_out, void *stre
  *
  * It takes the acquisition description itself (same fields and guards as
  * ctp_geom_create) plus the caller's device buffers, and computes exactly
- * what ctp_forward computes, with the same kernels.  It calls no cudaMalloc,
+ * what ctp_forward computes (bit for bit), always with one walk per ray: the
+ * shared slice walks of ctp_forward need scratch this call does not have.  It calls no cudaMalloc,
  * cudaFree or other allocating routine, and uses no host heap: its per-view
  * records, the cylindrical column table and the y-fastest copy of the volume
  * live in one fixed device array of CTP_NOALLOC_SCRATCH_BYTES, which every
