@@ -64,6 +64,8 @@ def test_noalloc_matches_ctp_forward_on_two_calls_in_a_row():
         got = _noalloc_forward(g, vol)
         torch.cuda.synchronize()
         _close(got.cpu().numpy(), ref.cpu().numpy())
+        # the same records, layouts and walks: bit for bit
+        assert torch.equal(got, ref)
         check_forward(got.cpu().numpy(), oracle.forward(g, vol_np), oracle_chords(g), min(g.spacing), "noalloc")
         P.close()
 
@@ -86,6 +88,21 @@ def test_noalloc_two_geometries_queued_on_one_stream():
     s.synchronize()
     check_forward(y1.cpu().numpy(), oracle.forward(g1, v1), oracle_chords(g1), min(g1.spacing), "first")
     check_forward(y2.cpu().numpy(), oracle.forward(g2, v2), oracle_chords(g2), min(g2.spacing), "second")
+
+
+def test_noalloc_equals_the_shared_slice_forward():
+    """A parallel beam whose slices decouple: ctp_forward shares one walk
+    between 4 rows on interleaved copies, the no-allocation forward walks
+    every ray on its own; the sinograms are the same bit for bit."""
+    import torch
+    g = W.make_parallel(48, 40, 24, 30, 32, 61, pitch_u=1.0, pitch_v=1.0, start=0.05)
+    P = projector(g, {"slice_rows": 4})
+    assert P.info()["interleaved_slices"] == 1
+    vol = torch.from_numpy(np.random.default_rng(80).random(g.vol_shape).astype(np.float32)).cuda()
+    ref = P.forward(vol)
+    got = _noalloc_forward(g, vol)
+    torch.cuda.synchronize()
+    assert torch.equal(got, ref)
 
 
 @pytest.mark.parametrize("n_cols", [1500, 33000])
