@@ -122,7 +122,8 @@ def kernel_names(info):
     inter = "4" if info.get("interleaved_slices") else ""
     fwd = f"forward_rows{inter}_kernel" if rows else "forward_kernel"
     back = {1: "back_brick_kernel", 2: "back_sort_kernel",
-            3: f"back_scatter_rows{inter}_kernel" if rows else "back_scatter_kernel"}[info["adjoint_variant"]]
+            3: f"back_scatter_rows{inter}_kernel" if rows else "back_scatter_kernel",
+            4: "back_gather_kernel"}[info["adjoint_variant"]]
     return fwd, back
 
 
@@ -130,6 +131,9 @@ def launches_per_step(info):
     """Kernels of the library launched by one forward + one back projection
     (memsets are not kernels of the library)."""
     t = 1 if info["n_transposed_views"] > 0 else 0
+    if info["adjoint_variant"] == 4:                       # slice sums + gather
+        fwd = 2 if info.get("interleaved_slices") else 1 + t
+        return fwd + 2
     if info.get("interleaved_slices") and info["adjoint_variant"] == 3:
         return 4                      # interleave + forward, adjoint + deinterleave
     if info.get("interleaved_slices"):
@@ -278,7 +282,7 @@ def select_workload(args):
     return wl
 
 
-VARIANTS = {"auto": 0, "brick": 1, "sort": 2, "scatter": 3}
+VARIANTS = {"auto": 0, "brick": 1, "sort": 2, "scatter": 3, "gather": 4}
 
 
 def plan_of(args):
@@ -645,7 +649,7 @@ def run_ours(args, rank, world, local_rank):
                  "effective_gbs": B / (back_avg * 1e-3) / 1e9,
                  "frac_of_hbm": B / (back_avg * 1e-3) / 1e9 / peak,
                  "issue": issue_back, "traffic": measured_traffic(back_kernel, wl_key, g.n_views),
-                 "variant": {1: "brick", 2: "sort", 3: "scatter"}[info["adjoint_variant"]],
+                 "variant": {1: "brick", 2: "sort", 3: "scatter", 4: "gather"}[info["adjoint_variant"]],
                  "collision_ratio": info["collision_ratio"], "slice_rows": info.get("slice_rows", 1)},
         "roofline": {"kernel": dom_kernel,
                      "bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs",

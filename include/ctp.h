@@ -77,13 +77,29 @@ typedef enum {
 enum { CTP_BEAM_PARALLEL = 0, CTP_BEAM_CONE = 1 };
 enum { CTP_DET_FLAT = 0, CTP_DET_CYLINDRICAL = 1 };
 
-/* Adjoint variants.  AUTO picks by the collision ratio measured at create:
- * SCATTER (one global float add per ray-voxel segment, off the forward's
- * walk) below 13.5 contributions per distinct voxel of a warp batch, SORT
- * (warp sort and segmented sum, one add per distinct voxel) above.  BRICK
- * (shared-memory fixed point per voxel block) is never chosen automatically;
- * it is the bitwise-reproducible variant. */
-enum { CTP_ADJOINT_AUTO = 0, CTP_ADJOINT_BRICK = 1, CTP_ADJOINT_SORT = 2, CTP_ADJOINT_SCATTER = 3 };
+/* Adjoint variants.  AUTO picks GATHER where it applies (parallel beams
+ * whose rays lie in z-planes with detector rows stepping along z: one warp
+ * per (x, y) cell sums chord x slice-summed sinogram over the views and the
+ * crossing columns, writing every voxel once; bitwise reproducible; MBIRJAX
+ * "Projector kernels", paragraph "Forward scatters, back gathers"), else by
+ * the collision ratio measured at create: SCATTER (one global float add per
+ * ray-voxel segment, off the forward's walk) below 13.5 contributions per
+ * distinct voxel of a warp batch, SORT (warp sort and segmented sum, one add
+ * per distinct voxel) above.  BRICK (shared-memory fixed point per voxel
+ * block) is never chosen automatically; it is bitwise reproducible on every
+ * geometry.  Forcing GATHER where it does not apply fails with
+ * CTP_ERR_UNSUPPORTED (ctp_last_error_detail() names the reason: another
+ * beam or detector, rays leaving the z-planes, rays running along the
+ * detector's columns, columns more than 64 per voxel, or a ray of a view on an
+ * axis running within 1e-6 voxels of a grid line, where the slab walk's
+ * rounding decides the cell). */
+enum {
+  CTP_ADJOINT_AUTO = 0,
+  CTP_ADJOINT_BRICK = 1,
+  CTP_ADJOINT_SORT = 2,
+  CTP_ADJOINT_SCATTER = 3,
+  CTP_ADJOINT_GATHER = 4
+};
 
 /* Optional plan overrides (all zero = library defaults). */
 typedef struct {
@@ -123,7 +139,7 @@ typedef struct {
 typedef struct {
   int64_t n_rays, n_vox;
   int64_t scratch_bytes;        /* device memory the handle owns */
-  int32_t adjoint_variant;      /* variant ctp_back will run (BRICK, SORT or SCATTER) */
+  int32_t adjoint_variant;      /* variant ctp_back will run (BRICK, SORT, SCATTER or GATHER) */
   int32_t brick[3];
   int32_t view_groups;
   int32_t n_transposed_views;   /* views whose forward gathers from the y-fastest copy */
@@ -176,9 +192,13 @@ ctp_status ctp_forward(const ctp_geom *geom, const float *vol, float *sino, void
  * vol:  device pointer, float32 [nz][ny][nx], overwritten.
  * Same pointer, stream and synchronisation rules as ctp_forward.  A
  * non-finite sinogram value (NaN or infinity) is not dropped: with the
- * scatter and sort adjoints it reaches every voxel its ray crosses (NaN, or
- * an infinity); with the brick adjoint every voxel of each volume block whose
- * detector footprint holds it is written as NaN.
+ * scatter, sort and gather adjoints it reaches every voxel its ray crosses
+ * (NaN, or an infinity); with the brick adjoint every voxel of each volume
+ * block whose detector footprint holds it is written as NaN.
+ * The gather adjoint first sums the sinogram over the rows of each column
+ * that fall in one slice, into scratch the handle owns (n_views x n_cols x
+ * nz rounded up to 4 floats), so calls on one handle must not overlap in
+ * time (stream-order them).
  */
 ctp_status ctp_back(const ctp_geom *geom, const float *sino, float *vol, void *stream);
 
@@ -198,8 +218,8 @@ ctp_status ctp_back(const ctp_geom *geom, const float *sino, float *vol, void *s
  * member's sinogram is bit-identical to ctp_forward's.
  * With plan.batch_chunk >= 2 the brick adjoint takes member pairs in one
  * launch (its brick halved along y); their volumes then differ from
- * ctp_back's by fixed-point rounding only.  Otherwise, and for the scatter
- * and sort adjoints, it runs member by member.  n_batch < 0, or a
+ * ctp_back's by fixed-point rounding only.  Otherwise, and for the scatter,
+ * sort and gather adjoints, it runs member by member.  n_batch < 0, or a
  * batch whose element count exceeds 2^62, gives CTP_ERR_INVALID_ARGUMENT.
  * Same pointer, stream and synchronisation rules as ctp_forward / ctp_back.
  */

@@ -14,8 +14,9 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libctp.so")
-SOURCES = ["ctp_api.cu", "ctp_kernels.cu", "ctp_grad.cu", "ctp_noalloc.cu", "ctp_solvers.cu"]
-HEADERS = [os.path.join(CSRC, "ctp_internal.h"), os.path.join(CSRC, "ctp_ray.cuh"), os.path.join(INCLUDE, "ctp.h")]
+SOURCES = ["ctp_api.cu", "ctp_kernels.cu", "ctp_grad.cu", "ctp_gather.cu", "ctp_noalloc.cu", "ctp_solvers.cu"]
+HEADERS = [os.path.join(CSRC, "ctp_internal.h"), os.path.join(CSRC, "ctp_ray.cuh"), os.path.join(CSRC, "ctp_gather.h"),
+           os.path.join(INCLUDE, "ctp.h")]
 
 
 def nvcc_path() -> str:

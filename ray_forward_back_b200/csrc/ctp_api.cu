@@ -9,6 +9,7 @@
 #include <new>
 #include <vector>
 
+#include "ctp_gather.h"
 #include "ctp_internal.h"
 
 using ctp::BackLaunch;
@@ -38,6 +39,9 @@ struct ctp_geom {
   int64_t n_vol4 = 0;         // float4 elements of one interleaved copy
   bool wide4 = false;         // 64-bit offsets for the interleaved copies
   unsigned long long *d_counter = nullptr;
+  ctp::GatherView *d_gview = nullptr;  // gather adjoint: per-view records
+  float *d_ysum = nullptr;             // gather adjoint: slice sums of the sinogram [view][column][nz4]
+  ctp::GatherLaunch gather{};
   int64_t scratch_bytes = 0;
   int batch_chunk = 1;  // volumes per fused batched forward launch (y-fastest copies held)
 };
@@ -160,7 +164,7 @@ ctp_status validate_desc(const ctp_geom_desc *d) {
     return fail(CTP_ERR_INVALID_ARGUMENT, "a per-view vector array is NULL");
   if (d->plan) {
     const ctp_plan *p = d->plan;
-    if (p->adjoint_variant < CTP_ADJOINT_AUTO || p->adjoint_variant > CTP_ADJOINT_SCATTER)
+    if (p->adjoint_variant < CTP_ADJOINT_AUTO || p->adjoint_variant > CTP_ADJOINT_GATHER)
       return fail(CTP_ERR_INVALID_ARGUMENT, "plan.adjoint_variant %d", p->adjoint_variant);
     for (int k = 0; k < 3; ++k)
       if (p->brick[k] < 0 || p->brick[k] > 1024) return fail(CTP_ERR_INVALID_ARGUMENT, "plan.brick[%d]", k);
@@ -421,6 +425,8 @@ void free_geom(ctp_geom *g) {
   cudaFree(g->d_volT);
   cudaFree(g->d_vol4);
   cudaFree(g->d_counter);
+  cudaFree(g->d_gview);
+  cudaFree(g->d_ysum);
   delete g;
 }
 
@@ -481,6 +487,7 @@ unsigned long long debug_collect() {
   std::lock_guard<std::mutex> lock(g_debug_mu);
   if (!g_debug_pending) g_debug_pending = ctp::debug_take_word_kernels();
   if (!g_debug_pending) g_debug_pending = ctp::debug_take_word_grad();
+  if (!g_debug_pending) g_debug_pending = ctp::debug_take_word_gather();
   return g_debug_pending;
 }
 #endif
@@ -632,6 +639,18 @@ ctp_status ctp_geom_create(const ctp_geom_desc *desc, ctp_geom **out) {
     g->n_vol4 = (g->nz + 3) / 4 * g->nx * g->ny;
     g->wide4 = g->wide_index || 4 * g->n_vol4 >= (int64_t)0x7fffffff;
   }
+  // Gather adjoint: decoupled slices whose views all suit it, unless the
+  // plan names another variant.
+  const int forced = plan ? plan->adjoint_variant : CTP_ADJOINT_AUTO;
+  std::vector<ctp::GatherView> gviews;
+  std::string gather_why = "the rays do not lie in z-planes with rows stepping along z";
+  const bool gather_ok = slices && ctp::build_gather_views(views, vd, g->n_cols, gviews, gather_why);
+  const bool use_gather = gather_ok && (forced == CTP_ADJOINT_AUTO || forced == CTP_ADJOINT_GATHER);
+  if (forced == CTP_ADJOINT_GATHER && !gather_ok) {
+    delete g;
+    return fail(CTP_ERR_UNSUPPORTED, "gather adjoint: %s", gather_why.c_str());
+  }
+  if (use_gather) g->gather = ctp::plan_gather(vd, dm);
   if (ctp::back_brick_smem_bytes(g->back.brick) > 200 * 1024) {
     delete g;
     return fail(CTP_ERR_INVALID_ARGUMENT, "adjoint brick needs more than 200 KB of shared memory");
@@ -656,11 +675,18 @@ ctp_status ctp_geom_create(const ctp_geom_desc *desc, ctp_geom **out) {
     st = alloc((void **)&g->d_vol4, sizeof(float4) * (size_t)g->n_vol4 * (f.any_transposed ? 2 : 1),
                "volumes interleaved by 4 slices");
   if (st == CTP_OK) st = alloc((void **)&g->d_counter, sizeof(unsigned long long), "counter");
+  if (st == CTP_OK && use_gather)
+    st = alloc((void **)&g->d_gview, sizeof(ctp::GatherView) * gviews.size(), "gather view records");
+  if (st == CTP_OK && use_gather)
+    st = alloc((void **)&g->d_ysum, sizeof(float) * (size_t)g->n_views * (size_t)g->n_cols * (size_t)g->gather.nz4,
+               "slice sums of the sinogram");
   cudaError_t e = cudaSuccess;
   if (st == CTP_OK) {
     e = cudaMemcpy(g->d_views, views.data(), vbytes, cudaMemcpyHostToDevice);
     if (e == cudaSuccess && !trig.empty())
       e = cudaMemcpy(g->d_trig, trig.data(), sizeof(double) * trig.size(), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && use_gather)
+      e = cudaMemcpy(g->d_gview, gviews.data(), sizeof(ctp::GatherView) * gviews.size(), cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = ctp::prepare_back_brick(ctp::back_brick_smem_bytes(g->back.brick));
     if (e == cudaSuccess && g->batch_chunk >= 2)
       e = ctp::prepare_back_brick(ctp::back_brick_smem_bytes(g->back2.brick, 2), 2);
@@ -671,9 +697,11 @@ ctp_status ctp_geom_create(const ctp_geom_desc *desc, ctp_geom **out) {
     free_geom(g);
     return st;
   }
-  // adjoint variant: forced by the plan, else by the measured collision ratio
-  const int forced = plan ? plan->adjoint_variant : CTP_ADJOINT_AUTO;
-  if (forced == CTP_ADJOINT_BRICK || forced == CTP_ADJOINT_SORT || forced == CTP_ADJOINT_SCATTER)
+  // adjoint variant: forced by the plan, else the gather where it applies,
+  // else by the measured collision ratio
+  if (use_gather)
+    g->adjoint_variant = CTP_ADJOINT_GATHER;
+  else if (forced == CTP_ADJOINT_BRICK || forced == CTP_ADJOINT_SORT || forced == CTP_ADJOINT_SCATTER)
     g->adjoint_variant = forced;
   else
     g->adjoint_variant = g->collision_ratio >= kSortMinCollisionRatio ? CTP_ADJOINT_SORT : CTP_ADJOINT_SCATTER;
@@ -847,6 +875,12 @@ ctp_status ctp_back_power(const ctp_geom *g, const float *sino, float *vol, int 
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pending error before ctp_back");
+  if (g->adjoint_variant == CTP_ADJOINT_GATHER) {
+    // slice sums, then one warp per (x, y) cell writes every slice of it
+    e = ctp::launch_back_gather(g->fwd, g->gather, g->d_views, g->d_gview, sino, g->d_ysum, vol, power, s);
+    if (e != cudaSuccess) return cuda_fail(e, "adjoint launch");
+    return CTP_OK;
+  }
   const bool sorted = g->adjoint_variant == CTP_ADJOINT_SORT;
   const bool scatter = g->adjoint_variant == CTP_ADJOINT_SCATTER;
   if (scatter && g->fwd.interleaved) {

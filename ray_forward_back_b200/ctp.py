@@ -34,6 +34,8 @@ CTP_DET_CYLINDRICAL = 1
 CTP_ADJOINT_AUTO = 0
 CTP_ADJOINT_BRICK = 1
 CTP_ADJOINT_SORT = 2
+CTP_ADJOINT_SCATTER = 3
+CTP_ADJOINT_GATHER = 4
 
 EXPORTED = ["ctp_geom_create", "ctp_geom_destroy", "ctp_geom_query", "ctp_forward", "ctp_back",
             "ctp_forward_batch", "ctp_back_batch", "ctp_back_power", "ctp_geometry_gradient", "ctp_count_updates", "ctp_forward_noalloc", "ctp_solve", "ctp_solver_workspace_bytes",

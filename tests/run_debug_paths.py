@@ -3,7 +3,8 @@
 record: prints ``debug_word <value>`` (0 when every index stayed in bounds).
 
 Run as ``python -m tests.run_debug_paths``.  Covered: forward, every adjoint
-variant with coefficient powers 1 and 2, batched forward and fused batched
+variant (the gather adjoint on the geometries it applies to) with
+coefficient powers 1 and 2, batched forward and fused batched
 adjoint, shared slice walks, geometry gradients, the update count and the
 no-allocation forward, on the ragged geometries of the parity tests; then
 view subsets of workloads 2, 3 and 4 at their full volume and detector size.
@@ -22,7 +23,8 @@ def exercise(g, torch, ctp, dev, small=True):
     rng = np.random.default_rng(9)
     vol = torch.from_numpy(rng.random(g.vol_shape).astype(np.float32)).to(dev)
     sino = torch.from_numpy(rng.random(g.sino_shape).astype(np.float32)).to(dev)
-    plans = [{"adjoint_variant": v} for v in (1, 2, 3)]
+    # 0: the automatic choice, the gather adjoint where it applies
+    plans = [{"adjoint_variant": v} for v in (0, 1, 2, 3)]
     if g.beam == 0:
         plans += [{"adjoint_variant": 3, "slice_rows": r} for r in (2, 4)]
     for plan in plans:

@@ -52,11 +52,12 @@ def test_batched_members_meet_the_oracle():
         check_forward(y[b], oracle.forward(g, vols[b]), chord, min(g.spacing), f"member {b}")
 
 
-@pytest.mark.parametrize("variant", [1, 3])
-@pytest.mark.parametrize("name", ["cone_flat", "parallel_both_layouts"])
+@pytest.mark.parametrize("name,variant", [("cone_flat", 1), ("cone_flat", 3), ("parallel_both_layouts", 1),
+                                          ("parallel_both_layouts", 3), ("parallel_both_layouts", 4)])
 def test_batched_back_equals_single_calls(name, variant):
     """Member by member, the batched adjoint is the single call: bit for bit
-    with the brick adjoint (integer sums, fixed order), to FP32 accumulation
+    with the brick adjoint (integer sums, fixed order) and the gather adjoint
+    (each voxel summed by one thread in a fixed order), to FP32 accumulation
     order with the scatter adjoint (float adds in whatever order the atomics
     land)."""
     import torch
@@ -69,7 +70,7 @@ def test_batched_back_equals_single_calls(name, variant):
     for a in range(2):
         for b in range(2):
             single = P.back(sino[a, b].contiguous())
-            if variant == 1:
+            if variant in (1, 4):
                 assert torch.equal(x[a, b], single)
             else:
                 torch.testing.assert_close(x[a, b], single, rtol=1e-5, atol=1e-6 * float(single.abs().max()))

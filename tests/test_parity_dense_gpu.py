@@ -80,7 +80,10 @@ def test_dense_full_size_parity(index):
     sino = np.random.default_rng(wl.seed + 7).random(g.sino_shape, dtype=np.float32)
     x_ref = oracle_pool.back(g, sino)
     failures = []
-    for variant, name in VARIANTS.items():
+    variants = dict(VARIANTS)
+    if full["adjoint_variant"] == 4:
+        variants[4] = "gather"
+    for variant, name in variants.items():
         P = projector(g, dict(plan, adjoint_variant=variant))
         assert P.info()["adjoint_variant"] == variant
         x = gpu_back(P, sino)

@@ -319,9 +319,11 @@ def high_magnification_cone():
 def test_collision_ratio_measured_and_dispatch_consistent():
     """The ratio measured at create is >= 1 and grows with ray density; the
     automatic choice is the sort adjoint for dense rays (ratio >= 13.5) and
-    the scatter adjoint otherwise, and both results meet the tolerances."""
+    the scatter adjoint otherwise (on geometries without decoupled slices,
+    where the gather adjoint does not apply), and both results meet the
+    tolerances."""
     dense = high_magnification_cone()
-    sparse = ragged_geometries()["parallel_ragged"]
+    sparse = ragged_geometries()["cone_ragged"]
     Pd, Ps = projector(dense), projector(sparse)
     rd, rs = Pd.info()["collision_ratio"], Ps.info()["collision_ratio"]
     assert rs >= 1.0 and rd >= 1.0
