@@ -95,11 +95,14 @@ def kernel_counters(kernel, workload_index):
 
 def measured_traffic(kernel, workload_index, n_views):
     """DRAM bytes of one full launch: the small capture's bytes scaled by the
-    view count (each view's rays are an equal share of the work)."""
+    view count (each view's rays are an equal share of the work), except a
+    part that does not depend on the views (fixed_dram_bytes: the gather
+    adjoint's output volume, written once)."""
     k = kernel_counters(kernel, workload_index)
     if k is None:
         return None
-    return int(round(k["dram_bytes"] * n_views / k["views"]))
+    fixed = k.get("fixed_dram_bytes", 0)
+    return int(round(fixed + (k["dram_bytes"] - fixed) * n_views / k["views"]))
 
 
 def issue_fraction(kernel, workload_index, updates_per_s, sm_mhz, n_sm):

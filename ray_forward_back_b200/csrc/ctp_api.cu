@@ -639,18 +639,21 @@ ctp_status ctp_geom_create(const ctp_geom_desc *desc, ctp_geom **out) {
     g->n_vol4 = (g->nz + 3) / 4 * g->nx * g->ny;
     g->wide4 = g->wide_index || 4 * g->n_vol4 >= (int64_t)0x7fffffff;
   }
-  // Gather adjoint: decoupled slices whose views all suit it, unless the
-  // plan names another variant.
+  // Gather adjoint: decoupled slices whose views all suit it, when the plan
+  // names it, or automatically once its grid fills the device (four blocks
+  // per SM; below that the scatter adjoint measured faster).
   const int forced = plan ? plan->adjoint_variant : CTP_ADJOINT_AUTO;
   std::vector<ctp::GatherView> gviews;
   std::string gather_why = "the rays do not lie in z-planes with rows stepping along z";
   const bool gather_ok = slices && ctp::build_gather_views(views, vd, g->n_cols, gviews, gather_why);
-  const bool use_gather = gather_ok && (forced == CTP_ADJOINT_AUTO || forced == CTP_ADJOINT_GATHER);
   if (forced == CTP_ADJOINT_GATHER && !gather_ok) {
     delete g;
     return fail(CTP_ERR_UNSUPPORTED, "gather adjoint: %s", gather_why.c_str());
   }
-  if (use_gather) g->gather = ctp::plan_gather(vd, dm);
+  g->gather = ctp::plan_gather(vd, dm);
+  const int64_t gather_blocks = (int64_t)g->gather.tiles_x * g->gather.tiles_y * g->gather.n_zchunks;
+  const bool use_gather = gather_ok && (forced == CTP_ADJOINT_GATHER ||
+                                        (forced == CTP_ADJOINT_AUTO && gather_blocks >= 4 * (int64_t)sm_count));
   if (ctp::back_brick_smem_bytes(g->back.brick) > 200 * 1024) {
     delete g;
     return fail(CTP_ERR_INVALID_ARGUMENT, "adjoint brick needs more than 200 KB of shared memory");

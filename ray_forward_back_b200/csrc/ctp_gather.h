@@ -22,7 +22,7 @@ namespace ctp {
 // direction lies on an axis (axis 1: along x, axis 2: along y, including
 // directions whose drift across the volume is below 1e-9 voxels) place the
 // ray by the floor of its minor-axis position, as the slab walk does.
-struct GatherView {
+struct __align__(16) GatherView {
   double g0, gx, gy;  // column coordinate of a cell centre
   double kap;         // offset of the cell centre per column
   double halfw;       // candidate columns: |gamma - c| <= halfw

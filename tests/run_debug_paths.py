@@ -23,12 +23,18 @@ def exercise(g, torch, ctp, dev, small=True):
     rng = np.random.default_rng(9)
     vol = torch.from_numpy(rng.random(g.vol_shape).astype(np.float32)).to(dev)
     sino = torch.from_numpy(rng.random(g.sino_shape).astype(np.float32)).to(dev)
-    # 0: the automatic choice, the gather adjoint where it applies
-    plans = [{"adjoint_variant": v} for v in (0, 1, 2, 3)]
+    plans = [{"adjoint_variant": v} for v in (1, 2, 3, 4)]
     if g.beam == 0:
         plans += [{"adjoint_variant": 3, "slice_rows": r} for r in (2, 4)]
     for plan in plans:
-        with ctp.Projector(g, device=dev.index, plan=plan) as P:
+        try:
+            P = ctp.Projector(g, device=dev.index, plan=plan)
+        except ctp.CtpError as e:
+            # the gather adjoint (4) applies to decoupled parallel slices only
+            if plan["adjoint_variant"] == 4 and e.status == ctp.CTP_ERR_UNSUPPORTED:
+                continue
+            raise
+        with P:
             P.forward(vol)
             P.back(sino)
             P.back_power(sino, 2)

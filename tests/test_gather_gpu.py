@@ -2,8 +2,10 @@
 
 Parallel beams whose rays lie in z-planes with detector rows stepping along
 z: the adjoint is computed voxel by voxel from closed-form chords and the
-sinogram's slice sums.  Checked: the adjoint tolerances (relative L2, per
-voxel), squared coefficients, the adjoint identity, bitwise reproducibility,
+sinogram's slice sums (forced through the plan on these small geometries,
+where the automatic choice is the scatter).  Checked: the adjoint
+tolerances (relative L2, per voxel), squared coefficients, the adjoint
+identity, bitwise reproducibility,
 non-finite propagation, batches, slice counts that take every lane layout
 (1, 2 and 4 float4 groups per lane, several slice chunks), the automatic
 choice and the geometries it refuses."""
@@ -43,7 +45,7 @@ def _tolerances(be, label):
 @pytest.mark.parametrize("name", sorted(gather_geometries()))
 def test_gather_matches_oracle(name):
     g = gather_geometries()[name]
-    P = projector(g)
+    P = projector(g, {"adjoint_variant": GATHER})
     assert P.info()["adjoint_variant"] == GATHER
     rng = np.random.default_rng(21)
     sino = rng.random(g.sino_shape).astype(np.float32)
@@ -56,18 +58,22 @@ def test_gather_matches_oracle(name):
     assert adjoint_mismatch(P, g) <= 1e-5
 
 
-def test_gather_workload0_is_the_default_and_meets_the_oracle():
+def test_gather_workload0_meets_the_oracle_and_the_automatic_choice():
+    """Workload 0 through the gather; the automatic choice takes the gather
+    once its grid holds four blocks per SM (workload 4), the scatter below
+    that (workload 0, 256 blocks)."""
     wl = W.workload(0)
-    P = projector(wl.geom)
-    assert P.info()["adjoint_variant"] == GATHER
+    P = projector(wl.geom, {"adjoint_variant": GATHER})
     sino = wl.sinogram()
     _tolerances(back_errors(gpu_back(P, sino), oracle.back(wl.geom, sino)), wl.name)
+    assert projector(wl.geom).info()["adjoint_variant"] == 3
+    assert projector(W.workload(4).geom).info()["adjoint_variant"] == GATHER
 
 
 def test_gather_is_bitwise_reproducible_and_batches_member_by_member():
     import torch
     g = gather_geometries()["parallel_ragged"]
-    P = projector(g)
+    P = projector(g, {"adjoint_variant": GATHER})
     torch.manual_seed(8)
     sino = torch.rand((3,) + tuple(g.sino_shape), device="cuda")
     single = [P.back(sino[b].contiguous()) for b in range(3)]
@@ -80,7 +86,7 @@ def test_gather_is_bitwise_reproducible_and_batches_member_by_member():
 def test_gather_propagates_a_non_finite_ray_to_the_voxels_it_crosses():
     import torch
     g = gather_geometries()["parallel_ragged"]
-    P = projector(g)
+    P = projector(g, {"adjoint_variant": GATHER})
     v, r, c = 4, 17, 40
     sino = np.random.default_rng(2).random(g.sino_shape).astype(np.float32)
     sino[v, r, c] = np.nan
