@@ -125,9 +125,42 @@ __global__ void __launch_bounds__(kGatherThreads, 2)
   const double xd = (double)x, yd = (double)y;
   const int nc = P.n_cols;
   [[maybe_unused]] const size_t n_ysum4 = (size_t)P.n_views * nc * g4;
-  for (int v = 0; v < P.n_views; ++v) {
+  const float4* __restrict__ colv = reinterpret_cast<const float4*>(ysum);  // view v's first column
+  auto add = [&](float w, const float4* __restrict__ src) {
+#pragma unroll
+    for (int j = 0; j < kJ; ++j) {
+      if (ok[j] && CTP_IN_BOUNDS((src - reinterpret_cast<const float4*>(ysum)) + q[j], n_ysum4, 23)) {
+        const float4 t = __ldg(src + q[j]);
+        acc[j].x = fmaf(w, t.x, acc[j].x);
+        acc[j].y = fmaf(w, t.y, acc[j].y);
+        acc[j].z = fmaf(w, t.z, acc[j].z);
+        acc[j].w = fmaf(w, t.w, acc[j].w);
+      }
+    }
+  };
+  for (int v = 0; v < P.n_views; ++v, colv += (size_t)nc * g4) {
     const GatherView& G = gv[v];
     const double gam = fma(yd, G.gy, fma(xd, G.gx, G.g0));
+    if (G.two) {
+      // at most two columns cross the cell: the first candidate and the next
+      const double c0 = fmax(0.0, ceil(gam - G.halfw));
+      const double cmax = fmin((double)(nc - 1), floor(gam + G.halfw));
+      const double d0 = G.wh - fabs((gam - c0) * G.kap);
+      const double d1 = G.wh - fabs((gam - (c0 + 1.0)) * G.kap);
+      const bool h0 = c0 <= cmax && d0 > 0.0;
+      const bool h1 = c0 + 1.0 <= cmax && d1 > 0.0;
+      if (!(h0 || h1)) continue;
+      const float4* __restrict__ src0 = colv + (size_t)(int)c0 * g4;
+      if (h0) {
+        const float len = fminf(G.lmax, (float)d0 * G.inv_slope);
+        add(kPower == 2 ? len * len : len, src0);
+      }
+      if (h1) {
+        const float len = fminf(G.lmax, (float)d1 * G.inv_slope);
+        add(kPower == 2 ? len * len : len, src0 + g4);
+      }
+      continue;
+    }
     const int clo = (int)fmax(0.0, ceil(gam - G.halfw));
     const int chi = (int)fmin((double)(nc - 1), floor(gam + G.halfw));
     for (int c = clo; c <= chi; ++c) {
@@ -142,19 +175,7 @@ __global__ void __launch_bounds__(kGatherThreads, 2)
         if (floor(am) != (G.axis == 1 ? yd : xd)) continue;
         len = G.lmax;
       }
-      const float w = kPower == 2 ? len * len : len;
-      const size_t col4 = ((size_t)v * nc + c) * g4;
-      const float4* __restrict__ src = reinterpret_cast<const float4*>(ysum) + col4;
-#pragma unroll
-      for (int j = 0; j < kJ; ++j) {
-        if (ok[j] && CTP_IN_BOUNDS(col4 + q[j], n_ysum4, 23)) {
-          const float4 t = __ldg(src + q[j]);
-          acc[j].x = fmaf(w, t.x, acc[j].x);
-          acc[j].y = fmaf(w, t.y, acc[j].y);
-          acc[j].z = fmaf(w, t.z, acc[j].z);
-          acc[j].w = fmaf(w, t.w, acc[j].w);
-        }
-      }
+      add(kPower == 2 ? len * len : len, colv + (size_t)c * g4);
     }
   }
   const size_t plane = (size_t)P.nx * P.ny;
@@ -241,6 +262,8 @@ bool build_gather_views(const std::vector<ViewRec>& views, const VolDesc& vd, in
     G.lmax = (float)std::fmin(adx > 0.0 ? 1.0 / adx : inf, ady > 0.0 ? 1.0 / ady : inf);
     G.inv_slope = axis == 0 ? (float)(1.0 / (adx * ady)) : 0.f;
     G.axis = axis;
+    // at most two integers lie within halfw of any column coordinate
+    G.two = axis == 0 && G.halfw < 1.0 ? 1 : 0;
     const int k = axis == 2 ? 0 : 1;
     G.p00m = V.p00[k];
     G.dum = V.du[k];

@@ -30,7 +30,7 @@ struct __align__(16) GatherView {
   float lmax;         // chord along the full cell in the ray's major axis
   float inv_slope;    // 1 / (|D_x| |D_y|), general views
   int32_t axis;       // 0 general, 1 along x, 2 along y
-  int32_t pad;
+  int32_t two;        // general view whose cells at most two columns cross
   double p00m, dum, om, invm;  // axis views: minor-axis p00, du, origin and 1 / spacing
 };
 
