@@ -16,12 +16,14 @@
  * FP32 (same page, table row backend="numba", and its paragraph on segment
  * setup from the endpoint nearer the volume centre); walks that run the
  * whole volume re-derive their FP32 parameters from the FP64 set-up every 64
- * slabs.  The forward projection is deterministic.  The automatic adjoints
- * (ray scatter, sort / segment-reduce) add FP32 contributions with global
- * atomics, so their last bits depend on scheduling (the pages promise no
- * bitwise determinism for scatter accumulation, same page); the brick
- * adjoint, available through the plan, sums exactly as 32-bit fixed point
- * inside each block of the volume and is bitwise reproducible.
+ * slabs.  The forward projection is deterministic.  The ray-driven
+ * adjoints (ray scatter, sort / segment-reduce) add FP32 contributions with
+ * global atomics, so their last bits depend on scheduling (the pages promise
+ * no bitwise determinism for scatter accumulation, same page); the gather
+ * adjoint (decoupled parallel slices) sums each voxel in one thread in a
+ * fixed order, and the brick adjoint, available through the plan, sums
+ * exactly as 32-bit fixed point inside each block of the volume: both are
+ * bitwise reproducible.
  *
  * Layouts (same page, "Batch dimensions and axis spacing"):
  *   volume    float32 [nz][ny][nx], x fastest, contiguous
