@@ -1,7 +1,8 @@
 """The benchmark's bookkeeping on the CPU: on two gloo ranks every rank sees
 the slowest rank's timings and the whole-job throughput counts all ranks'
 work over that time; the digest that keys the committed DRAM-traffic
-capture ignores comments only."""
+capture ignores comments only; each plan's kernels, launch count and
+traffic model."""
 import os
 import socket
 
@@ -83,3 +84,24 @@ def test_committed_kernel_counters_match_the_sources():
     f = bench.issue_fraction("forward_rows4_kernel", 4, 3.0e12, 1965.0, 148)
     assert 0.5 < f["frac"] < 1.0 and 0.2 < f["warp_instructions_per_update"] < 0.4
     assert bench.measured_traffic("back_scatter_rows4_kernel", 4, 900) > 1e9
+
+
+def test_kernel_bookkeeping_of_each_plan():
+    """The bench names the kernels of the plan it timed, counts the library's
+    launches per step, and scales the gather adjoint's committed DRAM bytes
+    by the view count except its output volume, written once."""
+    import bench
+    gather = {"slice_rows": 4, "interleaved_slices": 1, "adjoint_variant": 4, "n_transposed_views": 450}
+    assert bench.kernel_names(gather) == ("forward_rows4_kernel", "back_gather_kernel")
+    assert bench.launches_per_step(gather) == 4        # interleave + forward, slice sums + gather
+    scatter = dict(gather, adjoint_variant=3)
+    assert bench.kernel_names(scatter) == ("forward_rows4_kernel", "back_scatter_rows4_kernel")
+    assert bench.launches_per_step(scatter) == 4       # interleave + forward, adjoint + deinterleave
+    cone = {"slice_rows": 1, "interleaved_slices": 0, "adjoint_variant": 3, "n_transposed_views": 7}
+    assert bench.kernel_names(cone) == ("forward_kernel", "back_scatter_kernel")
+    assert bench.launches_per_step(cone) == 4          # transposes on both sides
+    k = bench.kernel_counters("back_gather_kernel", 4)
+    assert k is not None and 0 < k["fixed_dram_bytes"] < k["dram_bytes"]
+    assert bench.measured_traffic("back_gather_kernel", 4, k["views"]) == k["dram_bytes"]
+    full = bench.measured_traffic("back_gather_kernel", 4, 15 * k["views"])
+    assert full == k["fixed_dram_bytes"] + 15 * (k["dram_bytes"] - k["fixed_dram_bytes"])
