@@ -83,8 +83,9 @@ enum { CTP_DET_FLAT = 0, CTP_DET_CYLINDRICAL = 1 };
  * whose rays lie in z-planes with detector rows stepping along z: one warp
  * per (x, y) cell sums chord x slice-summed sinogram over the views and the
  * crossing columns, writing every voxel once; bitwise reproducible; MBIRJAX
- * "Projector kernels", paragraph "Forward scatters, back gathers") and its
- * grid of 4 x 4-cell blocks holds at least four blocks per SM, else by
+ * "Projector kernels", paragraph "Forward scatters, back gathers"), its
+ * grid of 4 x 4-cell blocks holds at least four blocks per SM and the volume
+ * has more than 128 slices, else by
  * the collision ratio measured at create: SCATTER (one global float add per
  * ray-voxel segment, off the forward's walk) below 13.5 contributions per
  * distinct voxel of a warp batch, SORT (warp sort and segmented sum, one add

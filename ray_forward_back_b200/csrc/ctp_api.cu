@@ -641,7 +641,9 @@ ctp_status ctp_geom_create(const ctp_geom_desc *desc, ctp_geom **out) {
   }
   // Gather adjoint: decoupled slices whose views all suit it, when the plan
   // names it, or automatically once its grid fills the device (four blocks
-  // per SM; below that the scatter adjoint measured faster).
+  // per SM; below that the scatter adjoint measured faster) and the volume
+  // has more than 128 slices (at most one float4 group of slices per lane
+  // leaves the per-(cell, view) work unamortised).
   const int forced = plan ? plan->adjoint_variant : CTP_ADJOINT_AUTO;
   std::vector<ctp::GatherView> gviews;
   std::string gather_why = "the rays do not lie in z-planes with rows stepping along z";
@@ -652,8 +654,9 @@ ctp_status ctp_geom_create(const ctp_geom_desc *desc, ctp_geom **out) {
   }
   g->gather = ctp::plan_gather(vd, dm);
   const int64_t gather_blocks = (int64_t)g->gather.tiles_x * g->gather.tiles_y * g->gather.n_zchunks;
-  const bool use_gather = gather_ok && (forced == CTP_ADJOINT_GATHER ||
-                                        (forced == CTP_ADJOINT_AUTO && gather_blocks >= 4 * (int64_t)sm_count));
+  const bool use_gather =
+      gather_ok && (forced == CTP_ADJOINT_GATHER || (forced == CTP_ADJOINT_AUTO && g->gather.nz4 > 128 &&
+                                                     gather_blocks >= 4 * (int64_t)sm_count));
   if (ctp::back_brick_smem_bytes(g->back.brick) > 200 * 1024) {
     delete g;
     return fail(CTP_ERR_INVALID_ARGUMENT, "adjoint brick needs more than 200 KB of shared memory");
