@@ -60,8 +60,9 @@ def test_gather_matches_oracle(name):
 
 def test_gather_workload0_meets_the_oracle_and_the_automatic_choice():
     """Workload 0 through the gather; the automatic choice takes the gather
-    once its grid holds four blocks per SM (workload 4), the scatter below
-    that (workload 0, 256 blocks)."""
+    once its grid holds four blocks per SM and the volume has more than 128
+    slices (workload 4), the scatter otherwise (workload 0: 256 blocks, 64
+    slices)."""
     wl = W.workload(0)
     P = projector(wl.geom, {"adjoint_variant": GATHER})
     sino = wl.sinogram()
