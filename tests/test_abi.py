@@ -113,8 +113,19 @@ def test_cylindrical_needs_cone_and_orthogonal_frame(lib):
     _expect(ctp.CTP_ERR_INVALID_ARGUMENT, g)
 
 
+def test_header_constants_match_the_binding():
+    """Every enumerator of include/ctp.h has the binding's value."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    consts = dict((k, int(v)) for k, v in re.findall(r"\b(CTP_[A-Z0-9_]+)\s*=\s*(\d+)", text))
+    assert {"CTP_ADJOINT_GATHER", "CTP_ADJOINT_SCATTER", "CTP_ERR_UNSUPPORTED", "CTP_DET_CYLINDRICAL"} <= set(consts)
+    for name, value in consts.items():
+        assert getattr(ctp, name) == value, name
+
+
 def test_bad_plan(lib):
     _expect(ctp.CTP_ERR_INVALID_ARGUMENT, _cone(), {"adjoint_variant": 7})
+    _expect(ctp.CTP_ERR_INVALID_ARGUMENT, _cone(), {"adjoint_variant": 5})
+    _expect(ctp.CTP_ERR_INVALID_ARGUMENT, _cone(), {"adjoint_variant": -1})
     _expect(ctp.CTP_ERR_INVALID_ARGUMENT, _cone(), {"brick": (0, -1, 0)})
     for chunk in (-1, 3, 8):
         _expect(ctp.CTP_ERR_INVALID_ARGUMENT, _cone(), {"batch_chunk": chunk})
